@@ -1,0 +1,387 @@
+"""Throughput of the SketchSSM decode path on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--sketch-dtype bf16|f32] [--impl ours|reference]
+
+A step is one decode window of the whole hot path over the workload's batch:
+W-1 non-flush steps (ss_decode_step) and one flush (ss_flush), i.e. every
+(sequence, head) advances W tokens.  The metric is decode steps per second in
+(sequence x head) units: batch * heads * W per window / device time.
+
+Timing: each kernel launch is bracketed by CUDA events on the launching
+stream, and a 256 MiB L2-evicting write runs between launches outside the
+events, so every launch starts with a cold L2 (126 MB); the K timed windows
+are bracketed by a barrier and torch.cuda.synchronize() on both sides, and
+the time is the max over ranks.  Under torchrun every rank decodes its own
+copy of the workload (weak scaling; sequences are independent, so no data
+collective exists on this path).
+
+--impl reference times the fp64 CPU oracle on the host cores over a bounded
+sample of the same workload (the pages publish no runnable implementation).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (barrier and max over ranks only)
+# ---------------------------------------------------------------------------
+def dist_init(backend):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    rank = dist.get_rank() if world > 1 else 0
+    return rank, world
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Whole-job throughput: every rank processed units_per_rank in at most seconds_max."""
+    return units_per_rank * world / seconds_max
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def kernel_traffic_record(name):
+    """ncu-measured DRAM bytes per launch, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    src = os.path.join(ROOT, "ssm_decode_b200", "csrc", "ss_kernels.cu")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        r = rec.get(name)
+        if r and r.get("source_sha") == sha:
+            return r
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def run_ours(args, rank, world):
+    import torch
+    from ssm_decode_b200 import binding as B
+    from ssm_decode_b200 import synth
+    from ssm_decode_b200.layer import DecodeLayer
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[args.workload]
+    skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
+    W = wl.window
+    st = synth.static_inputs(wl)
+    layer = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev)
+    layer.load(st.state, st.basis, st.coef, st.A)
+    st.state = None
+    host_inputs = [synth.step_inputs(wl, st, t) for t in range(W)]
+    toks = [layer.token(x) for x in host_inputs]
+    l2 = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    units = wl.units
+
+    def window(events=None):
+        for p in range(W):
+            if events is not None:
+                l2.add_(1.0)
+                events[p][0].record(stream)
+            layer.step(toks[p])
+            if events is not None:
+                events[p][1].record(stream)
+
+    layer.prime()
+    for _ in range(args.warmup):
+        window([(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(W)])
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(W)]
+           for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    barrier(dev)
+    n0 = B.ss_launch_count()
+    with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            window(evs[k])
+        torch.cuda.synchronize()
+    barrier(dev)
+    launches = B.ss_launch_count() - n0
+    dec_t = [evs[k][p][0].elapsed_time(evs[k][p][1]) for k in range(args.steps) for p in range(W - 1)]
+    fl_t = [evs[k][W - 1][0].elapsed_time(evs[k][W - 1][1]) for k in range(args.steps)]
+    total_ms = sum(dec_t) + sum(fl_t)
+    total_ms_max = reduce_max(total_ms, dev)
+    value = weak_scaling_value(units * W * args.steps, world, total_ms_max / 1e3)
+
+    # per-kernel roofline (algorithmic bytes from the library's traffic model)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    dec_bytes = [B.ss_traffic_bytes(layer.plan, B.SS_OP_DECODE, p) for p in range(W - 1)]
+    dec_b = sum(t["read_bytes"] + t["write_bytes"] for t in dec_bytes) / max(W - 1, 1)
+    fl = B.ss_traffic_bytes(layer.plan, B.SS_OP_FLUSH)
+    fl_b = fl["read_bytes"] + fl["write_bytes"]
+    kernels = {}
+    for name, ts, nbytes in (("decode_kernel", dec_t, dec_b), ("flush_kernel", fl_t, fl_b)):
+        if not ts:
+            continue
+        avg_s = sum(ts) / len(ts) / 1e3
+        ach = nbytes / avg_s / 1e9
+        rec = kernel_traffic_record(name)
+        kernels[name] = {"launches": len(ts), "avg_us": avg_s * 1e6, "bytes_per_launch": nbytes,
+                         "achieved_gbs": ach, "frac": ach / peak, "share": sum(ts) / total_ms,
+                         "traffic": rec["dram_bytes_per_launch"] if rec else None}
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    d = kernels[dom]
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(d["achieved_gbs"], 1), "peak": peak,
+                "unit": "GB/s", "frac": round(d["frac"], 4), "traffic": d["traffic"],
+                "peak_source": f"{peak_kind} hbm_gbs"}
+
+    # baselines in the same library: Standard (exact step) and ReplaySSM, one window each
+    baselines = {}
+    for name, fn in (("standard", layer.exact_step), ("replay", layer.replay_step)):
+        ts = []
+        for _ in range(2):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(W)]
+            for p in range(W):
+                l2.add_(1.0)
+                ev[p][0].record(stream)
+                fn(toks[p])
+                ev[p][1].record(stream)
+            torch.cuda.synchronize()
+            ts.append(sum(a.elapsed_time(b) for a, b in ev))
+        t = min(ts)
+        baselines[name] = {"ms_per_window": t, "value": units * W / (t / 1e3),
+                           "sketch_speedup": (t / (total_ms / args.steps))}
+    layer.prime()
+
+    # end to end through the C ABI: pinned host inputs in, outputs back, every window
+    keys = ("q", "k", "v", "gate") + (() if wl.family == synth.MAMBA2 else ("beta",))
+    pin = [{k: torch.from_numpy(np.ascontiguousarray(x[k].view(np.int16) if x[k].dtype == np.uint16 else x[k]))
+            .pin_memory() for k in keys} for x in host_inputs]
+    host_out = torch.empty((W,) + tuple(layer.out.shape), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for x in pin for t in x.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_times = []
+    for k in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for p in range(W):
+            for key, t in pin[p].items():
+                toks[p][key].copy_(t, non_blocking=True)
+            layer.step(toks[p])
+            host_out[p].copy_(layer.out, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if k >= args.warmup:
+            e2e_times.append(a.elapsed_time(b))
+    e2e_ms = reduce_max(sum(e2e_times), dev)
+    e2e = {"value": weak_scaling_value(units * W * args.steps, world, e2e_ms / 1e3),
+           "unit": "seq*heads/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    result = {
+        "metric": "decode steps/sec (seq*heads/s), flush + sketched decode",
+        "value": value, "unit": "seq*heads/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "family": synth.FAMILY_NAMES[wl.family], "batch": wl.batch,
+                   "heads": wl.heads, "dk": wl.dk, "dv": wl.dv, "window": W, "mean_rank": wl.mean_rank,
+                   "sketch": args.sketch_dtype, "inputs": "bf16 q/k/v, fp32 state",
+                   "l2": "evicted before every launch (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roofline, "kernels": kernels, "baselines": baselines, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clk.summary(),
+    }
+    return result
+
+
+# ---------------------------------------------------------------------------
+# the oracle on host cores (cpu_baseline, and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_window_rate(wl_name, n_seq, windows=1, budget_s=None):
+    """Time the fp64 oracle decoding windows of a sample of n_seq sequences."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import sketchssm_oracle as orc
+    from ssm_decode_b200 import synth
+    wl = synth.WORKLOADS[wl_name]
+    sub = synth.shrink(wl, batch=n_seq)
+    st = synth.static_inputs(sub)
+    inputs = [synth.step_inputs(sub, st, t) for t in range(wl.window)]
+    sess = orc.Session(wl.family, st.state, wl.window, st.A, st.basis, st.coef, st.offsets,
+                       sketch_bf16=True)
+    with threadpool_limits(limits=1):
+        sess.prime()
+        times = []
+        t_start = time.perf_counter()
+        while True:
+            t0 = time.perf_counter()
+            for p in range(wl.window):
+                sess.step(inputs[p])
+            times.append(time.perf_counter() - t0)
+            if budget_s is None and len(times) >= windows:
+                break
+            if budget_s is not None and time.perf_counter() - t_start >= budget_s:
+                break
+    units = n_seq * wl.heads * wl.window
+    return units, times, wl
+
+
+def cpu_baseline(args):
+    n_seq = 4
+    units, times, wl = oracle_window_rate(args.workload, n_seq, budget_s=12.0)
+    t = sum(times) / len(times)
+    return {"value": units / t, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_seq} of {wl.batch} sequences x {wl.heads} heads, {len(times)} full windows "
+                      f"of {wl.window} steps (fp64 numpy, 1 thread)"}
+
+
+def run_reference(args):
+    n_seq = 2
+    units, times, wl = oracle_window_rate(args.workload, n_seq, windows=args.warmup + args.steps)
+    times = times[args.warmup:] or times
+    t = sum(times)
+    value = units * len(times) / t
+    return {
+        "metric": "decode steps/sec (seq*heads/s), flush + sketched decode", "impl": "reference",
+        "value": value, "unit": "seq*heads/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t / len(times) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "dk": wl.dk, "dv": wl.dv,
+                   "window": wl.window, "mean_rank": wl.mean_rank, "sketch": "bf16"},
+        "cpu_baseline": {"value": value, "unit": "seq*heads/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{n_seq} of {wl.batch} sequences x {wl.heads} heads per step "
+                                   f"(one window of {wl.window} tokens), fp64 numpy, 1 thread"},
+        "e2e": {"value": value, "unit": "seq*heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="mamba2_b320")
+    ap.add_argument("--sketch-dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    rank, world = dist_init("nccl")
+    res = run_ours(args, rank, world)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args)
+        print(json.dumps(res), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+/*
+ * sketchssm.h -- C ABI of the SketchSSM decode path on NVIDIA B200 (sm_100a).
+ *
+ * SketchSSM ("Write to the Full State, Read from a Compact Sketch", arXiv
+ * 2609.33051) keeps exact updates of a linear-attention / SSM recurrent state
+ * but, between periodic flushes, answers reads from a low-rank sketch of it:
+ *
+ *   - state update  S_t = M_t S_{t-1} + B_t, read o_t = S_t^T q_t
+ *       (SketchSSM project page, "01 / The idea", equation "Full state");
+ *   - flush, once per window of W steps: read the full state once, apply the
+ *       W buffered updates, write it back and refresh the sketch
+ *       U = S^T Omega (project page, "02 / How to Make a Sketch"; paper §4.1
+ *       and App. B as summarised on the paperlayer page);
+ *   - non-flush steps: o^ = U (C q~) + (exact term of the buffered updates),
+ *       with q~ the query mapped back through the buffered transitions
+ *       (project page, "Coefficient vector & readout"; paper §3.2, §C.1).
+ *
+ * Families (B_t = b_t k_t v_t^T in all three):
+ *   SS_MAMBA2  M_t = a_t I,                          a_t = exp(dt_t A_h), b_t = dt_t
+ *   SS_GDN     M_t = a_t (I - beta_t k_t k_t^T),      b_t = beta_t
+ *   SS_KDA     M_t = (I - beta_t k_t k_t^T) Diag(a_t), a_t in (0,1)^dk, b_t = beta_t
+ *
+ * Conventions for every entry point:
+ *   - Ownership: the caller allocates every device buffer; the library keeps
+ *     only a small host-side plan (shapes, ranks, window phase).  No call
+ *     allocates device memory or synchronises the stream.
+ *   - Pointers marked "device" must be device (or managed) addresses aligned
+ *     to 16 bytes; a misaligned pointer returns SS_ERR_ALIGNMENT.
+ *   - Launches are asynchronous on `stream` (NULL = the legacy default
+ *     stream).  A call that returns an error launches nothing and leaves the
+ *     plan unchanged.  Errors raised later by the device surface on the
+ *     caller's next CUDA synchronisation.
+ *   - No call throws, exits or aborts; every call returns an ss_status.
+ *     ss_last_error_string() describes the last failure on this thread.
+ *   - bf16 tensors are passed as their uint16_t bit patterns.
+ *
+ * Layouts (row-major, B = batch, H = heads, R = sum of ranks):
+ *   state      float    [B][H][dk][dv]        device, read/write
+ *   ring_k     uint16_t [B][H][W][dk]  bf16   device, read/write
+ *   ring_v     uint16_t [B][H][W][dv]  bf16   device, read/write
+ *   ring_gate  float    [B][H][Wg]            Mamba-2 dt / GDN a  (Wg = W rounded up to 4)
+ *              float    [B][H][W][dk]         KDA a
+ *   ring_beta  float    [B][H][Wg]            GDN/KDA beta; unused for Mamba-2 (may be NULL)
+ *   sketch     float or bf16 [B][R][dv]       row off_h + i is u_i = S^T omega_i of head h
+ *   basis      float    [R][dk]               row off_h + i is omega_i of head h (shared by the batch)
+ *   coef       float    [R][dk]               rows off_h .. off_h + r_h - 1 are head h's map C
+ *   A          float    [H]                   Mamba-2 decay rates (A_h < 0 for decay)
+ *   q, k       uint16_t [B][H][dk] bf16;  v uint16_t [B][H][dv] bf16
+ *   gate       float    [B][H] (Mamba-2 dt, GDN a) or [B][H][dk] (KDA a)
+ *   beta       float    [B][H] (GDN/KDA)
+ *   out        float    [B][H][dv]
+ *   with off_h = r_0 + ... + r_{h-1}.
+ */
+#ifndef SKETCHSSM_H
+#define SKETCHSSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-compatible with cudaStream_t / CUstream. */
+typedef struct CUstream_st* ss_stream;
+
+typedef enum {
+    SS_OK = 0,
+    SS_ERR_INVALID_ARG = 1,   /* NULL pointer, bad size, unknown enum */
+    SS_ERR_ALIGNMENT = 2,     /* a device pointer is not 16-byte aligned */
+    SS_ERR_UNSUPPORTED = 3,   /* shape outside the compiled set */
+    SS_ERR_SCHEDULE = 4,      /* call not legal at the plan's window phase */
+    SS_ERR_CUDA = 5           /* the CUDA runtime refused the launch */
+} ss_status;
+
+typedef enum { SS_MAMBA2 = 0, SS_GDN = 1, SS_KDA = 2 } ss_family;
+typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_sketch_dtype;
+
+/* Supported sizes: dk, dv in {64, 128}; 1 <= window <= 32; 1 <= heads <=
+ * SS_MAX_HEADS; batch >= 1; 0 <= ranks[h] <= dk. */
+#define SS_MAX_HEADS 512
+#define SS_MAX_WINDOW 32
+
+typedef struct {
+    int32_t family;          /* ss_family */
+    int32_t batch;           /* B: sequences decoded together */
+    int32_t heads;           /* H: state heads per sequence */
+    int32_t dk;              /* key / query dimension = state rows (Mamba-2 dstate) */
+    int32_t dv;              /* value dimension = state columns (Mamba-2 headdim) */
+    int32_t window;          /* W: steps per flush window */
+    const int32_t* ranks;    /* host [heads]: sketch rank r_h of each head; copied */
+    int32_t sketch_dtype;    /* ss_sketch_dtype of the stored sketch U */
+} ss_config;
+
+typedef struct ss_plan ss_plan;
+
+typedef struct {
+    size_t state, ring_k, ring_v, ring_gate, ring_beta, sketch, basis, coef, A;
+    size_t q, k, v, gate, beta, out;
+    int32_t total_rank;      /* R = sum of ranks */
+    int32_t gate_stride;     /* Wg (scalar-gate families) or W * dk (KDA), floats per (b, h) */
+} ss_sizes;
+
+typedef struct {
+    float* state;            /* device, see layouts */
+    uint16_t* ring_k;
+    uint16_t* ring_v;
+    float* ring_gate;
+    float* ring_beta;        /* may be NULL for Mamba-2 */
+    void* sketch;            /* NULL: no sketch is kept (ReplaySSM flushes) */
+    const float* basis;      /* needed when sketch != NULL */
+    const float* coef;       /* needed by ss_decode_step */
+    const float* A;          /* needed for Mamba-2 */
+} ss_buffers;
+
+typedef struct {
+    const uint16_t* q;       /* device bf16 [B][H][dk] */
+    const uint16_t* k;       /* device bf16 [B][H][dk] */
+    const uint16_t* v;       /* device bf16 [B][H][dv] */
+    const float* gate;       /* device [B][H] or KDA [B][H][dk] */
+    const float* beta;       /* device [B][H]; may be NULL for Mamba-2 */
+    float* out;              /* device [B][H][dv] */
+} ss_step_io;
+
+/* Operation codes for ss_traffic_bytes. */
+typedef enum {
+    SS_OP_DECODE = 0,        /* ss_decode_step at phase tau */
+    SS_OP_FLUSH = 1,         /* ss_flush with a token at phase W-1 (tau ignored) */
+    SS_OP_FLUSH_NO_TOKEN = 2,/* ss_flush(io = NULL) at phase tau */
+    SS_OP_PRIME = 3,         /* ss_prime */
+    SS_OP_EXACT = 4,         /* ss_exact_step */
+    SS_OP_REPLAY = 5,        /* ss_replay_step at phase tau */
+    SS_OP_REPLAY_FLUSH = 6   /* ss_flush with a token and sketch == NULL */
+} ss_op;
+
+typedef struct {
+    /* State-access traffic as the paper counts it (paper App. D, Table 4 as
+     * summarised on the paperlayer page): fp32 state reads and writes plus
+     * bf16 sketch + coefficient-map reads of G (dk + dv) elements per head at
+     * non-flush steps (plus G W bf16 projected erase vectors for GDN/KDA).
+     * Ring-buffer traffic and sketch/map writes are excluded, as there. */
+    double paper_read_bytes;
+    double paper_write_bytes;
+    /* Every byte this library's kernel for the call must move (inputs,
+     * ring slots, state, sketch, basis/map once per head, outputs).  This is
+     * the numerator of the HBM roofline. */
+    double read_bytes;
+    double write_bytes;
+} ss_traffic;
+
+/* Create a plan for one layer's decode.  The config (and ranks) are copied.
+ * Returns SS_ERR_INVALID_ARG / SS_ERR_UNSUPPORTED for bad shapes.  The plan
+ * starts at phase 0 with no valid sketch. */
+ss_status ss_create(const ss_config* cfg, ss_plan** out);
+ss_status ss_destroy(ss_plan* plan);
+
+/* Bytes of every buffer the caller must allocate for this plan. */
+ss_status ss_buffer_sizes(const ss_plan* plan, ss_sizes* out);
+
+/* Window phase (tokens buffered since the last flush) and whether the
+ * sketch is current.  ss_set_phase restores both, e.g. from a checkpoint of
+ * (state, ring, sketch); 0 <= phase <= W-1. */
+ss_status ss_get_phase(const ss_plan* plan, int32_t* phase, int32_t* sketch_valid);
+ss_status ss_set_phase(ss_plan* plan, int32_t phase, int32_t sketch_valid);
+
+/* U = S^T Omega from the current state with nothing buffered: a flush of
+ * zero updates (project page, "Precompute the basis outputs").  Legal at
+ * phase 0; needs bufs->sketch and bufs->basis.  Marks the sketch valid. */
+ss_status ss_prime(ss_plan* plan, const ss_buffers* bufs, ss_stream stream);
+
+/* Non-flush step (project page, "Per step · Non-flush"; paper §3.2, §C.1).
+ * Legal at phase p in 0..W-2 with a valid sketch.  Appends this token to
+ * ring slot p, then writes
+ *     out = U (C q~) + sum_{j<=p} b_j (k_j . x_j) v_j,
+ * x_p = q, x_{j-1} = M_j^T x_j, q~ = x_{-1}, without reading the state.
+ * Phase becomes p+1. */
+ss_status ss_decode_step(ss_plan* plan, const ss_buffers* bufs, const ss_step_io* io,
+                         ss_stream stream);
+
+/* Flush (paper §4.1, App. B).  With io != NULL: legal at phase W-1; the token
+ * is the window's W-th update; reads the state once, applies the W updates in
+ * order, writes the state, writes out = S_W^T q, and, if bufs->sketch !=
+ * NULL, refreshes U = S_W^T Omega (the sketch is then valid; otherwise it is
+ * marked stale).  With io == NULL: legal at any phase tau; applies the tau
+ * buffered updates, writes the state and (if bufs->sketch) the sketch; no
+ * output.  Phase becomes 0.  The ring slots are not modified. */
+ss_status ss_flush(ss_plan* plan, const ss_buffers* bufs, const ss_step_io* io,
+                   ss_stream stream);
+
+/* Standard baseline: S <- M S + B, out = S^T q, every step (paper App. D,
+ * "Standard").  Legal at phase 0; marks the sketch stale. */
+ss_status ss_exact_step(ss_plan* plan, const ss_buffers* bufs, const ss_step_io* io,
+                        ss_stream stream);
+
+/* ReplaySSM baseline non-flush step (GitHub repository page, "Overview";
+ * paper §1-§2): appends the token at slot p like ss_decode_step and writes
+ * the exact out = S0^T q~ + (buffered term), reading the full state but not
+ * writing it.  Legal at phase 0..W-2; phase becomes p+1.  Its flush is
+ * ss_flush with bufs->sketch == NULL. */
+ss_status ss_replay_step(ss_plan* plan, const ss_buffers* bufs, const ss_step_io* io,
+                         ss_stream stream);
+
+/* Traffic of one call for the whole batch (see ss_traffic).  tau = phase
+ * before the call for SS_OP_DECODE / SS_OP_REPLAY / SS_OP_FLUSH_NO_TOKEN. */
+ss_status ss_traffic_bytes(const ss_plan* plan, int32_t op, int32_t tau, ss_traffic* out);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t ss_launch_count(void);
+
+const char* ss_status_string(ss_status status);
+const char* ss_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SKETCHSSM_H */

@@ -255,8 +255,10 @@ class Session:
         self.ring.append(tok)
         qt, o_buf = effective_query(self.family, self.ring, q)
         o_hat = np.empty((self.B, self.H, self.V))
+        self.last_coefficients = []
         for h in range(self.H):
             o_hat[:, h] = sketched_output(self.U[h], self.C[h], qt[:, h], o_buf[:, h])
+            self.last_coefficients.append(np.einsum("rk,bk->br", self.C[h], qt[:, h]))
         return o_hat, read(self.S, qt) + o_buf
 
     def flush(self, inp=None, with_sketch=True):

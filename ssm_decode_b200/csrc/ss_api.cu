@@ -1,0 +1,396 @@
+// Host side of the SketchSSM C ABI (include/sketchssm.h): plans, argument
+// and schedule validation, the traffic model and kernel dispatch.  No call
+// here allocates device memory or synchronises a stream.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "ss_internal.h"
+
+namespace ss {
+int flush_smem_bytes(int family, int dk, int dv, int n, int rpad);
+int step_smem_bytes(int family, int dk, int dv, int P, int ubytes, bool replay);
+}  // namespace ss
+
+struct ss_plan {
+    ss_config cfg;
+    int32_t ranks[SS_MAX_HEADS];
+    int32_t off[SS_MAX_HEADS + 1];
+    int32_t R, rmax, Wg;
+    int32_t phase;
+    int32_t sketch_valid;
+};
+
+namespace {
+
+thread_local std::string g_err;
+std::atomic<uint64_t> g_launches{0};
+constexpr int kSmemLimit = 227 * 1024;
+
+ss_status fail(ss_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+ss_status ok() {
+    g_err.clear();
+    return SS_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+#define REQUIRE_PTR(ptr, what)                                                     \
+    do {                                                                           \
+        if ((ptr) == nullptr) return fail(SS_ERR_INVALID_ARG, "%s is NULL", what); \
+        if (!aligned16(ptr))                                                       \
+            return fail(SS_ERR_ALIGNMENT, "%s is not 16-byte aligned", what);      \
+    } while (0)
+
+#define CHECK(expr)                       \
+    do {                                  \
+        const ss_status _s = (expr);      \
+        if (_s != SS_OK) return _s;       \
+    } while (0)
+
+ss_status check_ring(const ss_plan* pl, const ss_buffers* b) {
+    REQUIRE_PTR(b->state, "bufs->state");
+    REQUIRE_PTR(b->ring_k, "bufs->ring_k");
+    REQUIRE_PTR(b->ring_v, "bufs->ring_v");
+    REQUIRE_PTR(b->ring_gate, "bufs->ring_gate");
+    if (pl->cfg.family != SS_MAMBA2) REQUIRE_PTR(b->ring_beta, "bufs->ring_beta");
+    if (pl->cfg.family == SS_MAMBA2) REQUIRE_PTR(b->A, "bufs->A");
+    return SS_OK;
+}
+
+ss_status check_io(const ss_plan* pl, const ss_step_io* io) {
+    if (io == nullptr) return fail(SS_ERR_INVALID_ARG, "io is NULL");
+    REQUIRE_PTR(io->q, "io->q");
+    REQUIRE_PTR(io->k, "io->k");
+    REQUIRE_PTR(io->v, "io->v");
+    REQUIRE_PTR(io->gate, "io->gate");
+    if (pl->cfg.family != SS_MAMBA2) REQUIRE_PTR(io->beta, "io->beta");
+    REQUIRE_PTR(io->out, "io->out");
+    return SS_OK;
+}
+
+ss::FlushParams flush_params(const ss_plan* pl, const ss_buffers* b, const ss_step_io* io) {
+    ss::FlushParams p;
+    std::memset(&p, 0, sizeof p);
+    p.state = b->state;
+    p.ring_k = b->ring_k;
+    p.ring_v = b->ring_v;
+    p.ring_gate = b->ring_gate;
+    p.ring_beta = b->ring_beta;
+    if (io) {
+        p.tok_q = io->q; p.tok_k = io->k; p.tok_v = io->v;
+        p.tok_gate = io->gate; p.tok_beta = io->beta; p.out = io->out;
+    }
+    p.sketch = b->sketch;
+    p.basis = b->basis;
+    p.A = b->A;
+    p.B = pl->cfg.batch; p.H = pl->cfg.heads; p.W = pl->cfg.window; p.Wg = pl->Wg; p.R = pl->R;
+    p.sketch_bf16 = pl->cfg.sketch_dtype == SS_BF16;
+    std::memcpy(p.off, pl->off, sizeof(int32_t) * (pl->cfg.heads + 1));
+    return p;
+}
+
+ss::StepParams step_params(const ss_plan* pl, const ss_buffers* b, const ss_step_io* io) {
+    ss::StepParams p;
+    std::memset(&p, 0, sizeof p);
+    p.state = b->state;
+    p.ring_k = b->ring_k; p.ring_v = b->ring_v; p.ring_gate = b->ring_gate; p.ring_beta = b->ring_beta;
+    p.tok_q = io->q; p.tok_k = io->k; p.tok_v = io->v; p.tok_gate = io->gate; p.tok_beta = io->beta;
+    p.sketch = b->sketch; p.coef = b->coef; p.A = b->A; p.out = io->out;
+    p.B = pl->cfg.batch; p.H = pl->cfg.heads; p.W = pl->cfg.window; p.Wg = pl->Wg; p.R = pl->R;
+    p.p = pl->phase;
+    p.sketch_bf16 = pl->cfg.sketch_dtype == SS_BF16;
+    std::memcpy(p.off, pl->off, sizeof(int32_t) * (pl->cfg.heads + 1));
+    return p;
+}
+
+ss_status launched(cudaError_t e, const char* what) {
+    if (e != cudaSuccess)
+        return fail(SS_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return SS_OK;
+}
+
+int esize(const ss_plan* pl) { return pl->cfg.sketch_dtype == SS_BF16 ? 2 : 4; }
+
+}  // namespace
+
+extern "C" {
+
+ss_status ss_create(const ss_config* cfg, ss_plan** out) {
+    if (cfg == nullptr || out == nullptr) return fail(SS_ERR_INVALID_ARG, "cfg or out is NULL");
+    *out = nullptr;
+    const ss_config& c = *cfg;
+    if (c.family < SS_MAMBA2 || c.family > SS_KDA) return fail(SS_ERR_INVALID_ARG, "unknown family %d", c.family);
+    if (c.batch < 1) return fail(SS_ERR_INVALID_ARG, "batch %d < 1", c.batch);
+    if (c.heads < 1 || c.heads > SS_MAX_HEADS)
+        return fail(SS_ERR_UNSUPPORTED, "heads %d outside 1..%d", c.heads, SS_MAX_HEADS);
+    if ((c.dk != 64 && c.dk != 128) || (c.dv != 64 && c.dv != 128))
+        return fail(SS_ERR_UNSUPPORTED, "dk=%d dv=%d: supported sizes are 64 and 128", c.dk, c.dv);
+    if (c.window < 1 || c.window > SS_MAX_WINDOW)
+        return fail(SS_ERR_UNSUPPORTED, "window %d outside 1..%d", c.window, SS_MAX_WINDOW);
+    if (c.sketch_dtype != SS_F32 && c.sketch_dtype != SS_BF16)
+        return fail(SS_ERR_INVALID_ARG, "unknown sketch dtype %d", c.sketch_dtype);
+    if (c.ranks == nullptr) return fail(SS_ERR_INVALID_ARG, "ranks is NULL");
+    if ((long long)c.batch * c.heads > (1ll << 31) / 2)
+        return fail(SS_ERR_UNSUPPORTED, "batch * heads too large");
+    ss_plan* pl = new (std::nothrow) ss_plan;
+    if (pl == nullptr) return fail(SS_ERR_INVALID_ARG, "out of host memory");
+    std::memset(pl, 0, sizeof *pl);
+    pl->cfg = c;
+    pl->cfg.ranks = nullptr;
+    pl->off[0] = 0;
+    pl->rmax = 0;
+    for (int h = 0; h < c.heads; ++h) {
+        const int r = c.ranks[h];
+        if (r < 0 || r > c.dk) {
+            delete pl;
+            return fail(SS_ERR_INVALID_ARG, "ranks[%d] = %d outside 0..dk", h, r);
+        }
+        pl->ranks[h] = r;
+        pl->off[h + 1] = pl->off[h] + r;
+        if (r > pl->rmax) pl->rmax = r;
+    }
+    pl->R = pl->off[c.heads];
+    pl->Wg = (c.window + 3) & ~3;
+    // Every launch must fit one head (flush) or one warp (decode) in shared memory.
+    const int rpad = (pl->rmax + 1 + 3) & ~3;
+    const int fl = ss::flush_smem_bytes(c.family, c.dk, c.dv, c.window, rpad);
+    const int dec = ss::step_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax * c.dv * esize(pl), false);
+    if (fl > kSmemLimit || dec > kSmemLimit) {
+        delete pl;
+        return fail(SS_ERR_UNSUPPORTED, "window %d with max rank %d needs %d / %d bytes of shared memory",
+                    c.window, pl->rmax, fl, dec);
+    }
+    *out = pl;
+    return ok();
+}
+
+ss_status ss_destroy(ss_plan* plan) {
+    delete plan;
+    return ok();
+}
+
+ss_status ss_buffer_sizes(const ss_plan* pl, ss_sizes* out) {
+    if (pl == nullptr || out == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or out is NULL");
+    const ss_config& c = pl->cfg;
+    const size_t BH = size_t(c.batch) * c.heads, K = c.dk, V = c.dv, W = c.window;
+    std::memset(out, 0, sizeof *out);
+    out->state = BH * K * V * 4;
+    out->ring_k = BH * W * K * 2;
+    out->ring_v = BH * W * V * 2;
+    out->ring_gate = (c.family == SS_KDA ? BH * W * K : BH * pl->Wg) * 4;
+    out->ring_beta = c.family == SS_MAMBA2 ? 0 : BH * pl->Wg * 4;
+    out->sketch = size_t(c.batch) * pl->R * V * esize(pl);
+    out->basis = size_t(pl->R) * K * 4;
+    out->coef = size_t(pl->R) * K * 4;
+    out->A = c.family == SS_MAMBA2 ? size_t(c.heads) * 4 : 0;
+    out->q = BH * K * 2;
+    out->k = BH * K * 2;
+    out->v = BH * V * 2;
+    out->gate = (c.family == SS_KDA ? BH * K : BH) * 4;
+    out->beta = c.family == SS_MAMBA2 ? 0 : BH * 4;
+    out->out = BH * V * 4;
+    out->total_rank = pl->R;
+    out->gate_stride = c.family == SS_KDA ? c.window * c.dk : pl->Wg;
+    return ok();
+}
+
+ss_status ss_get_phase(const ss_plan* pl, int32_t* phase, int32_t* sketch_valid) {
+    if (pl == nullptr) return fail(SS_ERR_INVALID_ARG, "plan is NULL");
+    if (phase) *phase = pl->phase;
+    if (sketch_valid) *sketch_valid = pl->sketch_valid;
+    return ok();
+}
+
+ss_status ss_set_phase(ss_plan* pl, int32_t phase, int32_t sketch_valid) {
+    if (pl == nullptr) return fail(SS_ERR_INVALID_ARG, "plan is NULL");
+    if (phase < 0 || phase > pl->cfg.window - 1)
+        return fail(SS_ERR_INVALID_ARG, "phase %d outside 0..W-1", phase);
+    pl->phase = phase;
+    pl->sketch_valid = sketch_valid ? 1 : 0;
+    return ok();
+}
+
+ss_status ss_prime(ss_plan* pl, const ss_buffers* b, ss_stream stream) {
+    if (pl == nullptr || b == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or bufs is NULL");
+    if (pl->phase != 0)
+        return fail(SS_ERR_SCHEDULE, "ss_prime needs phase 0 (phase is %d): flush first", pl->phase);
+    REQUIRE_PTR(b->state, "bufs->state");
+    REQUIRE_PTR(b->sketch, "bufs->sketch");
+    REQUIRE_PTR(b->basis, "bufs->basis");
+    ss::FlushParams p = flush_params(pl, b, nullptr);
+    p.n_ring = 0; p.has_token = 0; p.do_sketch = 1;
+    CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
+                                    reinterpret_cast<cudaStream_t>(stream)), "prime"));
+    pl->sketch_valid = 1;
+    return ok();
+}
+
+ss_status ss_decode_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_stream stream) {
+    if (pl == nullptr || b == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or bufs is NULL");
+    if (pl->phase > pl->cfg.window - 2)
+        return fail(SS_ERR_SCHEDULE, "ss_decode_step at phase %d of window %d: the next step must flush",
+                    pl->phase, pl->cfg.window);
+    if (!pl->sketch_valid)
+        return fail(SS_ERR_SCHEDULE, "ss_decode_step needs a current sketch (ss_prime or ss_flush first)");
+    CHECK(check_ring(pl, b));
+    REQUIRE_PTR(b->sketch, "bufs->sketch");
+    REQUIRE_PTR(b->coef, "bufs->coef");
+    CHECK(check_io(pl, io));
+    const ss::StepParams p = step_params(pl, b, io);
+    CHECK(launched(ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
+                                     reinterpret_cast<cudaStream_t>(stream)), "decode"));
+    pl->phase += 1;
+    return ok();
+}
+
+ss_status ss_flush(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_stream stream) {
+    if (pl == nullptr || b == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or bufs is NULL");
+    if (io != nullptr && pl->phase != pl->cfg.window - 1)
+        return fail(SS_ERR_SCHEDULE, "ss_flush with a token needs phase W-1 = %d (phase is %d)",
+                    pl->cfg.window - 1, pl->phase);
+    CHECK(check_ring(pl, b));
+    if (io != nullptr) CHECK(check_io(pl, io));
+    const bool sk = b->sketch != nullptr;
+    if (sk) {
+        REQUIRE_PTR(b->sketch, "bufs->sketch");
+        REQUIRE_PTR(b->basis, "bufs->basis");
+    }
+    ss::FlushParams p = flush_params(pl, b, io);
+    p.n_ring = pl->phase;
+    p.has_token = io != nullptr;
+    p.do_sketch = sk;
+    CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
+                                    reinterpret_cast<cudaStream_t>(stream)), "flush"));
+    pl->phase = 0;
+    pl->sketch_valid = sk;
+    return ok();
+}
+
+ss_status ss_exact_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_stream stream) {
+    if (pl == nullptr || b == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or bufs is NULL");
+    if (pl->phase != 0)
+        return fail(SS_ERR_SCHEDULE, "ss_exact_step needs phase 0 (phase is %d)", pl->phase);
+    REQUIRE_PTR(b->state, "bufs->state");
+    if (pl->cfg.family == SS_MAMBA2) REQUIRE_PTR(b->A, "bufs->A");
+    CHECK(check_io(pl, io));
+    ss::FlushParams p = flush_params(pl, b, io);
+    p.n_ring = 0; p.has_token = 1; p.do_sketch = 0;
+    CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, 0,
+                                    reinterpret_cast<cudaStream_t>(stream)), "exact"));
+    pl->sketch_valid = 0;
+    return ok();
+}
+
+ss_status ss_replay_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_stream stream) {
+    if (pl == nullptr || b == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or bufs is NULL");
+    if (pl->phase > pl->cfg.window - 2)
+        return fail(SS_ERR_SCHEDULE, "ss_replay_step at phase %d of window %d: the next step must flush",
+                    pl->phase, pl->cfg.window);
+    CHECK(check_ring(pl, b));
+    CHECK(check_io(pl, io));
+    const ss::StepParams p = step_params(pl, b, io);
+    CHECK(launched(ss::launch_replay(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p,
+                                     reinterpret_cast<cudaStream_t>(stream)), "replay"));
+    pl->phase += 1;
+    return ok();
+}
+
+ss_status ss_traffic_bytes(const ss_plan* pl, int32_t op, int32_t tau, ss_traffic* out) {
+    if (pl == nullptr || out == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or out is NULL");
+    const ss_config& c = pl->cfg;
+    const double K = c.dk, V = c.dv, W = c.window, B = c.batch, H = c.heads;
+    const double sk = esize(pl);
+    const bool m2 = c.family == SS_MAMBA2, kda = c.family == SS_KDA;
+    const double gate = kda ? 4 * K : 4, beta = m2 ? 0 : 4;
+    const double slot = 2 * K + 2 * V + gate + beta;
+    const double tok = 2 * K + slot;          // q plus the slot's fields
+    const double D = 4 * K * V;
+    const double A = m2 ? 4 * H : 0;
+    if (op == SS_OP_DECODE || op == SS_OP_REPLAY || op == SS_OP_FLUSH_NO_TOKEN) {
+        if (tau < 0 || tau > c.window - 1) return fail(SS_ERR_INVALID_ARG, "tau %d outside 0..W-1", tau);
+        if (op != SS_OP_FLUSH_NO_TOKEN && tau > c.window - 2)
+            return fail(SS_ERR_INVALID_ARG, "tau %d: a non-flush step needs tau <= W-2", tau);
+    }
+    double R = pl->R;   // sum of ranks over heads
+    double rd = 0, wr = 0, prd = 0, pwr = 0;
+    const double bh = B * H;
+    const double basis_bytes = R * K * 4;                // once per head per launch
+    const double sketch_bytes = B * R * V * sk;          // U of every sequence
+    const double paper_tg = B * R * (K + V) * 2 + (m2 ? 0 : B * R * W * 2);
+    switch (op) {
+        case SS_OP_DECODE:
+            rd = bh * (tok + tau * slot) + sketch_bytes + basis_bytes + A;
+            wr = bh * (slot + 4 * V);
+            prd = paper_tg;
+            break;
+        case SS_OP_FLUSH:
+            rd = bh * (D + (W - 1) * slot + tok) + basis_bytes + A;
+            wr = bh * (D + 4 * V) + sketch_bytes;
+            prd = bh * D; pwr = bh * D;
+            break;
+        case SS_OP_FLUSH_NO_TOKEN:
+            rd = bh * (D + tau * slot) + basis_bytes + A;
+            wr = bh * D + sketch_bytes;
+            prd = bh * D; pwr = bh * D;
+            break;
+        case SS_OP_PRIME:
+            rd = bh * D + basis_bytes;
+            wr = sketch_bytes;
+            prd = bh * D;
+            break;
+        case SS_OP_EXACT:
+            rd = bh * (D + tok) + A;
+            wr = bh * (D + 4 * V);
+            prd = bh * D; pwr = bh * D;
+            break;
+        case SS_OP_REPLAY:
+            rd = bh * (D + tok + tau * slot) + A;
+            wr = bh * (slot + 4 * V);
+            prd = bh * D;
+            break;
+        case SS_OP_REPLAY_FLUSH:
+            rd = bh * (D + (W - 1) * slot + tok) + A;
+            wr = bh * (D + 4 * V);
+            prd = bh * D; pwr = bh * D;
+            break;
+        default:
+            return fail(SS_ERR_INVALID_ARG, "unknown op %d", op);
+    }
+    out->paper_read_bytes = prd;
+    out->paper_write_bytes = pwr;
+    out->read_bytes = rd;
+    out->write_bytes = wr;
+    return ok();
+}
+
+uint64_t ss_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* ss_status_string(ss_status s) {
+    switch (s) {
+        case SS_OK: return "SS_OK";
+        case SS_ERR_INVALID_ARG: return "SS_ERR_INVALID_ARG";
+        case SS_ERR_ALIGNMENT: return "SS_ERR_ALIGNMENT";
+        case SS_ERR_UNSUPPORTED: return "SS_ERR_UNSUPPORTED";
+        case SS_ERR_SCHEDULE: return "SS_ERR_SCHEDULE";
+        case SS_ERR_CUDA: return "SS_ERR_CUDA";
+    }
+    return "unknown ss_status";
+}
+
+const char* ss_last_error_string(void) { return g_err.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal interface between the host API (ss_api.cu) and the kernels
+// (ss_kernels.cu).  Not part of the public ABI.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/sketchssm.h"
+
+namespace ss {
+
+// Parameters of the state-streaming kernel.  One launch serves ss_prime,
+// ss_flush (with or without a token), the ReplaySSM flush and ss_exact_step:
+// it applies `n_ring` buffered updates from the ring and, if `has_token`, the
+// step's own token as one more update; then it writes the state, the output
+// S^T q (if has_token) and the sketch S^T Omega (if do_sketch).
+struct FlushParams {
+    float* state;
+    const uint16_t* ring_k;
+    const uint16_t* ring_v;
+    const float* ring_gate;
+    const float* ring_beta;
+    const uint16_t* tok_q;
+    const uint16_t* tok_k;
+    const uint16_t* tok_v;
+    const float* tok_gate;
+    const float* tok_beta;
+    void* sketch;
+    const float* basis;
+    const float* A;
+    float* out;
+    int B, H, W, Wg, R;
+    int n_ring, has_token, do_sketch, sketch_bf16;
+    int off[SS_MAX_HEADS + 1];
+};
+
+// Parameters of the ring-append + windowed-read kernels (ss_decode_step and
+// ss_replay_step).  The token is appended at ring slot `p`; slots 0..p-1 are
+// the window's earlier updates.
+struct StepParams {
+    const float* state;      // replay only
+    uint16_t* ring_k;
+    uint16_t* ring_v;
+    float* ring_gate;
+    float* ring_beta;
+    const uint16_t* tok_q;
+    const uint16_t* tok_k;
+    const uint16_t* tok_v;
+    const float* tok_gate;
+    const float* tok_beta;
+    const void* sketch;      // decode only
+    const float* coef;       // decode only
+    const float* A;
+    float* out;
+    int B, H, W, Wg, R;
+    int p, sketch_bf16;
+    int off[SS_MAX_HEADS + 1];
+};
+
+// Launchers return the launch's cudaError_t (cudaSuccess when queued).
+// `rmax` is the largest per-head rank taking part in the launch.
+cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int rmax,
+                         cudaStream_t stream);
+cudaError_t launch_decode(int family, int dk, int dv, const StepParams& p, int rmax,
+                          cudaStream_t stream);
+cudaError_t launch_replay(int family, int dk, int dv, const StepParams& p,
+                          cudaStream_t stream);
+
+}  // namespace ss

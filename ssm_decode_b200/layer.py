@@ -1,0 +1,107 @@
+"""One layer's decode buffers on the device, driven through the C ABI.
+
+PyTorch only allocates device memory and supplies the stream; every step of
+the decode path runs in libsketchssm.so's kernels.  The layout of each buffer
+is the one include/sketchssm.h documents.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import binding as B
+
+
+def _dev(x, dtype, device):
+    import torch
+    if isinstance(x, np.ndarray):
+        if x.dtype == np.uint16:
+            x = x.view(np.int16)
+        x = torch.from_numpy(np.ascontiguousarray(x))
+    return x.to(device=device, dtype=dtype).contiguous()
+
+
+class DecodeLayer:
+    """Plan plus caller-owned device buffers for one linear-attention layer."""
+
+    def __init__(self, family, batch, heads, dk, dv, window, ranks, sketch_dtype=B.SS_F32,
+                 device="cuda"):
+        import torch
+        self.plan = B.Plan(family, batch, heads, dk, dv, window, ranks, sketch_dtype)
+        self.family, self.batch, self.heads, self.dk, self.dv, self.window = family, batch, heads, dk, dv, window
+        self.device = device
+        sz = B.ss_buffer_sizes(self.plan)
+        self.R = sz["total_rank"]
+        Wg = (window + 3) & ~3
+        f32, i16 = torch.float32, torch.int16
+        z = lambda *shape, dtype=f32: torch.zeros(shape, dtype=dtype, device=device)
+        self.state = z(batch, heads, dk, dv)
+        self.ring_k = z(batch, heads, window, dk, dtype=i16)
+        self.ring_v = z(batch, heads, window, dv, dtype=i16)
+        self.ring_gate = z(batch, heads, window, dk) if family == B.SS_KDA else z(batch, heads, Wg)
+        self.ring_beta = None if family == B.SS_MAMBA2 else z(batch, heads, Wg)
+        sk_dtype = torch.float32 if sketch_dtype == B.SS_F32 else torch.bfloat16
+        self.sketch = torch.zeros((batch, max(self.R, 1), dv), dtype=sk_dtype, device=device)
+        self.basis = z(max(self.R, 1), dk)
+        self.coef = z(max(self.R, 1), dk)
+        self.A = z(heads)
+        self.out = z(batch, heads, dv)
+        self.sketch_dtype = sketch_dtype
+
+    # -- data -------------------------------------------------------------------
+    def load(self, state=None, basis=None, coef=None, A=None):
+        if state is not None:
+            self.state.copy_(_dev(state, self.state.dtype, self.device))
+        if basis is not None and self.R:
+            self.basis.copy_(_dev(basis, self.basis.dtype, self.device))
+        if coef is not None and self.R:
+            self.coef.copy_(_dev(coef, self.coef.dtype, self.device))
+        if A is not None:
+            self.A.copy_(_dev(A, self.A.dtype, self.device))
+
+    def token(self, inp):
+        """Move one step's raw inputs (numpy or torch) to the device."""
+        import torch
+        t = {k: _dev(inp[k], torch.int16, self.device) for k in ("q", "k", "v")}
+        t["gate"] = _dev(inp["gate"], torch.float32, self.device)
+        t["beta"] = _dev(inp["beta"], torch.float32, self.device)
+        return t
+
+    def bufs(self, with_sketch=True):
+        return B.make_buffers(self.state, self.ring_k, self.ring_v, self.ring_gate, self.ring_beta,
+                              self.sketch if with_sketch else None, self.basis, self.coef, self.A)
+
+    def io(self, tok, out=None):
+        beta = tok["beta"] if self.family != B.SS_MAMBA2 else None
+        return B.make_step_io(tok["q"], tok["k"], tok["v"], tok["gate"], beta,
+                              self.out if out is None else out)
+
+    @property
+    def phase(self):
+        return B.ss_get_phase(self.plan)[0]
+
+    # -- calls --------------------------------------------------------------------
+    def prime(self, stream=None):
+        B.ss_prime(self.plan, self.bufs(), stream)
+
+    def decode(self, tok, out=None, stream=None):
+        B.ss_decode_step(self.plan, self.bufs(), self.io(tok, out), stream)
+
+    def flush(self, tok=None, with_sketch=True, out=None, stream=None):
+        io = None if tok is None else self.io(tok, out)
+        B.ss_flush(self.plan, self.bufs(with_sketch), io, stream)
+
+    def step(self, tok, out=None, stream=None):
+        """One SketchSSM step: non-flush until the window's last token, then flush."""
+        if self.phase == self.window - 1:
+            self.flush(tok, out=out, stream=stream)
+        else:
+            self.decode(tok, out=out, stream=stream)
+
+    def exact_step(self, tok, out=None, stream=None):
+        B.ss_exact_step(self.plan, self.bufs(False), self.io(tok, out), stream)
+
+    def replay_step(self, tok, out=None, stream=None):
+        if self.phase == self.window - 1:
+            self.flush(tok, with_sketch=False, out=out, stream=stream)
+        else:
+            B.ss_replay_step(self.plan, self.bufs(False), self.io(tok, out), stream)

@@ -1,0 +1,184 @@
+"""Shared helpers of the GPU parity tests: run the CUDA library and the fp64
+oracle side by side on the same seeded inputs and compare.
+
+Tolerances (fp32 state and arithmetic, bf16 q/k/v):
+  * outputs, states, fp32 sketches: per vector / per head,
+    max|gpu - oracle| / max|oracle| <= 1e-4;
+  * bf16 sketch: every element within one bf16 ulp of the oracle's rounded
+    sketch, and each sketched output element within
+    1e-4 max|o| + sum_i |c_i| ulp(u_i[v]) of the oracle's (the sketch
+    entries may round differently when fp32 and fp64 straddle a tie);
+  * ring buffer: bit-exact.
+"""
+import numpy as np
+
+from oracle import sketchssm_oracle as orc
+from ssm_decode_b200 import binding as B
+from ssm_decode_b200 import synth
+from ssm_decode_b200.layer import DecodeLayer
+
+TOL = 1e-4
+
+
+def vec_relerr(g, o):
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    num = np.abs(g - o).max(axis=-1)
+    den = np.maximum(np.abs(o).max(axis=-1), 1e-30)
+    return float((num / den).max())
+
+
+def head_relerr(g, o):
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    num = np.abs(g - o).max(axis=(-2, -1))
+    den = np.maximum(np.abs(o).max(axis=(-2, -1)), 1e-30)
+    return float((num / den).max())
+
+
+def bf16_ulp(x):
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    _, e = np.frexp(np.where(x > 0, x, 1.0))
+    return np.ldexp(1.0, np.maximum(e - 8, -133))
+
+
+def to_np(t):
+    import torch
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.float().numpy().astype(np.float64)
+    if t.dtype == torch.int16:
+        return t.numpy().view(np.uint16)
+    return t.numpy()
+
+
+class Pair:
+    """A DecodeLayer on the GPU and an oracle Session fed the same bytes.
+
+    ``sel`` restricts the oracle to a subset of sequences (full-size runs
+    compare sampled sequences); the GPU always runs the whole batch.
+    """
+
+    def __init__(self, wl, st=None, sketch_dtype=B.SS_F32, sel=None):
+        import torch
+        self.wl = wl
+        self.st = st if st is not None else synth.static_inputs(wl)
+        self.sel = np.arange(wl.batch) if sel is None else np.asarray(sel)
+        self.layer = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, wl.window,
+                                 self.st.ranks, sketch_dtype)
+        self.layer.load(self.st.state, self.st.basis, self.st.coef, self.st.A)
+        self.sess = orc.Session(wl.family, self.st.state[self.sel], wl.window, self.st.A,
+                                self.st.basis, self.st.coef, self.st.offsets,
+                                sketch_bf16=sketch_dtype == B.SS_BF16)
+        self.bf16 = sketch_dtype == B.SS_BF16
+        self.ring_k = np.zeros((wl.batch, wl.heads, wl.window, wl.dk), np.uint16)
+        self.ring_v = np.zeros((wl.batch, wl.heads, wl.window, wl.dv), np.uint16)
+        self.worst = {"out": 0.0, "sketched": 0.0, "state": 0.0, "sketch": 0.0}
+        torch.cuda.synchronize()
+
+    # -- checks ------------------------------------------------------------------
+    def out(self):
+        import torch
+        torch.cuda.synchronize()
+        return to_np(self.layer.out)[self.sel]
+
+    def check_state(self):
+        err = head_relerr(to_np(self.layer.state)[self.sel], self.sess.S)
+        self.worst["state"] = max(self.worst["state"], err)
+        assert err <= TOL, f"state relerr {err:.3e}"
+
+    def check_sketch(self):
+        g = to_np(self.layer.sketch)[self.sel]
+        ref = self.sess.packed_sketch()
+        if self.bf16:
+            ok = np.abs(g - ref) <= bf16_ulp(ref) * (1 + 1e-9)
+            assert ok.all(), f"{(~ok).sum()} sketch entries beyond one bf16 ulp"
+            self.worst["sketch"] = max(self.worst["sketch"], float(np.mean(g != ref)))
+        else:
+            offs = self.st.offsets
+            for h in range(self.wl.heads):
+                if offs[h + 1] == offs[h]:
+                    continue
+                err = head_relerr(g[:, offs[h]:offs[h + 1]], ref[:, offs[h]:offs[h + 1]])
+                self.worst["sketch"] = max(self.worst["sketch"], err)
+                assert err <= TOL, f"sketch head {h} relerr {err:.3e}"
+
+    def check_ring(self):
+        ph = self.layer.phase
+        gk = to_np(self.layer.ring_k)
+        gv = to_np(self.layer.ring_v)
+        assert np.array_equal(gk[:, :, :ph], self.ring_k[:, :, :ph]), "ring keys differ"
+        assert np.array_equal(gv[:, :, :ph], self.ring_v[:, :, :ph]), "ring values differ"
+
+    # -- steps -------------------------------------------------------------------------
+    def prime(self):
+        self.layer.prime()
+        self.sess.prime()
+        self.check_sketch()
+
+    def _sub(self, inp):
+        return {k: v[self.sel] for k, v in inp.items()}
+
+    def _record(self, inp, slot):
+        self.ring_k[:, :, slot] = inp["k"]
+        self.ring_v[:, :, slot] = inp["v"]
+
+    def step(self, inp, ring=True):
+        """One SketchSSM step on both sides; compare."""
+        tok = self.layer.token(inp)
+        ph = self.layer.phase
+        self.layer.step(tok)
+        g = self.out()
+        if ph == self.wl.window - 1:
+            o = self.sess.flush(self._sub(inp))
+            err = vec_relerr(g, o)
+            self.worst["out"] = max(self.worst["out"], err)
+            assert err <= TOL, f"flush output relerr {err:.3e}"
+            self.check_state()
+            self.check_sketch()
+        else:
+            o_hat, _ = self.sess.decode(self._sub(inp))
+            if self.bf16:
+                ref_u = self.sess.packed_sketch()
+                bound = TOL * np.abs(o_hat).max(-1, keepdims=True)
+                offs = self.st.offsets
+                for h in range(self.wl.heads):
+                    c = self.sess.last_coefficients[h]                       # [b, r]
+                    u = ref_u[:, offs[h]:offs[h + 1]]                        # [b, r, V]
+                    bound[:, h] = bound[:, h] + np.einsum("br,brv->bv", np.abs(c), bf16_ulp(u))
+                excess = np.abs(g - o_hat) - bound * (1 + 1e-6)
+                assert (excess <= 0).all(), f"sketched output beyond bound by {excess.max():.3e}"
+                self.worst["sketched"] = max(self.worst["sketched"], vec_relerr(g, o_hat))
+            else:
+                err = vec_relerr(g, o_hat)
+                self.worst["sketched"] = max(self.worst["sketched"], err)
+                assert err <= TOL, f"sketched output relerr {err:.3e} at phase {ph}"
+            if ring:
+                self._record(inp, ph)
+                self.check_ring()
+
+    def exact_step(self, inp):
+        tok = self.layer.token(inp)
+        self.layer.exact_step(tok)
+        g = self.out()
+        o = self.sess.exact_step(self._sub(inp))
+        err = vec_relerr(g, o)
+        self.worst["out"] = max(self.worst["out"], err)
+        assert err <= TOL, f"exact-step output relerr {err:.3e}"
+        self.check_state()
+
+    def replay_step(self, inp):
+        tok = self.layer.token(inp)
+        ph = self.layer.phase
+        self.layer.replay_step(tok)
+        g = self.out()
+        if ph == self.wl.window - 1:
+            o = self.sess.flush(self._sub(inp), with_sketch=False)
+            self.check_state()
+        else:
+            o = self.sess.replay_step(self._sub(inp))
+            self._record(inp, ph)
+            self.check_ring()
+        err = vec_relerr(g, o)
+        self.worst["out"] = max(self.worst["out"], err)
+        assert err <= TOL, f"replay output relerr {err:.3e} at phase {ph}"
