@@ -4,10 +4,10 @@ oracle side by side on the same seeded inputs and compare.
 Tolerances (fp32 state and arithmetic, bf16 q/k/v):
   * outputs, states, fp32 sketches: per vector / per head,
     max|gpu - oracle| / max|oracle| <= 1e-4;
-  * bf16 sketch: every element within one bf16 ulp of the oracle's rounded
-    sketch, and each sketched output element within
-    1e-4 max|o| + sum_i |c_i| ulp(u_i[v]) of the oracle's (the sketch
-    entries may round differently when fp32 and fp64 straddle a tie);
+  * bf16 sketch: every element within a(u) = one bf16 ulp of the oracle's
+    rounded value + 1e-4 of the head's largest sketch entry (fp32 rounding
+    and ties straddled by fp32 and fp64), and each sketched output element
+    within 1e-4 max|o| + sum_i |c_i| a(u_i[v]) of the oracle's;
   * ring buffer: bit-exact.
 """
 import numpy as np
@@ -91,8 +91,8 @@ class Pair:
         g = to_np(self.layer.sketch)[self.sel]
         ref = self.sess.packed_sketch()
         if self.bf16:
-            ok = np.abs(g - ref) <= bf16_ulp(ref) * (1 + 1e-9)
-            assert ok.all(), f"{(~ok).sum()} sketch entries beyond one bf16 ulp"
+            ok = np.abs(g - ref) <= self._sketch_allowance(ref) * (1 + 1e-9)
+            assert ok.all(), f"{(~ok).sum()} sketch entries beyond one bf16 ulp + fp32 allowance"
             self.worst["sketch"] = max(self.worst["sketch"], float(np.mean(g != ref)))
         else:
             offs = self.st.offsets
@@ -109,6 +109,18 @@ class Pair:
         gv = to_np(self.layer.ring_v)
         assert np.array_equal(gk[:, :, :ph], self.ring_k[:, :, :ph]), "ring keys differ"
         assert np.array_equal(gv[:, :, :ph], self.ring_v[:, :, :ph]), "ring values differ"
+
+    def _sketch_allowance(self, ref):
+        """One bf16 ulp of the rounded value, plus the fp32 tolerance relative to the
+        head's largest sketch entry (entries near zero come from cancelling sums whose
+        fp32 rounding error can exceed a bf16 ulp of the tiny result)."""
+        allow = bf16_ulp(ref)
+        offs = self.st.offsets
+        for h in range(self.wl.heads):
+            blk = ref[:, offs[h]:offs[h + 1]]
+            if blk.size:
+                allow[:, offs[h]:offs[h + 1]] += TOL * np.abs(blk).max(axis=(1, 2), keepdims=True)
+        return allow
 
     # -- steps -------------------------------------------------------------------------
     def prime(self):
@@ -140,12 +152,13 @@ class Pair:
             o_hat, _ = self.sess.decode(self._sub(inp))
             if self.bf16:
                 ref_u = self.sess.packed_sketch()
-                bound = TOL * np.abs(o_hat).max(-1, keepdims=True)
+                allow_u = self._sketch_allowance(ref_u)
+                bound = np.broadcast_to(TOL * np.abs(o_hat).max(-1, keepdims=True), o_hat.shape).copy()
                 offs = self.st.offsets
                 for h in range(self.wl.heads):
                     c = self.sess.last_coefficients[h]                       # [b, r]
-                    u = ref_u[:, offs[h]:offs[h + 1]]                        # [b, r, V]
-                    bound[:, h] = bound[:, h] + np.einsum("br,brv->bv", np.abs(c), bf16_ulp(u))
+                    u = allow_u[:, offs[h]:offs[h + 1]]                      # [b, r, V]
+                    bound[:, h] += np.einsum("br,brv->bv", np.abs(c), u)
                 excess = np.abs(g - o_hat) - bound * (1 + 1e-6)
                 assert (excess <= 0).all(), f"sketched output beyond bound by {excess.max():.3e}"
                 self.worst["sketched"] = max(self.worst["sketched"], vec_relerr(g, o_hat))
