@@ -8,11 +8,13 @@ W-1 non-flush steps (ss_decode_step) and one flush (ss_flush), i.e. every
 (sequence, head) advances W tokens.  The metric is decode steps per second in
 (sequence x head) units: batch * heads * W per window / device time.
 
-Timing: each kernel launch is bracketed by CUDA events on the launching
-stream, and a 256 MiB L2-evicting write runs between launches outside the
-events, so every launch starts with a cold L2 (126 MB); the K timed windows
-are bracketed by a barrier and torch.cuda.synchronize() on both sides, and
-the time is the max over ranks.  Under torchrun every rank decodes its own
+Timing: like a model's decode step, a step runs every layer of a stack of
+--layers independent layers (own state, ring, sketch; default 4), so the
+inputs of consecutive launches are far larger than L2 (126 MB) and nothing
+is re-read from L2 across launches.  Launches go back to back; each is
+bracketed by CUDA events on the launching stream for the per-kernel
+figures, and the K timed windows by a barrier and torch.cuda.synchronize()
+on both sides; the time is the max over ranks.  Under torchrun every rank decodes its own
 copy of the workload (weak scaling; sequences are independent, so no data
 collective exists on this path).
 
@@ -99,6 +101,10 @@ class ClockSampler:
                  "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return self
+        t0 = time.time()                 # nvidia-smi takes a moment to print its first sample
+        while time.time() - t0 < 10 and os.path.getsize(self.path) == 0:
+            time.sleep(0.05)
         return self
 
     def __exit__(self, *exc):
@@ -133,14 +139,23 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def kernel_source_sha():
+    """Hash of the CUDA sources, to tell whether ncu counters are still current."""
+    d = os.path.join(ROOT, "ssm_decode_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
 def kernel_traffic_record(name):
     """ncu-measured DRAM bytes per launch, if taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
-    src = os.path.join(ROOT, "ssm_decode_b200", "csrc", "ss_kernels.cu")
     try:
         with open(path) as f:
             rec = json.load(f)
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        sha = kernel_source_sha()
         r = rec.get(name)
         if r and r.get("source_sha") == sha:
             return r
@@ -168,55 +183,72 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", local)
     wl = synth.WORKLOADS[args.workload]
     skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
-    W = wl.window
+    W, NL = wl.window, args.layers
     st = synth.static_inputs(wl)
-    layer = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev)
-    layer.load(st.state, st.basis, st.coef, st.A)
+    layers = []
+    for _ in range(NL):
+        lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev)
+        lay.load(st.state, st.basis, st.coef, st.A)
+        layers.append(lay)
     st.state = None
     host_inputs = [synth.step_inputs(wl, st, t) for t in range(W)]
-    toks = [layer.token(x) for x in host_inputs]
-    l2 = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    toks = [layers[0].token(x) for x in host_inputs]
     stream = torch.cuda.current_stream()
     units = wl.units
 
-    def window(events=None):
-        for p in range(W):
-            if events is not None:
-                l2.add_(1.0)
-                events[p][0].record(stream)
-            layer.step(toks[p])
-            if events is not None:
-                events[p][1].record(stream)
+    # One decode step of a model runs every layer; so does one step here.
+    # Layer l at window position p reads token set (p + l) mod W, so a token
+    # set is re-read only NL launches later, after far more than L2 (126 MB)
+    # has streamed through.
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
 
-    layer.prime()
-    for _ in range(args.warmup):
-        window([(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(W)])
-    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(W)]
-           for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    barrier(dev)
-    n0 = B.ss_launch_count()
+    def window(events, call=lambda lay, tok: lay.step(tok)):
+        for p in range(W):
+            for l, lay in enumerate(layers):
+                e0, e1 = events[p][l]
+                e0.record(stream)
+                call(lay, toks[(p + l) % W])
+                e1.record(stream)
+
+    def new_events():
+        return [[(ev(), ev()) for _ in range(NL)] for _ in range(W)]
+
+    for lay in layers:
+        lay.prime()
+    evs = [new_events() for _ in range(args.steps)]
+    # clocks are sampled from the start of the warm-up through the timed windows
     with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
+        for _ in range(args.warmup):
+            window(new_events())
         torch.cuda.synchronize()
+        barrier(dev)
+        n0 = B.ss_launch_count()
+        t_all0, t_all1 = ev(), ev()
+        torch.cuda.synchronize()
+        t_all0.record(stream)
         for k in range(args.steps):
             window(evs[k])
+        t_all1.record(stream)
         torch.cuda.synchronize()
-    barrier(dev)
+        barrier(dev)
     launches = B.ss_launch_count() - n0
-    dec_t = [evs[k][p][0].elapsed_time(evs[k][p][1]) for k in range(args.steps) for p in range(W - 1)]
-    fl_t = [evs[k][W - 1][0].elapsed_time(evs[k][W - 1][1]) for k in range(args.steps)]
-    total_ms = sum(dec_t) + sum(fl_t)
+    dec_t = [evs[k][p][l][0].elapsed_time(evs[k][p][l][1])
+             for k in range(args.steps) for p in range(W - 1) for l in range(NL)]
+    fl_t = [evs[k][W - 1][l][0].elapsed_time(evs[k][W - 1][l][1]) for k in range(args.steps) for l in range(NL)]
+    total_ms = t_all0.elapsed_time(t_all1)
     total_ms_max = reduce_max(total_ms, dev)
-    value = weak_scaling_value(units * W * args.steps, world, total_ms_max / 1e3)
+    value = weak_scaling_value(units * W * NL * args.steps, world, total_ms_max / 1e3)
 
     # per-kernel roofline (algorithmic bytes from the library's traffic model)
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
-    dec_bytes = [B.ss_traffic_bytes(layer.plan, B.SS_OP_DECODE, p) for p in range(W - 1)]
+    plan = layers[0].plan
+    dec_bytes = [B.ss_traffic_bytes(plan, B.SS_OP_DECODE, p) for p in range(W - 1)]
     dec_b = sum(t["read_bytes"] + t["write_bytes"] for t in dec_bytes) / max(W - 1, 1)
-    fl = B.ss_traffic_bytes(layer.plan, B.SS_OP_FLUSH)
+    fl = B.ss_traffic_bytes(plan, B.SS_OP_FLUSH)
     fl_b = fl["read_bytes"] + fl["write_bytes"]
+    kernel_ms = sum(dec_t) + sum(fl_t)
     kernels = {}
     for name, ts, nbytes in (("decode_kernel", dec_t, dec_b), ("flush_kernel", fl_t, fl_b)):
         if not ts:
@@ -225,55 +257,62 @@ def run_ours(args, rank, world):
         ach = nbytes / avg_s / 1e9
         rec = kernel_traffic_record(name)
         kernels[name] = {"launches": len(ts), "avg_us": avg_s * 1e6, "bytes_per_launch": nbytes,
-                         "achieved_gbs": ach, "frac": ach / peak, "share": sum(ts) / total_ms,
+                         "achieved_gbs": ach, "frac": ach / peak, "share": sum(ts) / kernel_ms,
                          "traffic": rec["dram_bytes_per_launch"] if rec else None}
+    if W > 1:
+        kernels["decode_kernel"]["by_phase_us"] = [
+            round(sum(evs[k][p][l][0].elapsed_time(evs[k][p][l][1]) for k in range(args.steps)
+                      for l in range(NL)) / (args.steps * NL) * 1e3, 2) for p in range(W - 1)]
     dom = max(kernels, key=lambda k: kernels[k]["share"])
     d = kernels[dom]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(d["achieved_gbs"], 1), "peak": peak,
                 "unit": "GB/s", "frac": round(d["frac"], 4), "traffic": d["traffic"],
-                "peak_source": f"{peak_kind} hbm_gbs"}
+                "peak_source": f"{peak_kind} hbm_gbs (burst copy; kernels timed inside the step)"}
 
-    # baselines in the same library: Standard (exact step) and ReplaySSM, one window each
+    # baselines in the same library: Standard (exact step) and ReplaySSM
     baselines = {}
-    for name, fn in (("standard", layer.exact_step), ("replay", layer.replay_step)):
+    for name, call in (("standard", lambda lay, tok: lay.exact_step(tok)),
+                       ("replay", lambda lay, tok: lay.replay_step(tok))):
         ts = []
         for _ in range(2):
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(W)]
-            for p in range(W):
-                l2.add_(1.0)
-                ev[p][0].record(stream)
-                fn(toks[p])
-                ev[p][1].record(stream)
+            e = new_events()
+            a, b = ev(), ev()
+            a.record(stream)
+            window(e, call)
+            b.record(stream)
             torch.cuda.synchronize()
-            ts.append(sum(a.elapsed_time(b) for a, b in ev))
+            ts.append(a.elapsed_time(b) / NL)
         t = min(ts)
         baselines[name] = {"ms_per_window": t, "value": units * W / (t / 1e3),
-                           "sketch_speedup": (t / (total_ms / args.steps))}
-    layer.prime()
+                           "sketch_speedup": t / (total_ms / (args.steps * NL))}
+    for lay in layers:
+        lay.prime()
 
-    # end to end through the C ABI: pinned host inputs in, outputs back, every window
+    # end to end through the C ABI: pinned host inputs in, outputs back, every call
     keys = ("q", "k", "v", "gate") + (() if wl.family == synth.MAMBA2 else ("beta",))
     pin = [{k: torch.from_numpy(np.ascontiguousarray(x[k].view(np.int16) if x[k].dtype == np.uint16 else x[k]))
             .pin_memory() for k in keys} for x in host_inputs]
-    host_out = torch.empty((W,) + tuple(layer.out.shape), dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for x in pin for t in x.values())
+    host_out = torch.empty((W, NL) + tuple(layers[0].out.shape), dtype=torch.float32).pin_memory()
+    h2d = NL * sum(t.numel() * t.element_size() for x in pin for t in x.values())
     d2h = host_out.numel() * host_out.element_size()
     e2e_times = []
     for k in range(args.warmup + args.steps):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a, b = ev(), ev()
         torch.cuda.synchronize()
         a.record(stream)
         for p in range(W):
-            for key, t in pin[p].items():
-                toks[p][key].copy_(t, non_blocking=True)
-            layer.step(toks[p])
-            host_out[p].copy_(layer.out, non_blocking=True)
+            for l, lay in enumerate(layers):
+                tok = toks[(p + l) % W]
+                for key, t in pin[(p + l) % W].items():
+                    tok[key].copy_(t, non_blocking=True)
+                lay.step(tok)
+                host_out[p, l].copy_(lay.out, non_blocking=True)
         b.record(stream)
         torch.cuda.synchronize()
         if k >= args.warmup:
             e2e_times.append(a.elapsed_time(b))
     e2e_ms = reduce_max(sum(e2e_times), dev)
-    e2e = {"value": weak_scaling_value(units * W * args.steps, world, e2e_ms / 1e3),
+    e2e = {"value": weak_scaling_value(units * W * NL * args.steps, world, e2e_ms / 1e3),
            "unit": "seq*heads/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     result = {
@@ -283,8 +322,9 @@ def run_ours(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl.name, "family": synth.FAMILY_NAMES[wl.family], "batch": wl.batch,
                    "heads": wl.heads, "dk": wl.dk, "dv": wl.dv, "window": W, "mean_rank": wl.mean_rank,
-                   "sketch": args.sketch_dtype, "inputs": "bf16 q/k/v, fp32 state",
-                   "l2": "evicted before every launch (256 MiB write)",
+                   "layers": NL, "sketch": args.sketch_dtype, "inputs": "bf16 q/k/v, fp32 state",
+                   "step": f"one window of {W} tokens through {NL} independent layers",
+                   "l2": f"inputs larger than L2: {NL} layers rotated, back-to-back launches",
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline, "kernels": kernels, "baselines": baselines, "e2e": e2e,
         "gpu_launches": launches, "clocks": clk.summary(),
@@ -356,10 +396,11 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="mamba2_b320")
     ap.add_argument("--sketch-dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

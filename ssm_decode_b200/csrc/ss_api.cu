@@ -12,7 +12,7 @@
 
 namespace ss {
 int flush_smem_bytes(int family, int dk, int dv, int n, int rpad);
-int step_smem_bytes(int family, int dk, int dv, int P, int ubytes, bool replay);
+int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz);
 }  // namespace ss
 
 struct ss_plan {
@@ -168,7 +168,7 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
     // Every launch must fit one head (flush) or one warp (decode) in shared memory.
     const int rpad = (pl->rmax + 1 + 3) & ~3;
     const int fl = ss::flush_smem_bytes(c.family, c.dk, c.dv, c.window, rpad);
-    const int dec = ss::step_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax * c.dv * esize(pl), false);
+    const int dec = ss::decode_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax, esize(pl));
     if (fl > kSmemLimit || dec > kSmemLimit) {
         delete pl;
         return fail(SS_ERR_UNSUPPORTED, "window %d with max rank %d needs %d / %d bytes of shared memory",

@@ -1,0 +1,73 @@
+// Device helpers shared by the SketchSSM kernels (sm_100a).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ss_internal.h"
+
+namespace ss {
+
+constexpr int MAMBA2 = SS_MAMBA2, GDN = SS_GDN, KDA = SS_KDA;
+constexpr unsigned FULL = 0xffffffffu;
+// Running decay products are kept inside [2^-32, 2^32]; outside it the decay is
+// folded into the stored state (see flush_kernel).
+constexpr float GAMMA_LO = 2.3283064365386963e-10f;
+constexpr float GAMMA_HI = 4294967296.0f;
+constexpr int SMEM_LIMIT = 227 * 1024;
+
+__host__ __device__ __forceinline__ int align16(int x) { return (x + 15) & ~15; }
+
+__device__ __forceinline__ float bf2f(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+__device__ __forceinline__ float bf2f_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf2f_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ uint16_t f2bf(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+// Copy `bytes` (a multiple of 16) with `nthreads` cooperating threads.
+__device__ __forceinline__ void stage(void* dst, const void* src, int bytes, int t, int nthreads) {
+    for (int o = t * 16; o < bytes; o += nthreads * 16)
+        cp_async16(static_cast<char*>(dst) + o, static_cast<const char*>(src) + o);
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 dup2(float x) { return make_float2(x, x); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(FULL, x, m);
+    return x;
+}
+
+// Instantiate FN<family, dk, dv> for the runtime (family, dk, dv).
+#define SS_DISPATCH(FN, ...)                                                              \
+    do {                                                                                  \
+        const int key = family * 100 + (dk == 128 ? 10 : 0) + (dv == 128 ? 1 : 0);          \
+        switch (key) {                                                                    \
+            case 0: return FN<MAMBA2, 64, 64>(__VA_ARGS__);                               \
+            case 1: return FN<MAMBA2, 64, 128>(__VA_ARGS__);                              \
+            case 10: return FN<MAMBA2, 128, 64>(__VA_ARGS__);                             \
+            case 11: return FN<MAMBA2, 128, 128>(__VA_ARGS__);                            \
+            case 100: return FN<GDN, 64, 64>(__VA_ARGS__);                                \
+            case 101: return FN<GDN, 64, 128>(__VA_ARGS__);                               \
+            case 110: return FN<GDN, 128, 64>(__VA_ARGS__);                               \
+            case 111: return FN<GDN, 128, 128>(__VA_ARGS__);                              \
+            case 200: return FN<KDA, 64, 64>(__VA_ARGS__);                                \
+            case 201: return FN<KDA, 64, 128>(__VA_ARGS__);                               \
+            case 210: return FN<KDA, 128, 64>(__VA_ARGS__);                               \
+            case 211: return FN<KDA, 128, 128>(__VA_ARGS__);                              \
+            default: return cudaErrorInvalidValue;                                        \
+        }                                                                                 \
+    } while (0)
+
+}  // namespace ss

@@ -1,0 +1,522 @@
+// flush_kernel: the state-streaming kernel of the SketchSSM decode path.
+//
+// For every (sequence, head) it reads the fp32 dk x dv state once, applies
+// the window's buffered updates (ring slots, then the step's own token) in
+// order, writes the state back and, fused into the same pass over the
+// registers, computes the exact output S^T q and the sketch U = S^T Omega
+// (paper §4.1 and App. B as summarised on the paperlayer page: one full-state
+// read per window refreshes the sketch, whose construction is fused into the
+// update kernel; project page "02 / How to Make a Sketch", u_i = S^T omega_i).
+// One launch serves ss_prime (zero updates), ss_flush with or without a
+// token, the ReplaySSM flush (no sketch) and the Standard step (one update).
+//
+// Work split.  The kernel is persistent: CTA c walks heads c, c + gridDim.x,
+// ...  A head is held by 2*dv threads, dv/4 column groups x 8 row blocks;
+// each thread keeps a (dk/8) x 4 tile as fp32 pairs of adjacent columns, so
+// tile loads/stores are 16-byte accesses and every update is a packed
+// fp32x2 FMA.  While a head is computed from registers, cp.async brings the
+// next head's state tile and window into shared memory.
+//
+// Scaled state.  Write Gamma_j for the product of the decays since the last
+// fold (a scalar for Mamba-2 and GDN, a dk-vector for KDA) and keep
+// S' = Diag(Gamma_j)^-1 S.  Then, with M_j and B_j = b_j k_j v_j^T:
+//     w_j = S'^T (Gamma_j ⊙ k_j)                   (delta rule only)
+//     d_j = b_j (v_j - w_j)                        (Mamba-2: d_j = b_j v_j)
+//     S'  <- S' + (k_j ⊘ Gamma_j) d_j^T
+// which is one FMA per state element for the write and one for the delta
+// rule's read; the decays cost nothing per element.  Scalar decays are folded
+// into the per-update coefficients instead of the keys.  When a running
+// product leaves [2^-32, 2^32] the decay is folded into S' (one multiply per
+// element) and the product restarts at 1; a zero decay is applied exactly so.
+#include "ss_common.cuh"
+
+namespace ss {
+namespace {
+
+// Floats of a duplicated, row-block-padded K-vector: 8 row blocks of dk/8
+// channels stored as (x, x) pairs, plus 4 floats of padding per block so the
+// row blocks a warp reads together fall in different banks.
+__host__ __device__ constexpr int kd_len(int K) { return 8 * (2 * (K / 8) + 4); }
+
+template <int K, int V>
+struct FS {
+    static constexpr int T = 2 * V;             // threads per CTA
+    static constexpr int R = K / 8;             // state rows per thread
+    static constexpr int KB = 2 * R + 4;        // floats per row block of a duplicated K-vector
+    static constexpr int KD = kd_len(K);
+};
+
+// Per-CTA shared-memory layout (byte offsets).  [tile .. ts] is written by
+// the prefetch of the next head; the rest is the current head's working set.
+struct FlushLayout {
+    int tile, kraw, vraw, graw, sg, sb, tq, ts, braw;
+    int kd, ku, fin, sc, pt, meta, total;
+};
+
+__host__ __device__ inline FlushLayout flush_layout(int fam, int K, int V, int n, int rpad) {
+    const int KD = kd_len(K);
+    FlushLayout L;
+    int o = 0;
+    L.tile = o; o += align16(K * V * 4);
+    L.kraw = o; o += align16(n * K * 2);
+    L.vraw = o; o += align16(n * V * 2);
+    L.graw = o; o += align16(fam == KDA ? n * K * 4 : 0);
+    L.sg = o;   o += align16(SS_MAX_WINDOW * 4);
+    L.sb = o;   o += align16(SS_MAX_WINDOW * 4);
+    L.tq = o;   o += align16(K * 2);
+    L.ts = o;   o += 16;
+    L.braw = o; o += align16(rpad * K * 4);
+    L.kd = o;   o += align16(n * KD * 4);
+    L.ku = o;   o += align16(fam == KDA ? n * KD * 4 : 0);
+    L.fin = o;  o += align16(fam == KDA ? KD * 4 : 0);
+    L.sc = o;   o += align16((n + 1) * 16);
+    L.pt = o;   o += align16(rpad * K * 4);
+    L.meta = o; o += 16;
+    L.total = o;
+    return L;
+}
+
+// Index of channel c's duplicated pair in a row-block-padded K-vector.
+template <int K>
+__device__ __forceinline__ int kdup(int c) {
+    constexpr int R = K / 8;
+    return (c / R) * (2 * R + 4) + (c % R) * 2;
+}
+
+template <int K, int V>
+__device__ __forceinline__ void prefetch_tile(const FlushParams& p, long long u, float* tile, int t) {
+    stage(tile, p.state + u * (long long)(K * V), K * V * 4, t, FS<K, V>::T);
+}
+
+template <int FAM, int K, int V>
+__device__ __forceinline__ void prefetch_window(const FlushParams& p, long long u, unsigned char* sh,
+                                                const FlushLayout& L, int t) {
+    constexpr int T = FS<K, V>::T;
+    const long long ring_row = u * p.W;
+    stage(sh + L.kraw, p.ring_k + ring_row * K, p.n_ring * K * 2, t, T);
+    stage(sh + L.vraw, p.ring_v + ring_row * V, p.n_ring * V * 2, t, T);
+    if (FAM == KDA) stage(sh + L.graw, p.ring_gate + ring_row * K, p.n_ring * K * 4, t, T);
+    const int n4 = (p.n_ring + 3) & ~3;
+    if (FAM != KDA) stage(sh + L.sg, p.ring_gate + u * p.Wg, n4 * 4, t, T);
+    if (FAM != MAMBA2) stage(sh + L.sb, p.ring_beta + u * p.Wg, n4 * 4, t, T);
+    if (p.has_token) {
+        stage(sh + L.kraw + p.n_ring * K * 2, p.tok_k + u * K, K * 2, t, T);
+        stage(sh + L.vraw + p.n_ring * V * 2, p.tok_v + u * V, V * 2, t, T);
+        if (FAM == KDA) stage(sh + L.graw + p.n_ring * K * 4, p.tok_gate + u * K, K * 4, t, T);
+        stage(sh + L.tq, p.tok_q + u * K, K * 2, t, T);
+        if (t == 0 && FAM != KDA) cp_async4(sh + L.ts, p.tok_gate + u);
+        if (t == 1 && FAM != MAMBA2) cp_async4(sh + L.ts + 4, p.tok_beta + u);
+    }
+    if (p.do_sketch) {
+        const int h = int(u % p.H);
+        stage(sh + L.braw, p.basis + (long long)p.off[h] * K, (p.off[h + 1] - p.off[h]) * K * 4, t, T);
+    }
+}
+
+// Sequential decay scan with folds, one warp, channels lane + 32 m
+// (the slow path; used when some running product leaves the range).
+template <int FAM, int K>
+__device__ void scan_with_folds(int n, int n_ring, const float* al_in, const float* bl_in,
+                                const uint16_t* kraw, const float* graw, float* kd, float* ku,
+                                float* fin, float4* sc, unsigned* meta, int lane) {
+    constexpr int CPL = K / 32;
+    float gam[CPL];
+#pragma unroll
+    for (int m = 0; m < CPL; ++m) gam[m] = 1.f;
+    unsigned mask = 0;
+    for (int j = 0; j < n; ++j) {
+        const float bj = bl_in[j];
+        float g[CPL];
+        bool need = false;
+#pragma unroll
+        for (int m = 0; m < CPL; ++m) {
+            const float a = (FAM == KDA) ? graw[j * K + lane + 32 * m] : al_in[j];
+            g[m] = gam[m] * a;
+            need |= !(g[m] >= GAMMA_LO && g[m] <= GAMMA_HI);
+        }
+        const bool fold = __any_sync(FULL, need);
+        if (FAM == KDA) {
+#pragma unroll
+            for (int m = 0; m < CPL; ++m) {
+                const int c = lane + 32 * m;
+                const float kv = bf2f(kraw[j * K + c]);
+                float2* kdp = reinterpret_cast<float2*>(kd + j * kd_len(K) + kdup<K>(c));
+                float2* kup = reinterpret_cast<float2*>(ku + j * kd_len(K) + kdup<K>(c));
+                if (fold) {            // ku carries the fold vector; Gamma_j = 1
+                    *kup = dup2(g[m]);
+                    *kdp = dup2(kv);
+                    gam[m] = 1.f;
+                } else {
+                    gam[m] = g[m];
+                    *kdp = dup2(g[m] * kv);
+                    *kup = dup2(kv * __frcp_rn(g[m]));
+                }
+            }
+            if (lane == 0) sc[j] = make_float4(bj, 1.f, 0.f, 0.f);
+        } else {
+            float rs = 1.f;
+            if (fold) { rs = g[0]; gam[0] = 1.f; }
+            else gam[0] = g[0];
+            if (lane == 0) sc[j] = make_float4(bj * __frcp_rn(gam[0]), gam[0], rs, 0.f);
+        }
+        if (fold) mask |= 1u << j;
+    }
+    if (FAM == KDA) {
+#pragma unroll
+        for (int m = 0; m < CPL; ++m)
+            *reinterpret_cast<float2*>(fin + kdup<K>(lane + 32 * m)) = dup2(gam[m]);
+    } else if (lane == 0) {
+        sc[n] = make_float4(gam[0], 0.f, 0.f, 0.f);
+    }
+    if (lane == 0) meta[0] = mask;
+}
+
+template <int FAM, int K, int V>
+__global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __grid_constant__ FlushParams p, int rpad) {
+    using S = FS<K, V>;
+    constexpr int R = S::R, KB = S::KB, KD = S::KD;
+    extern __shared__ __align__(16) unsigned char smem[];
+
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int cgw = lane & 3, rb = lane >> 2;
+    const int c0 = warp * 16 + cgw * 4;          // first of this thread's 4 columns
+    const int row0 = rb * R;                     // first of this thread's R rows
+    const long long units = (long long)p.B * p.H;
+    const int n = p.n_ring + p.has_token;
+    const FlushLayout L = flush_layout(FAM, K, V, n, rpad);
+    float* tile = reinterpret_cast<float*>(smem + L.tile);
+    const uint16_t* kraw = reinterpret_cast<const uint16_t*>(smem + L.kraw);
+    const uint16_t* vraw = reinterpret_cast<const uint16_t*>(smem + L.vraw);
+    const float* graw = reinterpret_cast<const float*>(smem + L.graw);
+    const float* sg = reinterpret_cast<const float*>(smem + L.sg);
+    const float* sb = reinterpret_cast<const float*>(smem + L.sb);
+    const uint16_t* tq = reinterpret_cast<const uint16_t*>(smem + L.tq);
+    const float* ts = reinterpret_cast<const float*>(smem + L.ts);
+    float* kd = reinterpret_cast<float*>(smem + L.kd);
+    float* ku = reinterpret_cast<float*>(smem + L.ku);
+    float* fin = reinterpret_cast<float*>(smem + L.fin);
+    float4* sc = reinterpret_cast<float4*>(smem + L.sc);
+    float* pt = reinterpret_cast<float*>(smem + L.pt);
+    const float* braw = reinterpret_cast<const float*>(smem + L.braw);
+    unsigned* meta = reinterpret_cast<unsigned*>(smem + L.meta);
+
+    long long u = blockIdx.x;
+    if (u < units) {
+        prefetch_tile<K, V>(p, u, tile, t);
+        prefetch_window<FAM, K, V>(p, u, smem, L, t);
+    }
+    cp_async_commit();
+
+    for (; u < units; u += gridDim.x) {
+        cp_async_wait_all();
+        __syncthreads();                                              // (A) head u staged
+        const int h = int(u % p.H);
+        const long long b = u / p.H;
+        const long long un = u + gridDim.x;
+
+        // 1. This thread's tile, pairs of adjacent columns.
+        float2 s[R][2];
+        {
+            const float* tb = tile + row0 * V + c0;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const float4 a = *reinterpret_cast<const float4*>(tb + i * V);
+                s[i][0] = make_float2(a.x, a.y);
+                s[i][1] = make_float2(a.z, a.w);
+            }
+        }
+
+        // 2. Per-head preparation: keys, decays, coefficients, extended basis.
+        const int r_h = p.do_sketch ? p.off[h + 1] - p.off[h] : 0;
+        const int next = r_h + p.has_token;                           // columns of [Omega_h | q]
+        const int nch = (next + 3) / 4;
+        bool bad = false;
+        if (t < K) {                                                  // one channel per thread
+            const int c = t;
+            const int pc = kdup<K>(c);
+            if (FAM == KDA) {
+                float gam = 1.f;
+                for (int j = 0; j < n; ++j) {
+                    const float g = gam * graw[j * K + c];
+                    bad |= !(g >= GAMMA_LO && g <= GAMMA_HI);
+                    gam = g;
+                    const float kv = bf2f(kraw[j * K + c]);
+                    *reinterpret_cast<float2*>(kd + j * KD + pc) = dup2(g * kv);
+                    *reinterpret_cast<float2*>(ku + j * KD + pc) = dup2(kv * __frcp_rn(g));
+                }
+                *reinterpret_cast<float2*>(fin + pc) = dup2(gam);
+            } else {
+#pragma unroll 4
+                for (int j = 0; j < n; ++j)
+                    *reinterpret_cast<float2*>(kd + j * KD + pc) = dup2(bf2f(kraw[j * K + c]));
+            }
+        }
+        // extended basis [Omega_h | q | 0 ...] rows, dk floats each
+        for (int idx = t * 4; idx < nch * 4 * K; idx += 2 * V * 4) {
+            const int e = idx / K, c = idx % K;
+            float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (e < r_h) {
+                val = *reinterpret_cast<const float4*>(braw + e * K + c);
+            } else if (e == r_h && p.has_token) {
+                const uint2 w = *reinterpret_cast<const uint2*>(tq + c);
+                val = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
+            }
+            *reinterpret_cast<float4*>(pt + e * K + c) = val;
+        }
+        if (FAM != KDA && warp == 0) {
+            // scalar decays: lane j holds (a_j, b_j); running products by a
+            // log-step scan; folds only if a product leaves the range.
+            float al = 1.f, bl = 0.f;
+            if (lane < n) {
+                const bool tok = lane >= p.n_ring;
+                const float g = tok ? ts[0] : sg[lane];
+                if (FAM == MAMBA2) { bl = g; al = expf(g * p.A[h]); }
+                else { al = g; bl = tok ? ts[1] : sb[lane]; }
+            }
+            float G = al;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const float y = __shfl_up_sync(FULL, G, m);
+                if (lane >= m) G *= y;
+            }
+            const bool out = lane < n && !(G >= GAMMA_LO && G <= GAMMA_HI);
+            if (!__any_sync(FULL, out)) {
+                if (lane < n) sc[lane] = make_float4(bl * __frcp_rn(G), G, 1.f, 0.f);
+                const float Gn = __shfl_sync(FULL, G, n > 0 ? n - 1 : 0);
+                if (lane == 0) { sc[n] = make_float4(n > 0 ? Gn : 1.f, 0.f, 0.f, 0.f); meta[0] = 0u; }
+            } else {
+                __shared__ float al_s[SS_MAX_WINDOW], bl_s[SS_MAX_WINDOW];
+                al_s[lane] = al;
+                bl_s[lane] = bl;
+                __syncwarp();
+                scan_with_folds<FAM, K>(n, p.n_ring, al_s, bl_s, kraw, graw, kd, ku, fin, sc, meta, lane);
+            }
+        }
+        if (FAM == KDA) {
+            const int any_bad = __syncthreads_or(bad);
+            if (warp == 0 && lane < n) {
+                const float bl = lane >= p.n_ring ? ts[1] : sb[lane];
+                if (!any_bad) sc[lane] = make_float4(bl, 1.f, 0.f, 0.f);
+            }
+            if (any_bad && warp == 0) {
+                __shared__ float bl_s[SS_MAX_WINDOW];
+                bl_s[lane] = lane < n ? (lane >= p.n_ring ? ts[1] : sb[lane]) : 0.f;
+                __syncwarp();
+                scan_with_folds<FAM, K>(n, p.n_ring, nullptr, bl_s, kraw, graw, kd, ku, fin, sc, meta, lane);
+            } else if (warp == 0 && lane == 0) {
+                meta[0] = 0u;
+            }
+        }
+        __syncthreads();                                              // (B)
+
+        // 3. The tile buffer is free: start the next head's state.
+        if (un < units) prefetch_tile<K, V>(p, un, tile, t);
+        cp_async_commit();
+
+        // 4. Apply the updates.
+        const unsigned mask = meta[0];
+        const float* kdb = kd + rb * KB;
+        const float* kub = ku + rb * KB;
+        for (int j = 0; j < n; ++j) {
+            const float4 scj = sc[j];
+            const bool fold = (mask >> j) & 1u;
+            if (fold) {
+                if (FAM == KDA) {
+#pragma unroll
+                    for (int i = 0; i < R; i += 2) {
+                        const float4 f = *reinterpret_cast<const float4*>(kub + j * KD + 2 * i);
+#pragma unroll
+                        for (int cp = 0; cp < 2; ++cp) {
+                            s[i][cp] = fmul2(s[i][cp], make_float2(f.x, f.y));
+                            s[i + 1][cp] = fmul2(s[i + 1][cp], make_float2(f.z, f.w));
+                        }
+                    }
+                } else {
+                    const float2 f = dup2(scj.z);
+#pragma unroll
+                    for (int i = 0; i < R; ++i)
+#pragma unroll
+                        for (int cp = 0; cp < 2; ++cp) s[i][cp] = fmul2(s[i][cp], f);
+                }
+            }
+            float2 kv[R];
+#pragma unroll
+            for (int i = 0; i < R; i += 2) {
+                const float4 f = *reinterpret_cast<const float4*>(kdb + j * KD + 2 * i);
+                kv[i] = make_float2(f.x, f.y);
+                kv[i + 1] = make_float2(f.z, f.w);
+            }
+            float2 w2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            if (FAM != MAMBA2) {
+#pragma unroll
+                for (int i = 0; i < R; ++i)
+#pragma unroll
+                    for (int cp = 0; cp < 2; ++cp) w2[cp] = ffma2(kv[i], s[i][cp], w2[cp]);
+#pragma unroll
+                for (int cp = 0; cp < 2; ++cp)
+#pragma unroll
+                    for (int m = 4; m <= 16; m <<= 1) {
+                        w2[cp].x += __shfl_xor_sync(FULL, w2[cp].x, m);
+                        w2[cp].y += __shfl_xor_sync(FULL, w2[cp].y, m);
+                    }
+            }
+            const uint2 vv = *reinterpret_cast<const uint2*>(vraw + j * V + c0);
+            const float2 v01 = make_float2(bf2f_lo(vv.x), bf2f_hi(vv.x));
+            const float2 v23 = make_float2(bf2f_lo(vv.y), bf2f_hi(vv.y));
+            float2 d2[2];
+            if (FAM == MAMBA2) {
+                d2[0] = fmul2(dup2(scj.x), v01);
+                d2[1] = fmul2(dup2(scj.x), v23);
+            } else {
+                const float2 ncw = dup2(FAM == GDN ? -scj.y : -1.f);
+                d2[0] = fmul2(dup2(scj.x), ffma2(ncw, w2[0], v01));
+                d2[1] = fmul2(dup2(scj.x), ffma2(ncw, w2[1], v23));
+            }
+            if (FAM == KDA && !fold) {
+#pragma unroll
+                for (int i = 0; i < R; i += 2) {
+                    const float4 f = *reinterpret_cast<const float4*>(kub + j * KD + 2 * i);
+                    kv[i] = make_float2(f.x, f.y);
+                    kv[i + 1] = make_float2(f.z, f.w);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < R; ++i)
+#pragma unroll
+                for (int cp = 0; cp < 2; ++cp) s[i][cp] = ffma2(kv[i], d2[cp], s[i][cp]);
+        }
+        __syncthreads();                                              // (C) window buffers read
+
+        // 5. The window buffers are free: start the next head's window.
+        if (un < units) prefetch_window<FAM, K, V>(p, un, smem, L, t);
+        cp_async_commit();
+
+        // 6. True state S = Diag(Gamma) S', written back.
+        if (FAM == KDA) {
+            const float* g = fin + rb * KB;
+#pragma unroll
+            for (int i = 0; i < R; i += 2) {
+                const float4 f = *reinterpret_cast<const float4*>(g + 2 * i);
+#pragma unroll
+                for (int cp = 0; cp < 2; ++cp) {
+                    s[i][cp] = fmul2(s[i][cp], make_float2(f.x, f.y));
+                    s[i + 1][cp] = fmul2(s[i + 1][cp], make_float2(f.z, f.w));
+                }
+            }
+        } else {
+            const float2 f = dup2(sc[n].x);
+#pragma unroll
+            for (int i = 0; i < R; ++i)
+#pragma unroll
+                for (int cp = 0; cp < 2; ++cp) s[i][cp] = fmul2(s[i][cp], f);
+        }
+        float* st = p.state + u * (long long)(K * V) + row0 * V + c0;
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+            __stcs(reinterpret_cast<float4*>(st + i * V), make_float4(s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y));
+
+        // 7. Fused read-out against [Omega_h | q], 4 basis columns per pass; a
+        //    3-level reduce-scatter over the row blocks leaves row block
+        //    (b2 b1 b0) with basis column 4 ch + 2 b2 + b1 for the state
+        //    columns c0 + 2 b0, c0 + 2 b0 + 1.
+        const int hb2 = (rb >> 2) & 1, hb1 = (rb >> 1) & 1, hb0 = rb & 1;
+        for (int ch = 0; ch < nch; ++ch) {
+            float2 acc[4][2];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[e][0] = acc[e][1] = make_float2(0.f, 0.f);
+                const float* prow = pt + (ch * 4 + e) * K + row0;
+#pragma unroll
+                for (int i = 0; i < R; i += 4) {
+                    const float4 pv = *reinterpret_cast<const float4*>(prow + i);
+                    const float pe[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                        for (int cp = 0; cp < 2; ++cp) acc[e][cp] = ffma2(dup2(pe[ii]), s[i + ii][cp], acc[e][cp]);
+                }
+            }
+            float v8[2][4];                      // level 1 (lane bit 4 = rb bit 2): basis columns {0,1} | {2,3}
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float2 lo0 = acc[e][0], lo1 = acc[e][1], hi0 = acc[e + 2][0], hi1 = acc[e + 2][1];
+                const float mine[4] = {hb2 ? hi0.x : lo0.x, hb2 ? hi0.y : lo0.y, hb2 ? hi1.x : lo1.x, hb2 ? hi1.y : lo1.y};
+                const float give[4] = {hb2 ? lo0.x : hi0.x, hb2 ? lo0.y : hi0.y, hb2 ? lo1.x : hi1.x, hb2 ? lo1.y : hi1.y};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) v8[e][c] = mine[c] + __shfl_xor_sync(FULL, give[c], 16);
+            }
+            float v4[4];                         // level 2 (lane bit 3 = rb bit 1)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float send = hb1 ? v8[0][c] : v8[1][c];
+                const float keep = hb1 ? v8[1][c] : v8[0][c];
+                v4[c] = keep + __shfl_xor_sync(FULL, send, 8);
+            }
+            float v2[2];                         // level 3 (lane bit 2 = rb bit 0): state columns
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const float send = hb0 ? v4[c] : v4[c + 2];
+                const float keep = hb0 ? v4[c + 2] : v4[c];
+                v2[c] = keep + __shfl_xor_sync(FULL, send, 4);
+            }
+            const int e = ch * 4 + hb2 * 2 + hb1;
+            const int col = c0 + hb0 * 2;
+            if (e < r_h) {
+                const long long row = b * p.R + p.off[h] + e;
+                if (p.sketch_bf16) {
+                    *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.sketch) + row * V + col) =
+                        uint32_t(f2bf(v2[0])) | (uint32_t(f2bf(v2[1])) << 16);
+                } else {
+                    *reinterpret_cast<float2*>(static_cast<float*>(p.sketch) + row * V + col) =
+                        make_float2(v2[0], v2[1]);
+                }
+            } else if (e == r_h && p.has_token) {
+                *reinterpret_cast<float2*>(p.out + u * V + col) = make_float2(v2[0], v2[1]);
+            }
+        }
+    }
+    cp_async_wait_all();
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+template <int FAM, int K, int V>
+cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
+    const int n = p.n_ring + p.has_token;
+    const int rpad = ((p.do_sketch ? rmax : 0) + p.has_token + 3) & ~3;
+    const int bytes = flush_layout(FAM, K, V, n, rpad).total;
+    if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
+    auto kern = flush_kernel<FAM, K, V>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, FS<K, V>::T, bytes);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    const long long units = (long long)p.B * p.H;
+    const long long cap = (long long)per_sm * sm_count();
+    const long long grid = units < cap ? units : cap;
+    kern<<<dim3(unsigned(grid)), dim3(FS<K, V>::T), bytes, stream>>>(p, rpad);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream) {
+    SS_DISPATCH(flush_t, p, rmax, stream);
+}
+
+int flush_smem_bytes(int family, int dk, int dv, int n, int rpad) {
+    return flush_layout(family, dk, dv, n, rpad).total;
+}
+
+}  // namespace ss
