@@ -81,6 +81,12 @@ typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_sketch_dtype;
 #define SS_MAX_HEADS 512
 #define SS_MAX_WINDOW 32
 
+/* Bits a kernel ORs into ss_buffers.status (a device word the caller owns
+ * and clears).  Kernels that wait for their own bulk copies bound each wait
+ * to about one second; if a wait runs out the kernel sets SS_DEVICE_TIMEOUT
+ * and returns without completing its outputs. */
+#define SS_DEVICE_TIMEOUT 1
+
 typedef struct {
     int32_t family;          /* ss_family */
     int32_t batch;           /* B: sequences decoded together */
@@ -111,6 +117,7 @@ typedef struct {
     const float* basis;      /* needed when sketch != NULL */
     const float* coef;       /* needed by ss_decode_step */
     const float* A;          /* needed for Mamba-2 */
+    int32_t* status;         /* optional device int32 (4-byte aligned), see SS_DEVICE_TIMEOUT; NULL: no report */
 } ss_buffers;
 
 typedef struct {
@@ -206,6 +213,14 @@ ss_status ss_traffic_bytes(const ss_plan* plan, int32_t op, int32_t tau, ss_traf
 
 /* Number of kernels this library has launched in this process. */
 uint64_t ss_launch_count(void);
+
+/* Testing hook.  With stall != 0 the next ss_decode_step or ss_replay_step of
+ * this plan makes one CTA expect more bytes than its bulk copies deliver, so
+ * that CTA's bounded wait runs out after about a second: it sets
+ * SS_DEVICE_TIMEOUT in bufs->status and returns, leaving its outputs
+ * incomplete; the rest of the launch completes.  The hook clears itself
+ * after that call.  Used to test the timeout path without a device fault. */
+ss_status ss_debug_stall_next_copy(ss_plan* plan, int32_t stall);
 
 const char* ss_status_string(ss_status status);
 const char* ss_last_error_string(void);

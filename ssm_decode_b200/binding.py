@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(HERE, "libsketchssm.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "sketchssm.h")
 
 SS_OK, SS_ERR_INVALID_ARG, SS_ERR_ALIGNMENT, SS_ERR_UNSUPPORTED, SS_ERR_SCHEDULE, SS_ERR_CUDA = range(6)
+SS_DEVICE_TIMEOUT = 1
 SS_MAMBA2, SS_GDN, SS_KDA = 0, 1, 2
 SS_F32, SS_BF16 = 0, 1
 (SS_OP_DECODE, SS_OP_FLUSH, SS_OP_FLUSH_NO_TOKEN, SS_OP_PRIME, SS_OP_EXACT, SS_OP_REPLAY,
@@ -37,7 +38,8 @@ class ss_sizes(ctypes.Structure):
 
 class ss_buffers(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("state", "ring_k", "ring_v", "ring_gate", "ring_beta", "sketch", "basis", "coef", "A")]
+                ("state", "ring_k", "ring_v", "ring_gate", "ring_beta", "sketch", "basis", "coef", "A",
+                 "status")]
 
 
 class ss_step_io(ctypes.Structure):
@@ -79,6 +81,7 @@ def lib():
             "ss_replay_step": ([P, ctypes.POINTER(ss_buffers), ctypes.POINTER(ss_step_io), P], S),
             "ss_traffic_bytes": ([P, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ss_traffic)], S),
             "ss_launch_count": ([], ctypes.c_uint64),
+            "ss_debug_stall_next_copy": ([P, ctypes.c_int32], S),
             "ss_status_string": ([S], ctypes.c_char_p),
             "ss_last_error_string": ([], ctypes.c_char_p),
         }
@@ -133,13 +136,15 @@ def _dt():
 
 
 def make_buffers(state=None, ring_k=None, ring_v=None, ring_gate=None, ring_beta=None, sketch=None,
-                 basis=None, coef=None, A=None):
+                 basis=None, coef=None, A=None, status=None):
+    import torch
     d = _dt()
     return ss_buffers(_ptr(state, "state", d["f32"]), _ptr(ring_k, "ring_k", d["bf16"]),
                       _ptr(ring_v, "ring_v", d["bf16"]), _ptr(ring_gate, "ring_gate", d["f32"]),
                       _ptr(ring_beta, "ring_beta", d["f32"]),
                       _ptr(sketch, "sketch", d["f32"] + d["bf16"]), _ptr(basis, "basis", d["f32"]),
-                      _ptr(coef, "coef", d["f32"]), _ptr(A, "A", d["f32"]))
+                      _ptr(coef, "coef", d["f32"]), _ptr(A, "A", d["f32"]),
+                      _ptr(status, "status", (torch.int32,)))
 
 
 def make_step_io(q, k, v, gate, beta, out):
@@ -230,6 +235,10 @@ def ss_traffic_bytes(plan, op, tau=0):
 
 def ss_launch_count():
     return int(lib().ss_launch_count())
+
+
+def ss_debug_stall_next_copy(plan, stall=True):
+    _check(lib().ss_debug_stall_next_copy(plan.handle, int(bool(stall))))
 
 
 def ss_status_string(s):

@@ -22,6 +22,7 @@ struct ss_plan {
     int32_t R, rmax, Wg;
     int32_t phase;
     int32_t sketch_valid;
+    int32_t stall_next;
 };
 
 namespace {
@@ -60,6 +61,19 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
         if (_s != SS_OK) return _s;       \
     } while (0)
 
+ss_status check_status(const ss_buffers* b) {
+    if (b->status != nullptr && (reinterpret_cast<uintptr_t>(b->status) & 3u) != 0)
+        return fail(SS_ERR_ALIGNMENT, "bufs->status is not 4-byte aligned");
+    return SS_OK;
+}
+
+// Consume the testing hook: the stall applies to one launch only.
+int take_stall(ss_plan* pl) {
+    const int s = pl->stall_next;
+    pl->stall_next = 0;
+    return s;
+}
+
 ss_status check_ring(const ss_plan* pl, const ss_buffers* b) {
     REQUIRE_PTR(b->state, "bufs->state");
     REQUIRE_PTR(b->ring_k, "bufs->ring_k");
@@ -96,6 +110,7 @@ ss::FlushParams flush_params(const ss_plan* pl, const ss_buffers* b, const ss_st
     p.sketch = b->sketch;
     p.basis = b->basis;
     p.A = b->A;
+    p.status = b->status;
     p.B = pl->cfg.batch; p.H = pl->cfg.heads; p.W = pl->cfg.window; p.Wg = pl->Wg; p.R = pl->R;
     p.sketch_bf16 = pl->cfg.sketch_dtype == SS_BF16;
     std::memcpy(p.off, pl->off, sizeof(int32_t) * (pl->cfg.heads + 1));
@@ -108,7 +123,7 @@ ss::StepParams step_params(const ss_plan* pl, const ss_buffers* b, const ss_step
     p.state = b->state;
     p.ring_k = b->ring_k; p.ring_v = b->ring_v; p.ring_gate = b->ring_gate; p.ring_beta = b->ring_beta;
     p.tok_q = io->q; p.tok_k = io->k; p.tok_v = io->v; p.tok_gate = io->gate; p.tok_beta = io->beta;
-    p.sketch = b->sketch; p.coef = b->coef; p.A = b->A; p.out = io->out;
+    p.sketch = b->sketch; p.coef = b->coef; p.A = b->A; p.out = io->out; p.status = b->status;
     p.B = pl->cfg.batch; p.H = pl->cfg.heads; p.W = pl->cfg.window; p.Wg = pl->Wg; p.R = pl->R;
     p.p = pl->phase;
     p.sketch_bf16 = pl->cfg.sketch_dtype == SS_BF16;
@@ -231,6 +246,7 @@ ss_status ss_prime(ss_plan* pl, const ss_buffers* b, ss_stream stream) {
     REQUIRE_PTR(b->state, "bufs->state");
     REQUIRE_PTR(b->sketch, "bufs->sketch");
     REQUIRE_PTR(b->basis, "bufs->basis");
+    CHECK(check_status(b));
     ss::FlushParams p = flush_params(pl, b, nullptr);
     p.n_ring = 0; p.has_token = 0; p.do_sketch = 1;
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
@@ -250,7 +266,9 @@ ss_status ss_decode_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io,
     REQUIRE_PTR(b->sketch, "bufs->sketch");
     REQUIRE_PTR(b->coef, "bufs->coef");
     CHECK(check_io(pl, io));
-    const ss::StepParams p = step_params(pl, b, io);
+    CHECK(check_status(b));
+    ss::StepParams p = step_params(pl, b, io);
+    p.stall = take_stall(pl);
     CHECK(launched(ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
                                      reinterpret_cast<cudaStream_t>(stream)), "decode"));
     pl->phase += 1;
@@ -269,6 +287,7 @@ ss_status ss_flush(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_st
         REQUIRE_PTR(b->sketch, "bufs->sketch");
         REQUIRE_PTR(b->basis, "bufs->basis");
     }
+    CHECK(check_status(b));
     ss::FlushParams p = flush_params(pl, b, io);
     p.n_ring = pl->phase;
     p.has_token = io != nullptr;
@@ -287,6 +306,7 @@ ss_status ss_exact_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
     REQUIRE_PTR(b->state, "bufs->state");
     if (pl->cfg.family == SS_MAMBA2) REQUIRE_PTR(b->A, "bufs->A");
     CHECK(check_io(pl, io));
+    CHECK(check_status(b));
     ss::FlushParams p = flush_params(pl, b, io);
     p.n_ring = 0; p.has_token = 1; p.do_sketch = 0;
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, 0,
@@ -302,7 +322,9 @@ ss_status ss_replay_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io,
                     pl->phase, pl->cfg.window);
     CHECK(check_ring(pl, b));
     CHECK(check_io(pl, io));
-    const ss::StepParams p = step_params(pl, b, io);
+    CHECK(check_status(b));
+    ss::StepParams p = step_params(pl, b, io);
+    p.stall = take_stall(pl);
     CHECK(launched(ss::launch_replay(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p,
                                      reinterpret_cast<cudaStream_t>(stream)), "replay"));
     pl->phase += 1;
@@ -378,6 +400,12 @@ ss_status ss_traffic_bytes(const ss_plan* pl, int32_t op, int32_t tau, ss_traffi
 }
 
 uint64_t ss_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+ss_status ss_debug_stall_next_copy(ss_plan* pl, int32_t stall) {
+    if (pl == nullptr) return fail(SS_ERR_INVALID_ARG, "plan is NULL");
+    pl->stall_next = stall ? 1 : 0;
+    return ok();
+}
 
 const char* ss_status_string(ss_status s) {
     switch (s) {

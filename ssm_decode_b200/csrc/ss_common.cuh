@@ -49,6 +49,62 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// ---------------------------------------------------------------------------
+// Bulk asynchronous copies (TMA, non-tensor) completing on an mbarrier.
+// Every wait is bounded by the global nanosecond timer; a wait that runs out
+// reports SS_DEVICE_TIMEOUT through the optional status word.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+    return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+// Make an mbarrier initialisation visible to the copy engine.
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+// Copy `bytes` (a multiple of 16, both addresses 16-byte aligned) global -> shared.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned phase) {
+    unsigned ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+    return t;
+}
+constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;   // one second
+
+// Wait for the phase `phase` of `bar`; false if the limit ran out first.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned phase) {
+    if (mbar_try_wait(bar, phase)) return true;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, phase))
+        if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
+    return true;
+}
+
+__device__ __forceinline__ void report_timeout(int32_t* status) {
+    if (status != nullptr) atomicOr(status, SS_DEVICE_TIMEOUT);
+}
+
 // Instantiate FN<family, dk, dv> for the runtime (family, dk, dv).
 #define SS_DISPATCH(FN, ...)                                                              \
     do {                                                                                  \

@@ -28,8 +28,10 @@ struct FlushParams {
     const float* basis;
     const float* A;
     float* out;
+    int32_t* status;
     int B, H, W, Wg, R;
     int n_ring, has_token, do_sketch, sketch_bf16;
+    int stall;               // testing hook: extra bytes expected by the first bulk wait
     int off[SS_MAX_HEADS + 1];
 };
 
@@ -51,8 +53,10 @@ struct StepParams {
     const float* coef;       // decode only
     const float* A;
     float* out;
+    int32_t* status;
     int B, H, W, Wg, R;
     int p, sketch_bf16;
+    int stall;               // testing hook: extra bytes expected by the first bulk wait
     int off[SS_MAX_HEADS + 1];
 };
 

@@ -10,22 +10,25 @@
 //  * replay_kernel -- the ReplaySSM non-flush step: the same append and
 //    sweep, then the exact read S0^T q~ + term over the full state.
 //
-// One warp serves one (sequence, head) unit; lane l owns dk/32 consecutive
-// key channels and dv/32 consecutive value channels.  Everything a unit
-// reads -- its live ring slots, its sketch rows and the step's token -- is
-// requested with cp.async at kernel entry, so a unit waits for memory once.
-// The warps of a decode CTA serve the same head for consecutive sequences,
-// so the head's coefficient map C is staged once per CTA.
+// A (sequence, head) unit is served by a group of lanes (16 in decode_kernel,
+// 32 in replay_kernel); lane l owns a slice of consecutive key channels and
+// value channels.  Everything a unit reads -- its live ring slots, its sketch
+// rows and the step's token -- is requested with cp.async at kernel entry, so
+// a unit waits for memory once.  The units of a decode CTA share one head, so
+// the head's coefficient map C is staged once per CTA.
 #include "ss_common.cuh"
 
 namespace ss {
 namespace {
 
-constexpr int DEC_MAX_WARPS = 8;
+#ifndef SS_DEC_MAX_WARPS
+#define SS_DEC_MAX_WARPS 4
+#endif
+constexpr int DEC_MAX_WARPS = SS_DEC_MAX_WARPS;   // warps (= units) per decode CTA
 
 // Per-unit shared-memory layout (byte offsets) of the staged window and token.
 struct UnitSmem {
-    int kraw, vraw, graw, gs, bs, ush, tq, tk, tv, tg, tsc, total;
+    int kraw, vraw, graw, gs, bs, ush, tq, tk, tv, tg, total;
 };
 
 __host__ __device__ inline UnitSmem unit_smem(int fam, int K, int V, int P, int ubytes) {
@@ -42,36 +45,54 @@ __host__ __device__ inline UnitSmem unit_smem(int fam, int K, int V, int P, int 
     L.tk = o;   o += align16(K * 2);
     L.tv = o;   o += align16(V * 2);
     L.tg = o;   o += align16(fam == KDA ? K * 4 : 0);
-    L.tsc = o;  o += 16;
     L.total = o;
     return L;
 }
 
-// Issue (lane-cooperative) cp.async copies of one unit's live ring slots
-// 0..p-1 and of the step's token.
+// Bytes the bulk copies of one unit move: live ring slots 0..p-1, the sketch
+// rows (decode only) and the step's token.
 template <int FAM, int K, int V>
-__device__ __forceinline__ void stage_unit(const StepParams& p, long long unit, int lane,
-                                           unsigned char* sh, const UnitSmem& L) {
-    const long long ring_row = unit * p.W;
-    const int P = p.p;
-    stage(sh + L.kraw, p.ring_k + ring_row * K, P * K * 2, lane, 32);
-    stage(sh + L.vraw, p.ring_v + ring_row * V, P * V * 2, lane, 32);
+__device__ __forceinline__ unsigned unit_bytes(int P, int ubytes) {
     const int P4 = (P + 3) & ~3;
-    if (FAM == KDA) stage(sh + L.graw, p.ring_gate + ring_row * K, P * K * 4, lane, 32);
-    else stage(sh + L.gs, p.ring_gate + unit * p.Wg, P4 * 4, lane, 32);
-    if (FAM != MAMBA2) stage(sh + L.bs, p.ring_beta + unit * p.Wg, P4 * 4, lane, 32);
-    stage(sh + L.tq, p.tok_q + unit * K, K * 2, lane, 32);
-    stage(sh + L.tk, p.tok_k + unit * K, K * 2, lane, 32);
-    stage(sh + L.tv, p.tok_v + unit * V, V * 2, lane, 32);
-    if (FAM == KDA) stage(sh + L.tg, p.tok_gate + unit * K, K * 4, lane, 32);
-    else if (lane == 0) cp_async4(sh + L.tsc, p.tok_gate + unit);
-    if (FAM != MAMBA2 && lane == 1) cp_async4(sh + L.tsc + 4, p.tok_beta + unit);
+    unsigned n = P * K * 2 + P * V * 2 + K * 2 + K * 2 + V * 2 + ubytes;
+    if (FAM == KDA) n += P * K * 4 + K * 4;
+    else if (P > 0) n += P4 * 4;
+    if (FAM != MAMBA2 && P > 0) n += P4 * 4;
+    return n;
+}
+
+// Issue (one lane) the bulk copies of one unit: its live ring slots 0..p-1,
+// `ubytes` of sketch rows from `usrc` (0 for replay) and the step's token.
+template <int FAM, int K, int V>
+__device__ __forceinline__ void stage_unit_bulk(const StepParams& p, long long unit, unsigned char* sh,
+                                                const UnitSmem& L, const void* usrc, int ubytes,
+                                                uint64_t* bar, unsigned extra) {
+    const int P = p.p;
+    mbar_expect_tx(bar, unit_bytes<FAM, K, V>(P, ubytes) + extra);
+    const long long ring_row = unit * p.W;
+    if (P > 0) {
+        const int P4 = (P + 3) & ~3;
+        bulk_g2s(sh + L.kraw, p.ring_k + ring_row * K, P * K * 2, bar);
+        bulk_g2s(sh + L.vraw, p.ring_v + ring_row * V, P * V * 2, bar);
+        if (FAM == KDA) bulk_g2s(sh + L.graw, p.ring_gate + ring_row * K, P * K * 4, bar);
+        else bulk_g2s(sh + L.gs, p.ring_gate + unit * p.Wg, P4 * 4, bar);
+        if (FAM != MAMBA2) bulk_g2s(sh + L.bs, p.ring_beta + unit * p.Wg, P4 * 4, bar);
+    }
+    if (ubytes > 0) bulk_g2s(sh + L.ush, usrc, ubytes, bar);
+    bulk_g2s(sh + L.tq, p.tok_q + unit * K, K * 2, bar);
+    bulk_g2s(sh + L.tk, p.tok_k + unit * K, K * 2, bar);
+    bulk_g2s(sh + L.tv, p.tok_v + unit * V, V * 2, bar);
+    if (FAM == KDA) bulk_g2s(sh + L.tg, p.tok_gate + unit * K, K * 4, bar);
 }
 
 // N consecutive bf16 values, widened.
 template <int N>
 __device__ __forceinline__ void ld_bf16(const uint16_t* src, float (&dst)[N]) {
-    if constexpr (N == 4) {
+    if constexpr (N == 8) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src);
+        dst[0] = bf2f_lo(w.x); dst[1] = bf2f_hi(w.x); dst[2] = bf2f_lo(w.y); dst[3] = bf2f_hi(w.y);
+        dst[4] = bf2f_lo(w.z); dst[5] = bf2f_hi(w.z); dst[6] = bf2f_lo(w.w); dst[7] = bf2f_hi(w.w);
+    } else if constexpr (N == 4) {
         const uint2 w = *reinterpret_cast<const uint2*>(src);
         dst[0] = bf2f_lo(w.x); dst[1] = bf2f_hi(w.x); dst[2] = bf2f_lo(w.y); dst[3] = bf2f_hi(w.y);
     } else {
@@ -83,9 +104,12 @@ __device__ __forceinline__ void ld_bf16(const uint16_t* src, float (&dst)[N]) {
 
 template <int N>
 __device__ __forceinline__ void ld_f32(const float* src, float (&dst)[N]) {
-    if constexpr (N == 4) {
-        const float4 f = *reinterpret_cast<const float4*>(src);
-        dst[0] = f.x; dst[1] = f.y; dst[2] = f.z; dst[3] = f.w;
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i) {
+            const float4 f = reinterpret_cast<const float4*>(src)[i];
+            dst[4 * i] = f.x; dst[4 * i + 1] = f.y; dst[4 * i + 2] = f.z; dst[4 * i + 3] = f.w;
+        }
     } else {
         static_assert(N == 2, "unsupported width");
         const float2 f = *reinterpret_cast<const float2*>(src);
@@ -94,65 +118,62 @@ __device__ __forceinline__ void ld_f32(const float* src, float (&dst)[N]) {
 }
 
 template <int N>
+__device__ __forceinline__ void st_f32(float* dst, const float (&v)[N]) {
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < N / 4; ++i)
+            reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+        *reinterpret_cast<float2*>(dst) = make_float2(v[0], v[1]);
+    }
+}
+
+template <int N>
 __device__ __forceinline__ void copy_bits(uint16_t* dst, const uint16_t* src) {
-    if constexpr (N == 4) *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+    if constexpr (N == 8) *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+    else if constexpr (N == 4) *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
     else *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
 }
 
-// The step's token as this lane sees it.
-template <int K, int V>
+// A unit is served by LPU lanes (16 or 32); lane l owns dk/LPU consecutive
+// key channels and dv/LPU consecutive value channels.
+template <int K, int V, int LPU>
 struct Tok {
-    static constexpr int EK = K / 32, EV = V / 32;
+    static constexpr int EK = K / LPU, EV = V / LPU;
     float q[EK], k[EK], v[EV], g[EK];
     float gs, b;   // scalar decay input (Mamba-2 dt, GDN a) and update strength b
 };
 
-// Append the staged token, bit for bit, at ring slot p and widen it.
-template <int FAM, int K, int V>
-__device__ __forceinline__ void append_token(const StepParams& p, long long unit, int lane,
-                                             const unsigned char* sh, const UnitSmem& L, Tok<K, V>& tk) {
-    constexpr int EK = K / 32, EV = V / 32;
-    const uint16_t* tq = reinterpret_cast<const uint16_t*>(sh + L.tq) + lane * EK;
-    const uint16_t* tkk = reinterpret_cast<const uint16_t*>(sh + L.tk) + lane * EK;
-    const uint16_t* tv = reinterpret_cast<const uint16_t*>(sh + L.tv) + lane * EV;
-    const float* tsc = reinterpret_cast<const float*>(sh + L.tsc);
-    const long long slot = unit * p.W + p.p;
-    copy_bits<EK>(p.ring_k + slot * K + lane * EK, tkk);
-    copy_bits<EV>(p.ring_v + slot * V + lane * EV, tv);
-    ld_bf16<EK>(tq, tk.q);
-    ld_bf16<EK>(tkk, tk.k);
-    ld_bf16<EV>(tv, tk.v);
-    if (FAM == KDA) {
-        ld_f32<EK>(reinterpret_cast<const float*>(sh + L.tg) + lane * EK, tk.g);
-        float* gdst = p.ring_gate + slot * K + lane * EK;
-        if constexpr (EK == 4) *reinterpret_cast<float4*>(gdst) = make_float4(tk.g[0], tk.g[1], tk.g[2], tk.g[3]);
-        else *reinterpret_cast<float2*>(gdst) = make_float2(tk.g[0], tk.g[1]);
-        tk.gs = 1.f;
-    } else {
-        tk.gs = tsc[0];
-        if (lane == 0) p.ring_gate[unit * p.Wg + p.p] = tk.gs;
+constexpr int lg2(int x) { return x <= 1 ? 0 : 1 + lg2(x / 2); }
+
+// Sum over the LPU lanes of a unit (LPU-aligned lane groups).
+template <int LPU>
+__device__ __forceinline__ float group_sum(float x) {
 #pragma unroll
-        for (int e = 0; e < EK; ++e) tk.g[e] = 1.f;
-    }
-    if (FAM != MAMBA2) {
-        tk.b = tsc[1];
-        if (lane == 0) p.ring_beta[unit * p.Wg + p.p] = tk.b;
-    } else {
-        tk.b = tk.gs;   // b_j = dt_j
-    }
+    for (int m = LPU / 2; m >= 1; m >>= 1) x += __shfl_xor_sync(FULL, x, m);
+    return x;
 }
 
-// Butterfly reduce-scatter of NR per-lane partial sums: afterwards lane l
-// holds the warp-wide total of entry l >> (5 - log2 NR).
-template <int NR>
-__device__ __forceinline__ float warp_reduce_scatter(float (&v)[NR], int lane) {
-    constexpr int LG = NR == 8 ? 3 : NR == 16 ? 4 : 5;
-    static_assert(NR == 8 || NR == 16 || NR == 32, "NR must be 8, 16 or 32");
+// Reduce-scatter of NR per-lane partial sums over a unit's LPU lanes.
+// Afterwards, with E = max(NR / LPU, 1), lane l holds in v[0 .. E) the totals
+// of the entries owned by l: entry j lives in lane holder(j), slot(j).
+template <int NR, int LPU>
+struct Scatter {
+    static constexpr int LH = lg2(NR) < lg2(LPU) ? lg2(NR) : lg2(LPU);   // halving levels
+    static constexpr int E = NR >= LPU ? NR / LPU : 1;
+    static constexpr int SH = lg2(LPU) - LH;                              // lanes per entry = 2^SH
+    __device__ static int holder(int j) { return (j / E) << SH; }
+    __device__ static int slot(int j) { return j % E; }
+};
+
+template <int NR, int LPU>
+__device__ __forceinline__ void group_reduce_scatter(float (&v)[NR], int l) {
+    using SC = Scatter<NR, LPU>;
 #pragma unroll
-    for (int lev = 0; lev < LG; ++lev) {
+    for (int lev = 0; lev < SC::LH; ++lev) {
         const int half = NR >> (lev + 1);
-        const int m = 16 >> lev;
-        const bool upper = (lane & m) != 0;
+        const int m = (LPU / 2) >> lev;
+        const bool upper = (l & m) != 0;
 #pragma unroll
         for (int i = 0; i < half; ++i) {
             const float send = upper ? v[i] : v[i + half];
@@ -161,22 +182,55 @@ __device__ __forceinline__ float warp_reduce_scatter(float (&v)[NR], int lane) {
         }
     }
 #pragma unroll
-    for (int m = 16 >> LG; m >= 1; m >>= 1) v[0] += __shfl_xor_sync(FULL, v[0], m);
-    return v[0];
+    for (int m = (1 << SC::SH) / 2; m >= 1; m >>= 1) v[0] += __shfl_xor_sync(FULL, v[0], m);
+}
+
+// Append the staged token, bit for bit, at ring slot p and widen it.
+template <int FAM, int K, int V, int LPU>
+__device__ __forceinline__ void append_token(const StepParams& p, long long unit, int l,
+                                             const unsigned char* sh, const UnitSmem& L, float tgate,
+                                             float tbeta, Tok<K, V, LPU>& tk) {
+    constexpr int EK = K / LPU, EV = V / LPU;
+    const uint16_t* tq = reinterpret_cast<const uint16_t*>(sh + L.tq) + l * EK;
+    const uint16_t* tkk = reinterpret_cast<const uint16_t*>(sh + L.tk) + l * EK;
+    const uint16_t* tv = reinterpret_cast<const uint16_t*>(sh + L.tv) + l * EV;
+    const long long slot = unit * p.W + p.p;
+    copy_bits<EK>(p.ring_k + slot * K + l * EK, tkk);
+    copy_bits<EV>(p.ring_v + slot * V + l * EV, tv);
+    ld_bf16<EK>(tq, tk.q);
+    ld_bf16<EK>(tkk, tk.k);
+    ld_bf16<EV>(tv, tk.v);
+    if (FAM == KDA) {
+        ld_f32<EK>(reinterpret_cast<const float*>(sh + L.tg) + l * EK, tk.g);
+        st_f32<EK>(p.ring_gate + slot * K + l * EK, tk.g);
+        tk.gs = 1.f;
+    } else {
+        tk.gs = tgate;
+        if (l == 0) p.ring_gate[unit * p.Wg + p.p] = tk.gs;
+#pragma unroll
+        for (int e = 0; e < EK; ++e) tk.g[e] = 1.f;
+    }
+    if (FAM != MAMBA2) {
+        tk.b = tbeta;
+        if (l == 0) p.ring_beta[unit * p.Wg + p.p] = tk.b;
+    } else {
+        tk.b = tk.gs;   // b_j = dt_j
+    }
 }
 
 // Mamba-2 window read in closed form (paper §C.1: q~ = d ⊙ q).  With no
 // erase term, x_j = (prod_{i>j} a_i) q, so each buffered update's read is
 // k_j . q scaled by a decay; the NR dot products are reduced together.
-template <int NR, int K, int V>
-__device__ __forceinline__ void sweep_mamba2(const StepParams& p, int h, int lane, const unsigned char* sh,
-                                             const UnitSmem& L, const Tok<K, V>& tk, float (&x)[K / 32],
-                                             float (&ob)[V / 32]) {
-    constexpr int EK = K / 32, EV = V / 32;
-    constexpr int SH = NR == 8 ? 2 : NR == 16 ? 1 : 0;
+template <int NR, int K, int V, int LPU>
+__device__ __forceinline__ void sweep_mamba2(const StepParams& p, int h, int l, int gbase,
+                                             const unsigned char* sh, const UnitSmem& L,
+                                             const Tok<K, V, LPU>& tk, float (&x)[K / LPU],
+                                             float (&ob)[V / LPU]) {
+    constexpr int EK = K / LPU, EV = V / LPU;
+    using SC = Scatter<NR, LPU>;
     const int P = p.p;
-    const uint16_t* kraw = reinterpret_cast<const uint16_t*>(sh + L.kraw) + lane * EK;
-    const uint16_t* vraw = reinterpret_cast<const uint16_t*>(sh + L.vraw) + lane * EV;
+    const uint16_t* kraw = reinterpret_cast<const uint16_t*>(sh + L.kraw) + l * EK;
+    const uint16_t* vraw = reinterpret_cast<const uint16_t*>(sh + L.vraw) + l * EV;
     const float* gs = reinterpret_cast<const float*>(sh + L.gs);
     float v[NR];
 #pragma unroll
@@ -193,47 +247,50 @@ __device__ __forceinline__ void sweep_mamba2(const StepParams& p, int h, int lan
         }
         v[j] = acc;
     }
-    const float dots = warp_reduce_scatter<NR>(v, lane);      // lane l: k_{l >> SH} . q
-    // lane j: dt_j, and the decay after update j, exp(A * sum_{i>j} dt_i)
+    group_reduce_scatter<NR, LPU>(v, l);
+    // decays: c_j = dt_j exp(A sum_{i>j} dt_i), computed for the entries this lane holds
     const float A = p.A[h];
-    const float dt = lane < P ? gs[lane] : (lane == P ? tk.gs : 0.f);
-    float incl = dt;
+    float pref = 0.f, my_pref[SC::E], my_dt[SC::E];
 #pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-        const float y = __shfl_up_sync(FULL, incl, m);
-        if (lane >= m) incl += y;
+    for (int i = 0; i < SC::E; ++i) { my_pref[i] = 0.f; my_dt[i] = 0.f; }
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+        const float dt = j < P ? gs[j] : (j == P ? tk.gs : 0.f);
+        pref += dt;
+        if (SC::holder(j) == (l & ~((1 << SC::SH) - 1))) { my_pref[SC::slot(j)] = pref; my_dt[SC::slot(j)] = dt; }
     }
-    const float total = __shfl_sync(FULL, incl, 31);
-    const float cs = dt * expf(A * (total - incl));
-    const float qs = expf(A * total);
+    float c[SC::E];
+#pragma unroll
+    for (int i = 0; i < SC::E; ++i) c[i] = my_dt[i] * expf(A * (pref - my_pref[i])) * v[i];
+    const float qs = expf(A * pref);
 #pragma unroll
     for (int e = 0; e < EK; ++e) x[e] = qs * tk.q[e];
 #pragma unroll
     for (int e = 0; e < EV; ++e) ob[e] = 0.f;
-#pragma unroll 4
-    for (int j = 0; j <= P; ++j) {
-        const float cj = __shfl_sync(FULL, cs, j) * __shfl_sync(FULL, dots, j << SH);
-        float vj[EV];
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+        const float cj = __shfl_sync(FULL, c[SC::slot(j)], gbase + SC::holder(j));
         if (j < P) {
+            float vj[EV];
             ld_bf16<EV>(vraw + j * V, vj);
-        } else {
 #pragma unroll
-            for (int e = 0; e < EV; ++e) vj[e] = tk.v[e];
+            for (int e = 0; e < EV; ++e) ob[e] = fmaf(cj, vj[e], ob[e]);
+        } else if (j == P) {
+#pragma unroll
+            for (int e = 0; e < EV; ++e) ob[e] = fmaf(cj, tk.v[e], ob[e]);
         }
-#pragma unroll
-        for (int e = 0; e < EV; ++e) ob[e] = fmaf(cj, vj[e], ob[e]);
     }
 }
 
 // Delta-rule (and generic) window read: the sequential backward sweep.
-template <int FAM, int K, int V>
-__device__ __forceinline__ void sweep_seq(const StepParams& p, int h, int lane, const unsigned char* sh,
-                                          const UnitSmem& L, const Tok<K, V>& tk, float (&x)[K / 32],
-                                          float (&ob)[V / 32]) {
-    constexpr int EK = K / 32, EV = V / 32;
-    const uint16_t* kraw = reinterpret_cast<const uint16_t*>(sh + L.kraw) + lane * EK;
-    const uint16_t* vraw = reinterpret_cast<const uint16_t*>(sh + L.vraw) + lane * EV;
-    const float* graw = reinterpret_cast<const float*>(sh + L.graw) + lane * EK;
+template <int FAM, int K, int V, int LPU>
+__device__ __forceinline__ void sweep_seq(const StepParams& p, int h, int l, const unsigned char* sh,
+                                          const UnitSmem& L, const Tok<K, V, LPU>& tk, float (&x)[K / LPU],
+                                          float (&ob)[V / LPU]) {
+    constexpr int EK = K / LPU, EV = V / LPU;
+    const uint16_t* kraw = reinterpret_cast<const uint16_t*>(sh + L.kraw) + l * EK;
+    const uint16_t* vraw = reinterpret_cast<const uint16_t*>(sh + L.vraw) + l * EV;
+    const float* graw = reinterpret_cast<const float*>(sh + L.graw) + l * EK;
     const float* gs = reinterpret_cast<const float*>(sh + L.gs);
     const float* bs = reinterpret_cast<const float*>(sh + L.bs);
     const float A = (FAM == MAMBA2) ? p.A[h] : 0.f;
@@ -263,10 +320,10 @@ __device__ __forceinline__ void sweep_seq(const StepParams& p, int h, int lane, 
             bj = (FAM == MAMBA2) ? a_s : bs[j];
         }
         if (FAM == MAMBA2) a_s = expf(a_s * A);
-        float kx = 0.f;
+        float k0 = 0.f, k1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < EK; ++e) kx = fmaf(kj[e], x[e], kx);
-        const float bsx = bj * warp_sum(kx);
+        for (int e = 0; e < EK; e += 2) { k0 = fmaf(kj[e], x[e], k0); k1 = fmaf(kj[e + 1], x[e + 1], k1); }
+        const float bsx = bj * group_sum<LPU>(k0 + k1);
 #pragma unroll
         for (int e = 0; e < EV; ++e) ob[e] = fmaf(bsx, vj[e], ob[e]);
 #pragma unroll
@@ -279,97 +336,148 @@ __device__ __forceinline__ void sweep_seq(const StepParams& p, int h, int lane, 
 }
 
 // c = C q~ for nr <= NR rows of C (shared memory), reduce-scattered; then
-// o += sum_i c_i u_i with the sketch rows in shared memory.
-template <int NR, int K, int V>
-__device__ __forceinline__ void readout(const float* csm, const unsigned char* ush, int nr, bool bf16,
-                                        int lane, const float (&x)[K / 32], float (&o)[V / 32]) {
-    constexpr int EK = K / 32, EV = V / 32;
-    constexpr int SH = NR == 8 ? 2 : NR == 16 ? 1 : 0;
+// o += sum_i c_i u_i, the sketch rows read through `U(i, u)`.
+template <int NR, int K, int V, int LPU, typename LoadU>
+__device__ __forceinline__ void readout(const float* csm, int nr, int l, int gbase, const float (&x)[K / LPU],
+                                        float (&o)[V / LPU], LoadU U) {
+    constexpr int EK = K / LPU, EV = V / LPU;
+    using SC = Scatter<NR, LPU>;
     float v[NR];
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
         float acc = 0.f;
         if (i < nr) {
             float cr[EK];
-            ld_f32<EK>(csm + i * K + lane * EK, cr);
+            ld_f32<EK>(csm + i * K + l * EK, cr);
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < EK; ++e) acc = fmaf(cr[e], x[e], acc);
+            for (int e = 0; e < EK; e += 2) { a0 = fmaf(cr[e], x[e], a0); a1 = fmaf(cr[e + 1], x[e + 1], a1); }
+            acc = a0 + a1;
         }
         v[i] = acc;
     }
-    const float c = warp_reduce_scatter<NR>(v, lane);
-#pragma unroll 4
-    for (int i = 0; i < nr; ++i) {
-        const float ci = __shfl_sync(FULL, c, i << SH);
-        float u[EV];
-        if (bf16) ld_bf16<EV>(reinterpret_cast<const uint16_t*>(ush) + i * V + lane * EV, u);
-        else ld_f32<EV>(reinterpret_cast<const float*>(ush) + i * V + lane * EV, u);
+    group_reduce_scatter<NR, LPU>(v, l);
 #pragma unroll
-        for (int e = 0; e < EV; ++e) o[e] = fmaf(ci, u[e], o[e]);
+    for (int i = 0; i < NR; ++i) {
+        const float ci = __shfl_sync(FULL, v[SC::slot(i)], gbase + SC::holder(i));
+        if (i < nr) {
+            float u[EV];
+            U(i, u);
+#pragma unroll
+            for (int e = 0; e < EV; ++e) o[e] = fmaf(ci, u[e], o[e]);
+        }
     }
 }
 
-template <int FAM, int K, int V>
-__device__ __forceinline__ void window_read(const StepParams& p, int h, int lane, const unsigned char* sh,
-                                            const UnitSmem& L, const Tok<K, V>& tk, float (&x)[K / 32],
-                                            float (&ob)[V / 32]) {
+template <int FAM, int K, int V, int LPU>
+__device__ __forceinline__ void window_read(const StepParams& p, int h, int l, int gbase, const unsigned char* sh,
+                                            const UnitSmem& L, const Tok<K, V, LPU>& tk, float (&x)[K / LPU],
+                                            float (&ob)[V / LPU]) {
     if constexpr (FAM == MAMBA2) {
         const int n = p.p + 1;
-        if (n <= 8) sweep_mamba2<8, K, V>(p, h, lane, sh, L, tk, x, ob);
-        else if (n <= 16) sweep_mamba2<16, K, V>(p, h, lane, sh, L, tk, x, ob);
-        else sweep_mamba2<32, K, V>(p, h, lane, sh, L, tk, x, ob);
+        if (n <= 8) sweep_mamba2<8, K, V, LPU>(p, h, l, gbase, sh, L, tk, x, ob);
+        else if (n <= 16) sweep_mamba2<16, K, V, LPU>(p, h, l, gbase, sh, L, tk, x, ob);
+        else sweep_mamba2<32, K, V, LPU>(p, h, l, gbase, sh, L, tk, x, ob);
     } else {
-        sweep_seq<FAM, K, V>(p, h, lane, sh, L, tk, x, ob);
+        sweep_seq<FAM, K, V, LPU>(p, h, l, sh, L, tk, x, ob);
     }
 }
 
 // ---------------------------------------------------------------------------
-// decode_kernel
+// decode_kernel: DEC_LPU lanes per unit.  CTA (x, h) serves head h for
+// consecutive sequences: one bulk copy stages h's coefficient map C, and the
+// first lane of each unit issues that unit's bulk copies; everything lands on
+// mbarriers, so each unit waits for memory once.
 // ---------------------------------------------------------------------------
+#ifndef SS_DEC_LPU
+#define SS_DEC_LPU 16
+#endif
+constexpr int DEC_LPU = SS_DEC_LPU;
+
+__host__ __device__ inline int dec_unit_bytes(int fam, int K, int V, int P, int ubytes) {
+    return 16 + unit_smem(fam, K, V, P, ubytes).total;      // mbarrier + staged unit
+}
+
 template <int FAM, int K, int V>
 __global__ void __launch_bounds__(DEC_MAX_WARPS * 32) decode_kernel(const __grid_constant__ StepParams p,
                                                                     int rmax) {
-    constexpr int EK = K / 32, EV = V / 32;
+    constexpr int LPU = DEC_LPU, UPW = 32 / LPU, EK = K / LPU, EV = V / LPU;
     extern __shared__ __align__(16) unsigned char smem[];
     const int wpc = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nbg = (p.B + wpc - 1) / wpc;
-    const int h = blockIdx.x / nbg;
-    const int b = (blockIdx.x % nbg) * wpc + warp;
+    const int hw = lane / LPU, l = lane % LPU, gbase = hw * LPU;
+    const int h = blockIdx.y;
+    const int b = (blockIdx.x * wpc + warp) * UPW + hw;
     const bool active = b < p.B;
     const long long unit = (long long)b * p.H + h;
     const int esz = p.sketch_bf16 ? 2 : 4;
     const int off = p.off[h], r = p.off[h + 1] - off;
+    const int ubytes = r * V * esz;
     const UnitSmem L = unit_smem(FAM, K, V, p.p, rmax * V * esz);
-    float* csm = reinterpret_cast<float*>(smem);
-    unsigned char* sh = smem + align16(rmax * K * 4) + warp * L.total;
+    const int cbytes = align16(rmax * K * 4);
+    const float* csm = reinterpret_cast<const float*>(smem);
+    uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + cbytes);
+    unsigned char* ubase = smem + cbytes + 16 + (warp * UPW + hw) * dec_unit_bytes(FAM, K, V, p.p, rmax * V * esz);
+    uint64_t* ubar = reinterpret_cast<uint64_t*>(ubase);
+    unsigned char* sh = ubase + 16;
 
-    stage(csm, p.coef + (long long)off * K, r * K * 4, threadIdx.x, blockDim.x);
-    if (active) {
-        stage_unit<FAM, K, V>(p, unit, lane, sh, L);
-        stage(sh + L.ush, static_cast<const char*>(p.sketch) + (b * (long long)p.R + off) * (V * esz),
-              r * V * esz, lane, 32);
+    if (threadIdx.x == 0) mbar_init(cbar, 1);
+    if (l == 0) mbar_init(ubar, 1);
+    fence_mbar_init();
+    __syncthreads();                                        // the only block barrier
+    const bool stall = p.stall && blockIdx.x == 0 && blockIdx.y == 0;
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(cbar, r * K * 4 + (stall ? 16u : 0u));
+        if (r > 0) bulk_g2s(smem, p.coef + (long long)off * K, r * K * 4, cbar);
     }
-    cp_async_commit();
-    cp_async_wait_all();
-    __syncthreads();
-    if (!active) return;                      // whole warps; no block barrier follows
+    if (active && l == 0)
+        stage_unit_bulk<FAM, K, V>(p, unit, sh, L,
+                                   static_cast<const char*>(p.sketch) + (b * (long long)p.R + off) * (V * esz),
+                                   ubytes, ubar, 0u);
+    float tgate = 0.f, tbeta = 0.f;                         // token scalars: plain loads
+    if (active) {
+        if (FAM != KDA) tgate = p.tok_gate[unit];
+        if (FAM != MAMBA2) tbeta = p.tok_beta[unit];
+    }
+    bool ok = mbar_wait(cbar, 0);
+    if (active) ok = mbar_wait(ubar, 0) && ok;
+    if (!ok) {                                              // a bounded wait ran out
+        report_timeout(p.status);
+        mbar_wait(cbar, 0);                                 // give own copies one more bounded wait
+        if (active) mbar_wait(ubar, 0);
+        return;
+    }
+    if (__all_sync(FULL, !active)) return;
 
-    Tok<K, V> tk;
-    append_token<FAM, K, V>(p, unit, lane, sh, L, tk);
+    // Lanes whose unit lies past the batch take part in the shuffles (on
+    // zeros, inside their own lane group) but store nothing.
+    Tok<K, V, LPU> tk;
+    if (active) {
+        append_token<FAM, K, V, LPU>(p, unit, l, sh, L, tgate, tbeta, tk);
+    } else {
+#pragma unroll
+        for (int e = 0; e < EK; ++e) { tk.q[e] = 0.f; tk.k[e] = 0.f; tk.g[e] = 1.f; }
+#pragma unroll
+        for (int e = 0; e < EV; ++e) tk.v[e] = 0.f;
+        tk.gs = 0.f;
+        tk.b = 0.f;
+    }
     float x[EK], ob[EV];
-    window_read<FAM, K, V>(p, h, lane, sh, L, tk, x, ob);
+    window_read<FAM, K, V, LPU>(p, h, l, gbase, sh, L, tk, x, ob);
+    const bool bf16 = p.sketch_bf16;
     for (int i0 = 0; i0 < r; i0 += 32) {
         const int nr = min(32, r - i0);
         const float* cs = csm + i0 * K;
         const unsigned char* us = sh + L.ush + i0 * V * esz;
-        if (nr <= 8) readout<8, K, V>(cs, us, nr, p.sketch_bf16, lane, x, ob);
-        else if (nr <= 16) readout<16, K, V>(cs, us, nr, p.sketch_bf16, lane, x, ob);
-        else readout<32, K, V>(cs, us, nr, p.sketch_bf16, lane, x, ob);
+        auto loadU = [&](int i, float (&u)[EV]) {
+            if (bf16) ld_bf16<EV>(reinterpret_cast<const uint16_t*>(us) + i * V + l * EV, u);
+            else ld_f32<EV>(reinterpret_cast<const float*>(us) + i * V + l * EV, u);
+        };
+        if (nr <= 8) readout<8, K, V, LPU>(cs, nr, l, gbase, x, ob, loadU);
+        else if (nr <= 16) readout<16, K, V, LPU>(cs, nr, l, gbase, x, ob, loadU);
+        else readout<32, K, V, LPU>(cs, nr, l, gbase, x, ob, loadU);
     }
-    float* dst = p.out + unit * V + lane * EV;
-    if constexpr (EV == 4) *reinterpret_cast<float4*>(dst) = make_float4(ob[0], ob[1], ob[2], ob[3]);
-    else *reinterpret_cast<float2*>(dst) = make_float2(ob[0], ob[1]);
+    if (active) st_f32<EV>(p.out + unit * V + l * EV, ob);
 }
 
 // ---------------------------------------------------------------------------
@@ -383,7 +491,7 @@ __device__ __forceinline__ int kpad4(int c) {
 }
 
 __host__ __device__ inline int replay_unit_bytes(int fam, int K, int V, int P) {
-    return unit_smem(fam, K, V, P, 0).total + align16((K + 16) * 4) + align16(V * 4);
+    return unit_smem(fam, K, V, P, 0).total + align16((K + 16) * 4) + align16(V * 4) + 16;   // + mbarrier
 }
 
 template <int FAM, int K, int V>
@@ -401,6 +509,7 @@ __global__ void __launch_bounds__(128) replay_kernel(const __grid_constant__ Ste
     unsigned char* sh = smem + hl * replay_unit_bytes(FAM, K, V, p.p);
     float* qt = reinterpret_cast<float*>(sh + L.total);
     float* obs = reinterpret_cast<float*>(sh + L.total + align16((K + 16) * 4));
+    bool timed_out = false;
 
     const float* st = p.state + unit * (long long)(K * V);
     float s[R][4];
@@ -412,19 +521,31 @@ __global__ void __launch_bounds__(128) replay_kernel(const __grid_constant__ Ste
         }
     }
     if (active && t < 32) {
-        stage_unit<FAM, K, V>(p, unit, lane, sh, L);
-        cp_async_commit();
-        cp_async_wait_all();
+        uint64_t* bar = reinterpret_cast<uint64_t*>(sh + L.total + align16((K + 16) * 4) + align16(V * 4));
+        if (lane == 0) {
+            mbar_init(bar, 1);
+            fence_mbar_init();
+            stage_unit_bulk<FAM, K, V>(p, unit, sh, L, nullptr, 0, bar, p.stall && unit == 0 ? 16u : 0u);
+        }
+        const float tgate = FAM != KDA ? p.tok_gate[unit] : 0.f;
+        const float tbeta = FAM != MAMBA2 ? p.tok_beta[unit] : 0.f;
         __syncwarp();
-        Tok<K, V> tk;
-        append_token<FAM, K, V>(p, unit, lane, sh, L, tk);
-        float x[EK], ob[EV];
-        window_read<FAM, K, V>(p, h, lane, sh, L, tk, x, ob);
+        timed_out = !mbar_wait(bar, 0);
+        if (timed_out) {
+            report_timeout(p.status);
+            mbar_wait(bar, 0);
+        } else {
+            Tok<K, V, 32> tk;
+            append_token<FAM, K, V, 32>(p, unit, lane, sh, L, tgate, tbeta, tk);
+            float x[EK], ob[EV];
+            window_read<FAM, K, V, 32>(p, h, lane, 0, sh, L, tk, x, ob);
 #pragma unroll
-        for (int e = 0; e < EK; ++e) qt[kpad4<K>(lane * EK + e)] = x[e];
+            for (int e = 0; e < EK; ++e) qt[kpad4<K>(lane * EK + e)] = x[e];
 #pragma unroll
-        for (int e = 0; e < EV; ++e) obs[lane * EV + e] = ob[e];
+            for (int e = 0; e < EV; ++e) obs[lane * EV + e] = ob[e];
+        }
     }
+    if (__syncthreads_or(timed_out)) return;
     __syncthreads();
     if (!active) return;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -452,21 +573,23 @@ __global__ void __launch_bounds__(128) replay_kernel(const __grid_constant__ Ste
 // launchers
 // ---------------------------------------------------------------------------
 int decode_bytes(int fam, int K, int V, int P, int rmax, int esz, int wpc) {
-    return align16(rmax * K * 4) + wpc * unit_smem(fam, K, V, P, rmax * V * esz).total;
+    return align16(rmax * K * 4) + 16 + wpc * (32 / DEC_LPU) * dec_unit_bytes(fam, K, V, P, rmax * V * esz);
 }
 
 template <int FAM, int K, int V>
 cudaError_t decode_t(const StepParams& p, int rmax, cudaStream_t stream) {
     const int esz = p.sketch_bf16 ? 2 : 4;
+    const int upw = 32 / DEC_LPU;
     int wpc = DEC_MAX_WARPS;
-    while (wpc > 1 && (decode_bytes(FAM, K, V, p.p, rmax, esz, wpc) > SMEM_LIMIT || wpc > p.B)) --wpc;
+    while (wpc > 1 && (decode_bytes(FAM, K, V, p.p, rmax, esz, wpc) > SMEM_LIMIT || (wpc - 1) * upw >= p.B)) --wpc;
     const int bytes = decode_bytes(FAM, K, V, p.p, rmax, esz, wpc);
     if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
-    const long long grid = (long long)p.H * ((p.B + wpc - 1) / wpc);
+    const int upc = wpc * upw;
+    const dim3 grid(unsigned((p.B + upc - 1) / upc), unsigned(p.H));
     auto kern = decode_kernel<FAM, K, V>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(unsigned(grid)), dim3(wpc * 32), bytes, stream>>>(p, rmax);
+    kern<<<grid, dim3(wpc * 32), bytes, stream>>>(p, rmax);
     return cudaGetLastError();
 }
 

@@ -45,6 +45,7 @@ class DecodeLayer:
         self.coef = z(max(self.R, 1), dk)
         self.A = z(heads)
         self.out = z(batch, heads, dv)
+        self.status = torch.zeros(4, dtype=torch.int32, device=device)   # device status word (+ padding)
         self.sketch_dtype = sketch_dtype
 
     # -- data -------------------------------------------------------------------
@@ -68,7 +69,8 @@ class DecodeLayer:
 
     def bufs(self, with_sketch=True):
         return B.make_buffers(self.state, self.ring_k, self.ring_v, self.ring_gate, self.ring_beta,
-                              self.sketch if with_sketch else None, self.basis, self.coef, self.A)
+                              self.sketch if with_sketch else None, self.basis, self.coef, self.A,
+                              self.status)
 
     def io(self, tok, out=None):
         beta = tok["beta"] if self.family != B.SS_MAMBA2 else None

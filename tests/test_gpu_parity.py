@@ -231,3 +231,29 @@ def test_sweep_points_sampled(cuda_ok, batch, window, mean_rank):
     p.prime()
     for t in range(window + 2):
         p.step(synth.step_inputs(wl, p.st, t), ring=False)
+
+
+@pytest.mark.parametrize("call", ["decode", "replay"])
+def test_bounded_wait_reports_timeout(cuda_ok, call):
+    """A launch whose bulk copies deliver fewer bytes than one CTA expects: that
+    CTA's bounded wait runs out, it sets SS_DEVICE_TIMEOUT in the status word
+    and returns; the context stays usable and later launches are clean."""
+    import torch
+    wl = small(synth.GDN, 128, 128, batch=4, heads=3, seed=1500)
+    p = Pair(wl)
+    p.layer.prime()
+    torch.cuda.synchronize()
+    assert int(p.layer.status[0]) == 0
+    B.ss_debug_stall_next_copy(p.layer.plan, True)
+    tok = p.layer.token(synth.step_inputs(wl, p.st, 0))
+    if call == "decode":
+        p.layer.decode(tok)
+    else:
+        B.ss_replay_step(p.layer.plan, p.layer.bufs(False), p.layer.io(tok))
+    torch.cuda.synchronize()
+    assert int(p.layer.status[0]) & B.SS_DEVICE_TIMEOUT
+    # the context is still usable: a fresh session runs clean and matches the oracle
+    q = Pair(wl)
+    run(q, 6)
+    torch.cuda.synchronize()
+    assert int(q.layer.status[0]) == 0
