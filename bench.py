@@ -24,6 +24,7 @@ sample of the same workload (the pages publish no runnable implementation).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -182,6 +183,8 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wl = synth.WORKLOADS[args.workload]
+    if args.batch:
+        wl = dataclasses.replace(wl, name=f"{wl.name}@batch{args.batch}", batch=args.batch)
     skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
     W, NL = wl.window, args.layers
     st = synth.static_inputs(wl)
@@ -401,6 +404,8 @@ def main():
     ap.add_argument("--workload", default="mamba2_b320")
     ap.add_argument("--sketch-dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
