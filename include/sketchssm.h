@@ -156,8 +156,15 @@ typedef struct {
 } ss_traffic;
 
 /* Create a plan for one layer's decode.  The config (and ranks) are copied.
- * Returns SS_ERR_INVALID_ARG / SS_ERR_UNSUPPORTED for bad shapes.  The plan
- * starts at phase 0 with no valid sketch. */
+ * Returns SS_ERR_INVALID_ARG / SS_ERR_UNSUPPORTED for bad shapes.
+ * SS_ERR_UNSUPPORTED also when a call of the plan would need more shared
+ * memory than one CTA has: the flush stages the window's keys, values and
+ * decays plus the basis rows of one head, and the decode step stages, per
+ * warp, the window's ring slots and sketch rows plus the head's map C
+ * (rmax x dk fp32), so very large ranks with long windows do not fit (e.g.
+ * rank 128 with dk = dv = 128 and W = 32).  Every rank up to 64 at W <= 16,
+ * and up to 32 at W <= 32, is supported.  The plan starts at phase 0
+ * with no valid sketch. */
 ss_status ss_create(const ss_config* cfg, ss_plan** out);
 ss_status ss_destroy(ss_plan* plan);
 

@@ -185,9 +185,10 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
     const int fl = ss::flush_smem_bytes(c.family, c.dk, c.dv, c.window, rpad);
     const int dec = ss::decode_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax, esize(pl));
     if (fl > kSmemLimit || dec > kSmemLimit) {
+        const int rmax = pl->rmax;
         delete pl;
         return fail(SS_ERR_UNSUPPORTED, "window %d with max rank %d needs %d / %d bytes of shared memory",
-                    c.window, pl->rmax, fl, dec);
+                    c.window, rmax, fl, dec);
     }
     *out = pl;
     return ok();

@@ -3,6 +3,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "ss_internal.h"
 
 namespace ss {
@@ -13,7 +15,8 @@ constexpr unsigned FULL = 0xffffffffu;
 // folded into the stored state (see flush_kernel).
 constexpr float GAMMA_LO = 2.3283064365386963e-10f;
 constexpr float GAMMA_HI = 4294967296.0f;
-constexpr int SMEM_LIMIT = 227 * 1024;
+constexpr int SMEM_LIMIT = 227 * 1024;        // dynamic shared memory per CTA
+constexpr int SMEM_SM = 228 * 1024;           // shared memory per SM (1 KB of it reserved per CTA)
 
 __host__ __device__ __forceinline__ int align16(int x) { return (x + 15) & ~15; }
 
@@ -69,6 +72,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
                  : "memory");
 }
 // Copy `bytes` (a multiple of 16, both addresses 16-byte aligned) global -> shared.
+// Plain arrival (no transaction bytes) on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
@@ -125,5 +133,75 @@ __device__ __forceinline__ void report_timeout(int32_t* status) {
             default: return cudaErrorInvalidValue;                                        \
         }                                                                                 \
     } while (0)
+
+// Streaming multiprocessors of the current device (148 on B200), for
+// persistent grids.
+inline int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+// Host-side cache of one kernel's launch attributes, per device: registers
+// per thread (queried once), the dynamic shared-memory limit set so far (the
+// attribute is only raised), and the last occupancy answer.  Steady-state
+// launches then make no attribute or occupancy queries.
+struct KernelCache {
+    static constexpr int MAXDEV = 16;
+    std::atomic<int> regs[MAXDEV] = {};
+    std::atomic<int> smem[MAXDEV] = {};
+    std::atomic<long long> occ[MAXDEV] = {};   // (block threads << 40) | (bytes << 8) | blocks per SM
+};
+
+inline int cur_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= KernelCache::MAXDEV) d = 0;
+    return d;
+}
+
+template <typename F>
+cudaError_t cached_regs(F kern, KernelCache& kc, int* regs) {
+    const int d = cur_device();
+    int r = kc.regs[d].load(std::memory_order_relaxed);
+    if (r <= 0) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        r = fa.numRegs > 0 ? fa.numRegs : 64;
+        kc.regs[d].store(r, std::memory_order_relaxed);
+    }
+    *regs = r;
+    return cudaSuccess;
+}
+
+template <typename F>
+cudaError_t ensure_smem(F kern, KernelCache& kc, int bytes) {
+    const int d = cur_device();
+    if (bytes <= kc.smem[d].load(std::memory_order_relaxed)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) kc.smem[d].store(bytes, std::memory_order_relaxed);
+    return e;
+}
+
+template <typename F>
+cudaError_t cached_occupancy(F kern, KernelCache& kc, int threads, int bytes, int* per_sm) {
+    const int d = cur_device();
+    const long long key = ((long long)threads << 40) | ((long long)bytes << 8);
+    const long long v = kc.occ[d].load(std::memory_order_relaxed);
+    if (v != 0 && (v & ~0xffLL) == key) { *per_sm = int(v & 0xff); return cudaSuccess; }
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, bytes);
+    if (e != cudaSuccess) return e;
+    if (n < 1) n = 1;
+    if (n > 255) n = 255;
+    kc.occ[d].store(key | n, std::memory_order_relaxed);
+    *per_sm = n;
+    return cudaSuccess;
+}
 
 }  // namespace ss

@@ -478,17 +478,6 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
     cp_async_wait_all();
 }
 
-int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
 template <int FAM, int K, int V>
 cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
     const int n = p.n_ring + p.has_token;
@@ -496,12 +485,12 @@ cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
     const int bytes = flush_layout(FAM, K, V, n, rpad).total;
     if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
     auto kern = flush_kernel<FAM, K, V>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    static KernelCache kc;
+    cudaError_t e = ensure_smem(kern, kc, bytes);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, FS<K, V>::T, bytes);
+    e = cached_occupancy(kern, kc, FS<K, V>::T, bytes, &per_sm);
     if (e != cudaSuccess) return e;
-    if (per_sm < 1) per_sm = 1;
     const long long units = (long long)p.B * p.H;
     const long long cap = (long long)per_sm * sm_count();
     const long long grid = units < cap ? units : cap;

@@ -10,21 +10,18 @@
 //  * replay_kernel -- the ReplaySSM non-flush step: the same append and
 //    sweep, then the exact read S0^T q~ + term over the full state.
 //
-// A (sequence, head) unit is served by a group of lanes (16 in decode_kernel,
-// 32 in replay_kernel); lane l owns a slice of consecutive key channels and
-// value channels.  Everything a unit reads -- its live ring slots, its sketch
-// rows and the step's token -- is requested with cp.async at kernel entry, so
-// a unit waits for memory once.  The units of a decode CTA share one head, so
-// the head's coefficient map C is staged once per CTA.
+// A (sequence, head) unit is served by one warp; lane l owns dk/32
+// consecutive key channels and dv/32 consecutive value channels.  Everything
+// a unit reads from HBM -- its live ring slots, its sketch rows and the
+// step's token -- arrives by bulk asynchronous copies (cp.async.bulk) that
+// complete on an mbarrier, issued by one lane, so a unit waits for memory
+// once.  Every wait is bounded: when one runs out the kernel sets
+// SS_DEVICE_TIMEOUT in the caller's status word and returns.
 #include "ss_common.cuh"
 
 namespace ss {
 namespace {
 
-#ifndef SS_DEC_MAX_WARPS
-#define SS_DEC_MAX_WARPS 4
-#endif
-constexpr int DEC_MAX_WARPS = SS_DEC_MAX_WARPS;   // warps (= units) per decode CTA
 
 // Per-unit shared-memory layout (byte offsets) of the staged window and token.
 struct UnitSmem {
@@ -384,100 +381,379 @@ __device__ __forceinline__ void window_read(const StepParams& p, int h, int l, i
 }
 
 // ---------------------------------------------------------------------------
-// decode_kernel: DEC_LPU lanes per unit.  CTA (x, h) serves head h for
-// consecutive sequences: one bulk copy stages h's coefficient map C, and the
-// first lane of each unit issues that unit's bulk copies; everything lands on
-// mbarriers, so each unit waits for memory once.
+// decode_kernel.  A unit is served by a group of G = dec_gl(family) lanes,
+// so a warp carries 32/G units (consecutive sequences of one head) through
+// every instruction.  Each lane owns chunks of consecutive key and value
+// channels (see Own), so a group's shared-memory reads are contiguous.  Dot
+// products are reduced over the group with a butterfly.
+//
+// CTA (x, h) serves head h; one bulk copy stages the head's coefficient rows
+// C (shared by the batch) once.  Warp w of CTA x takes the unit groups
+// x*wpc + w + k*nb*wpc (k = 0, 1, ...) and runs them through NS staging
+// buffers, issuing the bulk copies (live ring slots, sketch rows, token) of
+// its next NS-1 groups before computing the current one.  The launcher
+// below uses NS = 1 and one group per warp: on the bench shapes shared
+// memory, not registers, bounds the units resident on an SM, and spending it
+// on more CTAs measured faster than on deeper per-warp pipelines.
 // ---------------------------------------------------------------------------
-#ifndef SS_DEC_LPU
-#define SS_DEC_LPU 16
-#endif
-constexpr int DEC_LPU = SS_DEC_LPU;
+constexpr int DEC_WARPS = 4;              // warps per decode CTA
 
-__host__ __device__ inline int dec_unit_bytes(int fam, int K, int V, int P, int ubytes) {
-    return 16 + unit_smem(fam, K, V, P, ubytes).total;      // mbarrier + staged unit
+// Lanes per unit.  Mamba-2's reads are independent dot products, which 16
+// lanes (2 units per warp) reduce cheaply; the delta rule's sweep is serial
+// per unit, which 32 lanes (one unit per warp, more warps per SM) hide best.
+__host__ __device__ constexpr int dec_gl(int fam) { return fam == MAMBA2 ? 16 : 32; }
+
+__host__ __device__ inline int dec_stage_bytes(int fam, int K, int V, int P, int ubytes) {
+    return 16 + (32 / dec_gl(fam)) * unit_smem(fam, K, V, P, ubytes).total;   // mbarrier + the warp's units
 }
 
-template <int FAM, int K, int V>
-__global__ void __launch_bounds__(DEC_MAX_WARPS * 32) decode_kernel(const __grid_constant__ StepParams p,
-                                                                    int rmax) {
-    constexpr int LPU = DEC_LPU, UPW = 32 / LPU, EK = K / LPU, EV = V / LPU;
+// Sum over the G lanes of a unit.
+template <int G>
+__device__ __forceinline__ float gsum(float x) {
+#pragma unroll
+    for (int m = 1; m < G; m <<= 1) x += __shfl_xor_sync(FULL, x, m);
+    return x;
+}
+
+// Channel ownership inside a unit's lane group, for a row of N values: lane
+// l owns M chunks of CH consecutive channels, chunk m starting at
+// m * G * CH + l * CH, so a group's 16-byte shared-memory reads of a bf16
+// row cover contiguous bytes.
+template <int N, int G>
+struct Own {
+    static constexpr int E = N / G;                  // channels per lane
+    static constexpr int CH = E >= 8 ? 8 : E;         // channels per chunk
+    static constexpr int M = E / CH;                  // chunks per lane
+    __device__ static int base(int m, int l) { return m * G * CH + l * CH; }
+};
+
+__device__ __forceinline__ void unpack2(uint32_t w, float* d) { d[0] = bf2f_lo(w); d[1] = bf2f_hi(w); }
+
+// This lane's channels of a row of N bf16 / fp32 values.
+template <int N, int G>
+__device__ __forceinline__ void row_bf16(const uint16_t* row, int l, float (&d)[N / G]) {
+    using O = Own<N, G>;
+#pragma unroll
+    for (int m = 0; m < O::M; ++m) {
+        const uint16_t* src = row + O::base(m, l);
+        float* dd = d + m * O::CH;
+        if constexpr (O::CH == 8) {
+            const uint4 w = *reinterpret_cast<const uint4*>(src);
+            unpack2(w.x, dd); unpack2(w.y, dd + 2); unpack2(w.z, dd + 4); unpack2(w.w, dd + 6);
+        } else if constexpr (O::CH == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(src);
+            unpack2(w.x, dd); unpack2(w.y, dd + 2);
+        } else {
+            static_assert(O::CH == 2, "chunk of 2, 4 or 8");
+            unpack2(*reinterpret_cast<const uint32_t*>(src), dd);
+        }
+    }
+}
+template <int N, int G>
+__device__ __forceinline__ void row_f32(const float* row, int l, float (&d)[N / G]) {
+    using O = Own<N, G>;
+#pragma unroll
+    for (int m = 0; m < O::M; ++m) {
+        if constexpr (O::CH == 2) {
+            const float2 a = *reinterpret_cast<const float2*>(row + O::base(m, l));
+            d[2 * m] = a.x; d[2 * m + 1] = a.y;
+        } else {
+#pragma unroll
+            for (int q = 0; q < O::CH / 4; ++q) {
+                const float4 a = *reinterpret_cast<const float4*>(row + O::base(m, l) + 4 * q);
+                float* dd = d + m * O::CH + 4 * q;
+                dd[0] = a.x; dd[1] = a.y; dd[2] = a.z; dd[3] = a.w;
+            }
+        }
+    }
+}
+template <int N, int G, bool B16>
+__device__ __forceinline__ void row_any(const void* row, int l, float (&d)[N / G]) {
+    if constexpr (B16) row_bf16<N, G>(static_cast<const uint16_t*>(row), l, d);
+    else row_f32<N, G>(static_cast<const float*>(row), l, d);
+}
+// Copy this lane's channels of a bf16 / fp32 row, bit for bit.
+template <int N, int G>
+__device__ __forceinline__ void copy_row_bf16(uint16_t* dst, const uint16_t* src, int l) {
+    using O = Own<N, G>;
+#pragma unroll
+    for (int m = 0; m < O::M; ++m) {
+        if constexpr (O::CH == 8)
+            *reinterpret_cast<uint4*>(dst + O::base(m, l)) = *reinterpret_cast<const uint4*>(src + O::base(m, l));
+        else if constexpr (O::CH == 4)
+            *reinterpret_cast<uint2*>(dst + O::base(m, l)) = *reinterpret_cast<const uint2*>(src + O::base(m, l));
+        else
+            *reinterpret_cast<uint32_t*>(dst + O::base(m, l)) = *reinterpret_cast<const uint32_t*>(src + O::base(m, l));
+    }
+}
+template <int N, int G>
+__device__ __forceinline__ void copy_row_f32(float* dst, const float* src, int l) {
+    using O = Own<N, G>;
+#pragma unroll
+    for (int m = 0; m < O::M; ++m) {
+        if constexpr (O::CH == 2) {
+            *reinterpret_cast<float2*>(dst + O::base(m, l)) = *reinterpret_cast<const float2*>(src + O::base(m, l));
+        } else {
+#pragma unroll
+            for (int q = 0; q < O::CH / 4; ++q)
+                reinterpret_cast<float4*>(dst + O::base(m, l))[q] = reinterpret_cast<const float4*>(src + O::base(m, l))[q];
+        }
+    }
+}
+template <int N, int G>
+__device__ __forceinline__ void store_row_f32(float* dst, const float (&v)[N / G], int l) {
+    using O = Own<N, G>;
+#pragma unroll
+    for (int m = 0; m < O::M; ++m) {
+        if constexpr (O::CH == 2) {
+            *reinterpret_cast<float2*>(dst + O::base(m, l)) = make_float2(v[2 * m], v[2 * m + 1]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < O::CH / 4; ++q) {
+                const float* vv = v + m * O::CH + 4 * q;
+                reinterpret_cast<float4*>(dst + O::base(m, l))[q] = make_float4(vv[0], vv[1], vv[2], vv[3]);
+            }
+        }
+    }
+}
+
+template <int E>
+__device__ __forceinline__ float dot(const float (&a)[E], const float (&b)[E]) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) { s0 = fmaf(a[e], b[e], s0); s1 = fmaf(a[e + 1], b[e + 1], s1); }
+    return s0 + s1;
+}
+template <int E>
+__device__ __forceinline__ void axpy(float a, const float (&x)[E], float (&y)[E]) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) y[e] = fmaf(a, x[e], y[e]);
+}
+
+template <int FAM, int K, int V, bool UB16>
+__global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_constant__ StepParams p,
+                                                               int rmax, int ns, int stage_bytes) {
+    constexpr int G = dec_gl(FAM), UPW = 32 / G;
+    constexpr int EK = K / G, EV = V / G, ESZ = UB16 ? 2 : 4;
     extern __shared__ __align__(16) unsigned char smem[];
     const int wpc = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int hw = lane / LPU, l = lane % LPU, gbase = hw * LPU;
+    const int g = lane / G, l = lane % G;
     const int h = blockIdx.y;
-    const int b = (blockIdx.x * wpc + warp) * UPW + hw;
-    const bool active = b < p.B;
-    const long long unit = (long long)b * p.H + h;
-    const int esz = p.sketch_bf16 ? 2 : 4;
+    const int ngroups = (p.B + UPW - 1) / UPW;
+    const int gstride = gridDim.x * wpc;
+    const int g0 = blockIdx.x * wpc + warp;
     const int off = p.off[h], r = p.off[h + 1] - off;
-    const int ubytes = r * V * esz;
-    const UnitSmem L = unit_smem(FAM, K, V, p.p, rmax * V * esz);
+    const int P = p.p;
+    const UnitSmem L = unit_smem(FAM, K, V, P, rmax * V * ESZ);
     const int cbytes = align16(rmax * K * 4);
     const float* csm = reinterpret_cast<const float*>(smem);
     uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + cbytes);
-    unsigned char* ubase = smem + cbytes + 16 + (warp * UPW + hw) * dec_unit_bytes(FAM, K, V, p.p, rmax * V * esz);
-    uint64_t* ubar = reinterpret_cast<uint64_t*>(ubase);
-    unsigned char* sh = ubase + 16;
+    unsigned char* wbase = smem + cbytes + 16 + warp * ns * stage_bytes;
+    const bool stall = p.stall && blockIdx.x == 0 && blockIdx.y == 0 && warp == 0;
+    const float A = FAM == MAMBA2 ? p.A[h] : 0.f;
 
+    auto bar = [&](int s) { return reinterpret_cast<uint64_t*>(wbase + s * stage_bytes); };
+    unsigned pending = 0;      // bit s: stage s has copies in flight
+    auto issue = [&](int it) {                             // this warp's group `it` into stage it % ns
+        const int grp = g0 + it * gstride;
+        if (grp >= ngroups) return;
+        const int s = it % ns;
+        if (l == 0) {
+            const int b = grp * UPW + g;
+            if (b < p.B)
+                stage_unit_bulk<FAM, K, V>(p, (long long)b * p.H + h, wbase + s * stage_bytes + 16 + g * L.total, L,
+                                           static_cast<const char*>(p.sketch) + (b * (long long)p.R + off) * (V * ESZ),
+                                           r * V * ESZ, bar(s), (stall && it == 0 && g == 0) ? 16u : 0u);
+            else
+                mbar_arrive(bar(s));
+        }
+        pending |= 1u << s;
+    };
     if (threadIdx.x == 0) mbar_init(cbar, 1);
-    if (l == 0) mbar_init(ubar, 1);
+    if (lane == 0 && g0 < ngroups)
+        for (int s = 0; s < ns; ++s) mbar_init(bar(s), UPW);
     fence_mbar_init();
     __syncthreads();                                        // the only block barrier
-    const bool stall = p.stall && blockIdx.x == 0 && blockIdx.y == 0;
     if (threadIdx.x == 0) {
-        mbar_expect_tx(cbar, r * K * 4 + (stall ? 16u : 0u));
+        mbar_expect_tx(cbar, r * K * 4);
         if (r > 0) bulk_g2s(smem, p.coef + (long long)off * K, r * K * 4, cbar);
     }
-    if (active && l == 0)
-        stage_unit_bulk<FAM, K, V>(p, unit, sh, L,
-                                   static_cast<const char*>(p.sketch) + (b * (long long)p.R + off) * (V * esz),
-                                   ubytes, ubar, 0u);
-    float tgate = 0.f, tbeta = 0.f;                         // token scalars: plain loads
-    if (active) {
-        if (FAM != KDA) tgate = p.tok_gate[unit];
-        if (FAM != MAMBA2) tbeta = p.tok_beta[unit];
-    }
-    bool ok = mbar_wait(cbar, 0);
-    if (active) ok = mbar_wait(ubar, 0) && ok;
-    if (!ok) {                                              // a bounded wait ran out
-        report_timeout(p.status);
-        mbar_wait(cbar, 0);                                 // give own copies one more bounded wait
-        if (active) mbar_wait(ubar, 0);
-        return;
-    }
-    if (__all_sync(FULL, !active)) return;
+    if (g0 >= ngroups) return;                              // warp 0 always has a group
+    for (int it = 0; it < ns - 1; ++it) issue(it);
+    bool ok = __all_sync(FULL, mbar_wait(cbar, 0));
+    unsigned phases = 0;       // bit s: parity of the next phase of stage s
+    int it = 0;
+    for (int grp = g0; ok && grp < ngroups; ++it, grp += gstride) {
+        const int s = it % ns;
+        issue(it + ns - 1);                                    // its stage was freed by the last group
+        const int b = grp * UPW + g;
+        const bool active = b < p.B;
+        const long long u = (long long)b * p.H + h;
+        float tgate = 0.f, tbeta = 0.f;
+        if (active) {
+            if (FAM != KDA) tgate = p.tok_gate[u];
+            if (FAM != MAMBA2) tbeta = p.tok_beta[u];
+        }
+        ok = __all_sync(FULL, mbar_wait(bar(s), (phases >> s) & 1u));
+        if (!ok) break;
+        phases ^= 1u << s;
+        pending &= ~(1u << s);
+        const unsigned char* sh = wbase + s * stage_bytes + 16 + g * L.total;
+        const uint16_t* kraw = reinterpret_cast<const uint16_t*>(sh + L.kraw);
+        const uint16_t* vraw = reinterpret_cast<const uint16_t*>(sh + L.vraw);
+        const float* graw = reinterpret_cast<const float*>(sh + L.graw);
+        const float* gs = reinterpret_cast<const float*>(sh + L.gs);
+        const float* bs = reinterpret_cast<const float*>(sh + L.bs);
+        const uint16_t* tq = reinterpret_cast<const uint16_t*>(sh + L.tq);
+        const uint16_t* tk = reinterpret_cast<const uint16_t*>(sh + L.tk);
+        const uint16_t* tv = reinterpret_cast<const uint16_t*>(sh + L.tv);
+        const float* tg = reinterpret_cast<const float*>(sh + L.tg);
 
-    // Lanes whose unit lies past the batch take part in the shuffles (on
-    // zeros, inside their own lane group) but store nothing.
-    Tok<K, V, LPU> tk;
-    if (active) {
-        append_token<FAM, K, V, LPU>(p, unit, l, sh, L, tgate, tbeta, tk);
-    } else {
+        // 1. Append the token at ring slot P, bit for bit.
+        if (active) {
+            const long long slot = u * p.W + P;
+            copy_row_bf16<K, G>(p.ring_k + slot * K, tk, l);
+            copy_row_bf16<V, G>(p.ring_v + slot * V, tv, l);
+            if (FAM == KDA) copy_row_f32<K, G>(p.ring_gate + slot * K, tg, l);
+            else if (l == 0) p.ring_gate[u * p.Wg + P] = tgate;
+            if (FAM != MAMBA2 && l == 0) p.ring_beta[u * p.Wg + P] = tbeta;
+        }
+
+        // 2. Backward sweep from the token (j = P) to slot 0: x_P = q,
+        //    x_{j-1} = M_j^T x_j, term += b_j (k_j . x_j) v_j.
+        float x[EK], ob[EV], kj[EK], vj[EV];
+        row_bf16<K, G>(tq, l, x);
+        row_bf16<K, G>(tk, l, kj);
+        row_bf16<V, G>(tv, l, vj);
 #pragma unroll
-        for (int e = 0; e < EK; ++e) { tk.q[e] = 0.f; tk.k[e] = 0.f; tk.g[e] = 1.f; }
+        for (int e = 0; e < EV; ++e) ob[e] = 0.f;
+        if constexpr (FAM == MAMBA2) {
+            // No erase term: every read uses q, scaled by the later decays
+            // (gam = prod_{i > j} a_i).  The rows are independent, so they
+            // are taken 4 at a time: loads, dots and reductions overlap.
+            axpy<EV>(tgate * gsum<G>(dot<EK>(kj, x)), vj, ob);
+            float gam = expf(A * tgate);
+            int j = P - 1;
+            for (; j >= 3; j -= 4) {
+                float d[4], a[4], dt[4];
 #pragma unroll
-        for (int e = 0; e < EV; ++e) tk.v[e] = 0.f;
-        tk.gs = 0.f;
-        tk.b = 0.f;
+                for (int q = 0; q < 4; ++q) {
+                    float kk[EK];
+                    row_bf16<K, G>(kraw + (j - q) * K, l, kk);
+                    d[q] = dot<EK>(kk, x);
+                    dt[q] = gs[j - q];
+                    a[q] = expf(A * dt[q]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) d[q] = gsum<G>(d[q]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float vv[EV];
+                    row_bf16<V, G>(vraw + (j - q) * V, l, vv);
+                    axpy<EV>(dt[q] * gam * d[q], vv, ob);
+                    gam *= a[q];
+                }
+            }
+            for (; j >= 0; --j) {
+                row_bf16<K, G>(kraw + j * K, l, kj);
+                const float dj = gsum<G>(dot<EK>(kj, x));
+                const float dt = gs[j];
+                row_bf16<V, G>(vraw + j * V, l, vj);
+                axpy<EV>(dt * gam * dj, vj, ob);
+                gam *= expf(A * dt);
+            }
+#pragma unroll
+            for (int e = 0; e < EK; ++e) x[e] *= gam;          // q~ = (prod a) q
+        } else {
+            // Delta rule: each row's read depends on the previous erase, so
+            // the rows run in order; the next row is loaded while the current
+            // one is reduced.
+            float gam = 1.f;                                   // GDN: x_j = gam * y_j
+            float aj[EK];
+            {
+                const float t = tbeta * gsum<G>(dot<EK>(kj, x));
+                axpy<EV>(t, vj, ob);
+                if constexpr (FAM == GDN) {
+                    axpy<EK>(-t, kj, x);
+                    gam = tgate;
+                } else {
+                    row_f32<K, G>(tg, l, aj);
+#pragma unroll
+                    for (int e = 0; e < EK; ++e) x[e] = aj[e] * fmaf(-t, kj[e], x[e]);
+                }
+            }
+            if (P > 0) {
+                row_bf16<K, G>(kraw + (P - 1) * K, l, kj);
+                row_bf16<V, G>(vraw + (P - 1) * V, l, vj);
+            }
+            for (int j = P - 1; j >= 0; --j) {
+                float kc[EK], vc[EV];
+#pragma unroll
+                for (int e = 0; e < EK; ++e) kc[e] = kj[e];
+#pragma unroll
+                for (int e = 0; e < EV; ++e) vc[e] = vj[e];
+                const float bj = bs[j];
+                if constexpr (FAM == KDA) row_f32<K, G>(graw + j * K, l, aj);
+                const float part = dot<EK>(kc, x);
+                if (j > 0) {
+                    row_bf16<K, G>(kraw + (j - 1) * K, l, kj);
+                    row_bf16<V, G>(vraw + (j - 1) * V, l, vj);
+                }
+                const float t = bj * gsum<G>(part);
+                if constexpr (FAM == GDN) {
+                    axpy<EV>(gam * t, vc, ob);
+                    axpy<EK>(-t, kc, x);
+                    gam *= gs[j];
+                } else {
+                    axpy<EV>(t, vc, ob);
+#pragma unroll
+                    for (int e = 0; e < EK; ++e) x[e] = aj[e] * fmaf(-t, kc[e], x[e]);
+                }
+            }
+            if constexpr (FAM == GDN) {
+#pragma unroll
+                for (int e = 0; e < EK; ++e) x[e] *= gam;
+            }
+        }
+
+        // 3. Coefficients c = C q~ and the sketched read o = U c + term,
+        //    4 rows of C at a time.
+        const unsigned char* us = sh + L.ush;
+        int i = 0;
+        for (; i + 4 <= r; i += 4) {
+            float c[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float ci[EK];
+                row_f32<K, G>(csm + (i + q) * K, l, ci);
+                c[q] = dot<EK>(ci, x);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) c[q] = gsum<G>(c[q]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float ui[EV];
+                row_any<V, G, UB16>(us + (i + q) * V * ESZ, l, ui);
+                axpy<EV>(c[q], ui, ob);
+            }
+        }
+        for (; i < r; ++i) {
+            float ci[EK], ui[EV];
+            row_f32<K, G>(csm + i * K, l, ci);
+            const float c = gsum<G>(dot<EK>(ci, x));
+            row_any<V, G, UB16>(us + i * V * ESZ, l, ui);
+            axpy<EV>(c, ui, ob);
+        }
+        if (active) store_row_f32<V, G>(p.out + u * V, ob, l);
+        __syncwarp();                                          // stage s is free again
     }
-    float x[EK], ob[EV];
-    window_read<FAM, K, V, LPU>(p, h, l, gbase, sh, L, tk, x, ob);
-    const bool bf16 = p.sketch_bf16;
-    for (int i0 = 0; i0 < r; i0 += 32) {
-        const int nr = min(32, r - i0);
-        const float* cs = csm + i0 * K;
-        const unsigned char* us = sh + L.ush + i0 * V * esz;
-        auto loadU = [&](int i, float (&u)[EV]) {
-            if (bf16) ld_bf16<EV>(reinterpret_cast<const uint16_t*>(us) + i * V + l * EV, u);
-            else ld_f32<EV>(reinterpret_cast<const float*>(us) + i * V + l * EV, u);
-        };
-        if (nr <= 8) readout<8, K, V, LPU>(cs, nr, l, gbase, x, ob, loadU);
-        else if (nr <= 16) readout<16, K, V, LPU>(cs, nr, l, gbase, x, ob, loadU);
-        else readout<32, K, V, LPU>(cs, nr, l, gbase, x, ob, loadU);
+    if (!ok) {                                                 // a bounded wait ran out
+        if (lane == 0) report_timeout(p.status);
+        for (int t = 0; t < ns; ++t)                           // own copies: one more bounded wait
+            if ((pending >> t) & 1u) mbar_wait(bar(t), (phases >> t) & 1u);
+        if (warp == 0) mbar_wait(cbar, 0);
     }
-    if (active) st_f32<EV>(p.out + unit * V + l * EV, ob);
 }
 
 // ---------------------------------------------------------------------------
@@ -572,25 +848,33 @@ __global__ void __launch_bounds__(128) replay_kernel(const __grid_constant__ Ste
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-int decode_bytes(int fam, int K, int V, int P, int rmax, int esz, int wpc) {
-    return align16(rmax * K * 4) + 16 + wpc * (32 / DEC_LPU) * dec_unit_bytes(fam, K, V, P, rmax * V * esz);
+int decode_stage(int fam, int K, int V, int P, int rmax, int esz) {
+    return dec_stage_bytes(fam, K, V, P, rmax * V * esz);
+}
+
+template <int FAM, int K, int V, bool UB16>
+cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
+    constexpr int esz = UB16 ? 2 : 4, upw = 32 / dec_gl(FAM);
+    const int stage = decode_stage(FAM, K, V, p.p, rmax, esz);
+    const int cpart = align16(rmax * K * 4) + 16;
+    if (cpart + stage > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
+    int wpc = DEC_WARPS;
+    while (wpc > 1 && cpart + wpc * stage > SMEM_LIMIT) --wpc;
+    const int bytes = cpart + wpc * stage;
+    auto kern = decode_kernel<FAM, K, V, UB16>;
+    static KernelCache kc;
+    cudaError_t e = ensure_smem(kern, kc, bytes);
+    if (e != cudaSuccess) return e;
+    const long long groups = (p.B + upw - 1) / upw;
+    const long long nb = (groups + wpc - 1) / wpc;          // one group per warp
+    kern<<<dim3(unsigned(nb), unsigned(p.H)), dim3(wpc * 32), bytes, stream>>>(p, rmax, 1, stage);
+    return cudaGetLastError();
 }
 
 template <int FAM, int K, int V>
 cudaError_t decode_t(const StepParams& p, int rmax, cudaStream_t stream) {
-    const int esz = p.sketch_bf16 ? 2 : 4;
-    const int upw = 32 / DEC_LPU;
-    int wpc = DEC_MAX_WARPS;
-    while (wpc > 1 && (decode_bytes(FAM, K, V, p.p, rmax, esz, wpc) > SMEM_LIMIT || (wpc - 1) * upw >= p.B)) --wpc;
-    const int bytes = decode_bytes(FAM, K, V, p.p, rmax, esz, wpc);
-    if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
-    const int upc = wpc * upw;
-    const dim3 grid(unsigned((p.B + upc - 1) / upc), unsigned(p.H));
-    auto kern = decode_kernel<FAM, K, V>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, dim3(wpc * 32), bytes, stream>>>(p, rmax);
-    return cudaGetLastError();
+    return p.sketch_bf16 ? decode_launch<FAM, K, V, true>(p, rmax, stream)
+                         : decode_launch<FAM, K, V, false>(p, rmax, stream);
 }
 
 template <int FAM, int K, int V>
@@ -602,7 +886,8 @@ cudaError_t replay_t(const StepParams& p, cudaStream_t stream) {
     const long long units = (long long)p.B * p.H;
     const long long grid = (units + hpc - 1) / hpc;
     auto kern = replay_kernel<FAM, K, V>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, hpc * per_head);
+    static KernelCache kc;
+    cudaError_t e = ensure_smem(kern, kc, hpc * per_head);
     if (e != cudaSuccess) return e;
     kern<<<dim3(unsigned(grid)), dim3(hpc * V), hpc * per_head, stream>>>(p);
     return cudaGetLastError();
@@ -619,7 +904,7 @@ cudaError_t launch_replay(int family, int dk, int dv, const StepParams& p, cudaS
 }
 
 int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz) {
-    return decode_bytes(family, dk, dv, P, rmax, esz, 1);
+    return align16(rmax * dk * 4) + 16 + decode_stage(family, dk, dv, P, rmax, esz);
 }
 
 }  // namespace ss

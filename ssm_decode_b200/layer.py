@@ -6,6 +6,8 @@ is the one include/sketchssm.h documents.
 """
 from __future__ import annotations
 
+import weakref
+
 import numpy as np
 
 from . import binding as B
@@ -18,6 +20,16 @@ def _dev(x, dtype, device):
             x = x.view(np.int16)
         x = torch.from_numpy(np.ascontiguousarray(x))
     return x.to(device=device, dtype=dtype).contiguous()
+
+
+class Token(dict):
+    """One step's inputs on the device (q, k, v, gate, beta tensors).  The
+    C-ABI argument structs built from it are cached per layer, so a step
+    costs one library call; update the tensors in place (copy_) to reuse it."""
+
+    def __init__(self, *a, **kw):
+        super().__init__(*a, **kw)
+        self._io = {}
 
 
 class DecodeLayer:
@@ -47,6 +59,9 @@ class DecodeLayer:
         self.out = z(batch, heads, dv)
         self.status = torch.zeros(4, dtype=torch.int32, device=device)   # device status word (+ padding)
         self.sketch_dtype = sketch_dtype
+        # The buffers stay in place for the layer's life (load() copies into
+        # them), so their argument structs are built once.
+        self._bufs = {w: self._make_bufs(w) for w in (True, False)}
 
     # -- data -------------------------------------------------------------------
     def load(self, state=None, basis=None, coef=None, A=None):
@@ -62,20 +77,31 @@ class DecodeLayer:
     def token(self, inp):
         """Move one step's raw inputs (numpy or torch) to the device."""
         import torch
-        t = {k: _dev(inp[k], torch.int16, self.device) for k in ("q", "k", "v")}
+        t = Token((k, _dev(inp[k], torch.int16, self.device)) for k in ("q", "k", "v"))
         t["gate"] = _dev(inp["gate"], torch.float32, self.device)
         t["beta"] = _dev(inp["beta"], torch.float32, self.device)
         return t
 
     def bufs(self, with_sketch=True):
+        return self._bufs[bool(with_sketch)]
+
+    def _make_bufs(self, with_sketch):
         return B.make_buffers(self.state, self.ring_k, self.ring_v, self.ring_gate, self.ring_beta,
                               self.sketch if with_sketch else None, self.basis, self.coef, self.A,
                               self.status)
 
     def io(self, tok, out=None):
+        cache = getattr(tok, "_io", None) if out is None else None
+        if cache is not None:
+            hit = cache.get(id(self))
+            if hit is not None and hit[0]() is self:      # guard against a reused id()
+                return hit[1]
         beta = tok["beta"] if self.family != B.SS_MAMBA2 else None
-        return B.make_step_io(tok["q"], tok["k"], tok["v"], tok["gate"], beta,
-                              self.out if out is None else out)
+        io = B.make_step_io(tok["q"], tok["k"], tok["v"], tok["gate"], beta,
+                            self.out if out is None else out)
+        if cache is not None:
+            cache[id(self)] = (weakref.ref(self), io)
+        return io
 
     @property
     def phase(self):

@@ -60,6 +60,25 @@ def test_create_rejects_bad_shapes(L):
     assert code(window=1) == B.SS_OK and code(ranks=[0, 64, 1]) == B.SS_OK
 
 
+def test_supported_rank_and_window_range(L):
+    """The shared-memory limits stated for ss_create: every rank up to 64 at
+    W <= 16 and up to 32 at W <= 32 is accepted, for every family, shape and
+    sketch type; rank 128 with dk = dv = 128 at W = 32 is not."""
+    def ok(fam, dk, dv, W, r, sk):
+        try:
+            B.Plan(fam, 2, 2, dk, dv, W, [r, 1], sk)
+            return True
+        except B.SSError as e:
+            assert e.status == B.SS_ERR_UNSUPPORTED
+            return False
+    for fam in (B.SS_MAMBA2, B.SS_GDN, B.SS_KDA):
+        for dk, dv in ((64, 64), (64, 128), (128, 64), (128, 128)):
+            for sk in (B.SS_F32, B.SS_BF16):
+                assert ok(fam, dk, dv, 16, min(64, dk), sk)
+                assert ok(fam, dk, dv, 32, 32, sk)
+        assert not ok(fam, 128, 128, 32, 128, B.SS_F32)
+
+
 def test_buffer_sizes(L):
     p = B.Plan(B.SS_KDA, 3, 2, 128, 64, 6, [5, 7], B.SS_BF16)
     s = B.ss_buffer_sizes(p)
