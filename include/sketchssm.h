@@ -161,8 +161,8 @@ typedef struct {
  * memory than one CTA has: the flush stages the window's keys, values and
  * decays plus the basis rows of one head, and the decode step stages, per
  * warp, the window's ring slots and sketch rows plus the head's map C
- * (rmax x dk fp32), so very large ranks with long windows do not fit (e.g.
- * rank 128 with dk = dv = 128 and W = 32).  Every rank up to 64 at W <= 16,
+ * (rmax x dk fp32), so very large ranks with long windows may not fit (KDA
+ * with rank 128, dk = dv = 128 and W = 32 does not).  Every rank up to 64 at W <= 16,
  * and up to 32 at W <= 32, is supported.  The plan starts at phase 0
  * with no valid sketch. */
 ss_status ss_create(const ss_config* cfg, ss_plan** out);
@@ -221,8 +221,9 @@ ss_status ss_traffic_bytes(const ss_plan* plan, int32_t op, int32_t tau, ss_traf
 /* Number of kernels this library has launched in this process. */
 uint64_t ss_launch_count(void);
 
-/* Testing hook.  With stall != 0 the next ss_decode_step or ss_replay_step of
- * this plan makes one CTA expect more bytes than its bulk copies deliver, so
+/* Testing hook.  With stall != 0 the next launching call of this plan
+ * (ss_prime, ss_decode_step, ss_flush, ss_exact_step or ss_replay_step)
+ * makes one CTA expect more bytes than its bulk copies deliver, so
  * that CTA's bounded wait runs out after about a second: it sets
  * SS_DEVICE_TIMEOUT in bufs->status and returns, leaving its outputs
  * incomplete; the rest of the launch completes.  The hook clears itself

@@ -250,6 +250,7 @@ ss_status ss_prime(ss_plan* pl, const ss_buffers* b, ss_stream stream) {
     CHECK(check_status(b));
     ss::FlushParams p = flush_params(pl, b, nullptr);
     p.n_ring = 0; p.has_token = 0; p.do_sketch = 1;
+    p.stall = take_stall(pl);
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
                                     reinterpret_cast<cudaStream_t>(stream)), "prime"));
     pl->sketch_valid = 1;
@@ -293,6 +294,7 @@ ss_status ss_flush(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_st
     p.n_ring = pl->phase;
     p.has_token = io != nullptr;
     p.do_sketch = sk;
+    p.stall = take_stall(pl);
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
                                     reinterpret_cast<cudaStream_t>(stream)), "flush"));
     pl->phase = 0;
@@ -310,6 +312,7 @@ ss_status ss_exact_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
     CHECK(check_status(b));
     ss::FlushParams p = flush_params(pl, b, io);
     p.n_ring = 0; p.has_token = 1; p.do_sketch = 0;
+    p.stall = take_stall(pl);
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, 0,
                                     reinterpret_cast<cudaStream_t>(stream)), "exact"));
     pl->sketch_valid = 0;

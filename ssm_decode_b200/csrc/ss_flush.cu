@@ -14,8 +14,15 @@
 // ...  A head is held by 2*dv threads, dv/4 column groups x 8 row blocks;
 // each thread keeps a (dk/8) x 4 tile as fp32 pairs of adjacent columns, so
 // tile loads/stores are 16-byte accesses and every update is a packed
-// fp32x2 FMA.  While a head is computed from registers, cp.async brings the
-// next head's state tile and window into shared memory.
+// fp32x2 FMA.
+//
+// Memory.  One thread moves everything with bulk asynchronous copies
+// (cp.async.bulk) that complete on mbarriers: the next head's state tile
+// (one copy, issued once the current tile is in registers) and the next
+// head's window -- keys, values, decays, query and basis rows -- issued once
+// the current head's updates are done (the read-out works from its own copy
+// of the basis).  Every wait is bounded: when one runs out the kernel sets
+// SS_DEVICE_TIMEOUT in the caller's status word and returns.
 //
 // Scaled state.  Write Gamma_j for the product of the decays since the last
 // fold (a scalar for Mamba-2 and GDN, a dk-vector for KDA) and keep
@@ -46,25 +53,27 @@ struct FS {
     static constexpr int KD = kd_len(K);
 };
 
-// Per-CTA shared-memory layout (byte offsets).  [tile .. ts] is written by
-// the prefetch of the next head; the rest is the current head's working set.
+// Per-CTA shared-memory layout (byte offsets).  The window (keys, values,
+// decays, query and basis rows of one head) is refilled for the next head
+// as soon as the current head's updates are done; the read-out then works
+// from pt, the extended basis [Omega_h | q | 0 ...] built from it.
 struct FlushLayout {
-    int tile, kraw, vraw, graw, sg, sb, tq, ts, braw;
-    int kd, ku, fin, sc, pt, meta, total;
+    int tile, kraw, vraw, graw, sg, sb, tq, braw;
+    int kd, ku, fin, sc, pt, meta, bars, total;
 };
 
 __host__ __device__ inline FlushLayout flush_layout(int fam, int K, int V, int n, int rpad) {
     const int KD = kd_len(K);
+    const int n4 = (n + 3) & ~3;
     FlushLayout L;
     int o = 0;
     L.tile = o; o += align16(K * V * 4);
     L.kraw = o; o += align16(n * K * 2);
     L.vraw = o; o += align16(n * V * 2);
     L.graw = o; o += align16(fam == KDA ? n * K * 4 : 0);
-    L.sg = o;   o += align16(SS_MAX_WINDOW * 4);
-    L.sb = o;   o += align16(SS_MAX_WINDOW * 4);
+    L.sg = o;   o += align16(fam == KDA ? 0 : n4 * 4);
+    L.sb = o;   o += align16(fam == MAMBA2 ? 0 : n4 * 4);
     L.tq = o;   o += align16(K * 2);
-    L.ts = o;   o += 16;
     L.braw = o; o += align16(rpad * K * 4);
     L.kd = o;   o += align16(n * KD * 4);
     L.ku = o;   o += align16(fam == KDA ? n * KD * 4 : 0);
@@ -72,6 +81,7 @@ __host__ __device__ inline FlushLayout flush_layout(int fam, int K, int V, int n
     L.sc = o;   o += align16((n + 1) * 16);
     L.pt = o;   o += align16(rpad * K * 4);
     L.meta = o; o += 16;
+    L.bars = o; o += 16;                        // tile, window
     L.total = o;
     return L;
 }
@@ -83,34 +93,41 @@ __device__ __forceinline__ int kdup(int c) {
     return (c / R) * (2 * R + 4) + (c % R) * 2;
 }
 
-template <int K, int V>
-__device__ __forceinline__ void prefetch_tile(const FlushParams& p, long long u, float* tile, int t) {
-    stage(tile, p.state + u * (long long)(K * V), K * V * 4, t, FS<K, V>::T);
+// Bytes of one head's window copies (what the window mbarrier expects).
+template <int FAM, int K, int V>
+__device__ __forceinline__ unsigned window_bytes(const FlushParams& p, int r) {
+    const int n4r = (p.n_ring + 3) & ~3;
+    unsigned b = p.n_ring * (K * 2 + V * 2) + r * K * 4;
+    if (FAM == KDA) b += p.n_ring * K * 4;
+    else if (p.n_ring > 0) b += n4r * 4;
+    if (FAM != MAMBA2 && p.n_ring > 0) b += n4r * 4;
+    if (p.has_token) b += K * 2 + V * 2 + K * 2 + (FAM == KDA ? K * 4 : 0);
+    return b;
 }
 
+// Issue (one thread) the bulk copies of head u's window.
 template <int FAM, int K, int V>
-__device__ __forceinline__ void prefetch_window(const FlushParams& p, long long u, unsigned char* sh,
-                                                const FlushLayout& L, int t) {
-    constexpr int T = FS<K, V>::T;
+__device__ __forceinline__ void issue_window(const FlushParams& p, long long u, unsigned char* base,
+                                             const FlushLayout& L, uint64_t* bar, unsigned extra) {
+    const int h = int(u % p.H);
+    const int r = p.do_sketch ? p.off[h + 1] - p.off[h] : 0;
+    mbar_expect_tx(bar, window_bytes<FAM, K, V>(p, r) + extra);
     const long long ring_row = u * p.W;
-    stage(sh + L.kraw, p.ring_k + ring_row * K, p.n_ring * K * 2, t, T);
-    stage(sh + L.vraw, p.ring_v + ring_row * V, p.n_ring * V * 2, t, T);
-    if (FAM == KDA) stage(sh + L.graw, p.ring_gate + ring_row * K, p.n_ring * K * 4, t, T);
-    const int n4 = (p.n_ring + 3) & ~3;
-    if (FAM != KDA) stage(sh + L.sg, p.ring_gate + u * p.Wg, n4 * 4, t, T);
-    if (FAM != MAMBA2) stage(sh + L.sb, p.ring_beta + u * p.Wg, n4 * 4, t, T);
+    const int nr = p.n_ring, n4r = (nr + 3) & ~3;
+    if (nr > 0) {
+        bulk_g2s(base + L.kraw, p.ring_k + ring_row * K, nr * K * 2, bar);
+        bulk_g2s(base + L.vraw, p.ring_v + ring_row * V, nr * V * 2, bar);
+        if (FAM == KDA) bulk_g2s(base + L.graw, p.ring_gate + ring_row * K, nr * K * 4, bar);
+        else bulk_g2s(base + L.sg, p.ring_gate + u * p.Wg, n4r * 4, bar);
+        if (FAM != MAMBA2) bulk_g2s(base + L.sb, p.ring_beta + u * p.Wg, n4r * 4, bar);
+    }
     if (p.has_token) {
-        stage(sh + L.kraw + p.n_ring * K * 2, p.tok_k + u * K, K * 2, t, T);
-        stage(sh + L.vraw + p.n_ring * V * 2, p.tok_v + u * V, V * 2, t, T);
-        if (FAM == KDA) stage(sh + L.graw + p.n_ring * K * 4, p.tok_gate + u * K, K * 4, t, T);
-        stage(sh + L.tq, p.tok_q + u * K, K * 2, t, T);
-        if (t == 0 && FAM != KDA) cp_async4(sh + L.ts, p.tok_gate + u);
-        if (t == 1 && FAM != MAMBA2) cp_async4(sh + L.ts + 4, p.tok_beta + u);
+        bulk_g2s(base + L.kraw + nr * K * 2, p.tok_k + u * K, K * 2, bar);
+        bulk_g2s(base + L.vraw + nr * V * 2, p.tok_v + u * V, V * 2, bar);
+        if (FAM == KDA) bulk_g2s(base + L.graw + nr * K * 4, p.tok_gate + u * K, K * 4, bar);
+        bulk_g2s(base + L.tq, p.tok_q + u * K, K * 2, bar);
     }
-    if (p.do_sketch) {
-        const int h = int(u % p.H);
-        stage(sh + L.braw, p.basis + (long long)p.off[h] * K, (p.off[h + 1] - p.off[h]) * K * 4, t, T);
-    }
+    if (r > 0) bulk_g2s(base + L.braw, p.basis + (long long)p.off[h] * K, r * K * 4, bar);
 }
 
 // Sequential decay scan with folds, one warp, channels lane + 32 m
@@ -171,107 +188,68 @@ __device__ void scan_with_folds(int n, int n_ring, const float* al_in, const flo
     if (lane == 0) meta[0] = mask;
 }
 
-template <int FAM, int K, int V>
-__global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __grid_constant__ FlushParams p, int rpad) {
-    using S = FS<K, V>;
-    constexpr int R = S::R, KB = S::KB, KD = S::KD;
-    extern __shared__ __align__(16) unsigned char smem[];
 
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int cgw = lane & 3, rb = lane >> 2;
-    const int c0 = warp * 16 + cgw * 4;          // first of this thread's 4 columns
-    const int row0 = rb * R;                     // first of this thread's R rows
-    const long long units = (long long)p.B * p.H;
-    const int n = p.n_ring + p.has_token;
-    const FlushLayout L = flush_layout(FAM, K, V, n, rpad);
-    float* tile = reinterpret_cast<float*>(smem + L.tile);
-    const uint16_t* kraw = reinterpret_cast<const uint16_t*>(smem + L.kraw);
-    const uint16_t* vraw = reinterpret_cast<const uint16_t*>(smem + L.vraw);
-    const float* graw = reinterpret_cast<const float*>(smem + L.graw);
-    const float* sg = reinterpret_cast<const float*>(smem + L.sg);
-    const float* sb = reinterpret_cast<const float*>(smem + L.sb);
-    const uint16_t* tq = reinterpret_cast<const uint16_t*>(smem + L.tq);
-    const float* ts = reinterpret_cast<const float*>(smem + L.ts);
+// Per-head preparation (phase 2): duplicated keys (and for KDA the scaled
+// keys and their scan), the scalar-decay coefficients, and the rows of the
+// extended basis [Omega_h | q | 0 ...] after the basis rows.  Returns nothing;
+// sc[], kd[], ku[], fin[] and meta[0] are written for the update loop.
+template <int FAM, int K, int V>
+__device__ __forceinline__ void prepare_head(const FlushParams& p, int h, int n, int r_h, int rpad,
+                                             unsigned char* slot, const FlushLayout& L,
+                                             unsigned char* smem, float tgate, float tbeta, int t) {
+    using S = FS<K, V>;
+    constexpr int T = S::T, KD = S::KD, R = S::R;
+    const int lane = t & 31, warp = t >> 5;
+    const uint16_t* kraw = reinterpret_cast<const uint16_t*>(slot + L.kraw);
+    const float* graw = reinterpret_cast<const float*>(slot + L.graw);
+    const float* sg = reinterpret_cast<const float*>(slot + L.sg);
+    const float* sb = reinterpret_cast<const float*>(slot + L.sb);
+    const uint16_t* tq = reinterpret_cast<const uint16_t*>(slot + L.tq);
+    const float* braw = reinterpret_cast<const float*>(slot + L.braw);
+    float* pt = reinterpret_cast<float*>(smem + L.pt);
     float* kd = reinterpret_cast<float*>(smem + L.kd);
     float* ku = reinterpret_cast<float*>(smem + L.ku);
     float* fin = reinterpret_cast<float*>(smem + L.fin);
     float4* sc = reinterpret_cast<float4*>(smem + L.sc);
-    float* pt = reinterpret_cast<float*>(smem + L.pt);
-    const float* braw = reinterpret_cast<const float*>(smem + L.braw);
     unsigned* meta = reinterpret_cast<unsigned*>(smem + L.meta);
 
-    long long u = blockIdx.x;
-    if (u < units) {
-        prefetch_tile<K, V>(p, u, tile, t);
-        prefetch_window<FAM, K, V>(p, u, smem, L, t);
+    // the extended basis [Omega_h | q | 0 ...], rpad rows of dk floats
+    for (int idx = t * 4; idx < rpad * K; idx += T * 4) {
+        const int e = idx / K, c = idx % K;
+        float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e < r_h) {
+            val = *reinterpret_cast<const float4*>(braw + idx);
+        } else if (e == r_h && p.has_token) {
+            const uint2 w = *reinterpret_cast<const uint2*>(tq + c);
+            val = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
+        }
+        *reinterpret_cast<float4*>(pt + idx) = val;
     }
-    cp_async_commit();
 
-    for (; u < units; u += gridDim.x) {
-        cp_async_wait_all();
-        __syncthreads();                                              // (A) head u staged
-        const int h = int(u % p.H);
-        const long long b = u / p.H;
-        const long long un = u + gridDim.x;
-
-        // 1. This thread's tile, pairs of adjacent columns.
-        float2 s[R][2];
-        {
-            const float* tb = tile + row0 * V + c0;
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-                const float4 a = *reinterpret_cast<const float4*>(tb + i * V);
-                s[i][0] = make_float2(a.x, a.y);
-                s[i][1] = make_float2(a.z, a.w);
-            }
+    if (FAM != KDA) {
+        // duplicated keys, 8 channels (one 16-byte row piece) per step; the 8
+        // channels of a piece lie in one row block (dk/8 >= 8)
+        static_assert(R % 8 == 0, "row blocks of whole 8-channel pieces");
+        for (int pc = t; pc < n * (K / 8); pc += T) {
+            const int j = pc / (K / 8), c0 = (pc % (K / 8)) * 8;
+            const uint4 w = *reinterpret_cast<const uint4*>(kraw + j * K + c0);
+            float4* d = reinterpret_cast<float4*>(kd + j * KD + kdup<K>(c0));
+            const float k0 = bf2f_lo(w.x), k1 = bf2f_hi(w.x), k2 = bf2f_lo(w.y), k3 = bf2f_hi(w.y);
+            const float k4 = bf2f_lo(w.z), k5 = bf2f_hi(w.z), k6 = bf2f_lo(w.w), k7 = bf2f_hi(w.w);
+            d[0] = make_float4(k0, k0, k1, k1);
+            d[1] = make_float4(k2, k2, k3, k3);
+            d[2] = make_float4(k4, k4, k5, k5);
+            d[3] = make_float4(k6, k6, k7, k7);
         }
-
-        // 2. Per-head preparation: keys, decays, coefficients, extended basis.
-        const int r_h = p.do_sketch ? p.off[h + 1] - p.off[h] : 0;
-        const int next = r_h + p.has_token;                           // columns of [Omega_h | q]
-        const int nch = (next + 3) / 4;
-        bool bad = false;
-        if (t < K) {                                                  // one channel per thread
-            const int c = t;
-            const int pc = kdup<K>(c);
-            if (FAM == KDA) {
-                float gam = 1.f;
-                for (int j = 0; j < n; ++j) {
-                    const float g = gam * graw[j * K + c];
-                    bad |= !(g >= GAMMA_LO && g <= GAMMA_HI);
-                    gam = g;
-                    const float kv = bf2f(kraw[j * K + c]);
-                    *reinterpret_cast<float2*>(kd + j * KD + pc) = dup2(g * kv);
-                    *reinterpret_cast<float2*>(ku + j * KD + pc) = dup2(kv * __frcp_rn(g));
-                }
-                *reinterpret_cast<float2*>(fin + pc) = dup2(gam);
-            } else {
-#pragma unroll 4
-                for (int j = 0; j < n; ++j)
-                    *reinterpret_cast<float2*>(kd + j * KD + pc) = dup2(bf2f(kraw[j * K + c]));
-            }
-        }
-        // extended basis [Omega_h | q | 0 ...] rows, dk floats each
-        for (int idx = t * 4; idx < nch * 4 * K; idx += 2 * V * 4) {
-            const int e = idx / K, c = idx % K;
-            float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (e < r_h) {
-                val = *reinterpret_cast<const float4*>(braw + e * K + c);
-            } else if (e == r_h && p.has_token) {
-                const uint2 w = *reinterpret_cast<const uint2*>(tq + c);
-                val = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
-            }
-            *reinterpret_cast<float4*>(pt + e * K + c) = val;
-        }
-        if (FAM != KDA && warp == 0) {
+        if (warp == 0) {
             // scalar decays: lane j holds (a_j, b_j); running products by a
             // log-step scan; folds only if a product leaves the range.
             float al = 1.f, bl = 0.f;
             if (lane < n) {
                 const bool tok = lane >= p.n_ring;
-                const float g = tok ? ts[0] : sg[lane];
+                const float g = tok ? tgate : sg[lane];
                 if (FAM == MAMBA2) { bl = g; al = expf(g * p.A[h]); }
-                else { al = g; bl = tok ? ts[1] : sb[lane]; }
+                else { al = g; bl = tok ? tbeta : sb[lane]; }
             }
             float G = al;
 #pragma unroll
@@ -292,53 +270,125 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
                 scan_with_folds<FAM, K>(n, p.n_ring, al_s, bl_s, kraw, graw, kd, ku, fin, sc, meta, lane);
             }
         }
-        if (FAM == KDA) {
-            const int any_bad = __syncthreads_or(bad);
-            if (warp == 0 && lane < n) {
-                const float bl = lane >= p.n_ring ? ts[1] : sb[lane];
-                if (!any_bad) sc[lane] = make_float4(bl, 1.f, 0.f, 0.f);
+    } else {
+        bool bad = false;
+        if (t < K) {                                          // one channel per thread
+            const int c = t;
+            const int pc = kdup<K>(c);
+            float gam = 1.f;
+            for (int j = 0; j < n; ++j) {
+                const float g = gam * graw[j * K + c];
+                bad |= !(g >= GAMMA_LO && g <= GAMMA_HI);
+                gam = g;
+                const float kv = bf2f(kraw[j * K + c]);
+                *reinterpret_cast<float2*>(kd + j * KD + pc) = dup2(g * kv);
+                *reinterpret_cast<float2*>(ku + j * KD + pc) = dup2(kv * __frcp_rn(g));
             }
-            if (any_bad && warp == 0) {
-                __shared__ float bl_s[SS_MAX_WINDOW];
-                bl_s[lane] = lane < n ? (lane >= p.n_ring ? ts[1] : sb[lane]) : 0.f;
-                __syncwarp();
-                scan_with_folds<FAM, K>(n, p.n_ring, nullptr, bl_s, kraw, graw, kd, ku, fin, sc, meta, lane);
-            } else if (warp == 0 && lane == 0) {
-                meta[0] = 0u;
+            *reinterpret_cast<float2*>(fin + pc) = dup2(gam);
+        }
+        const int any_bad = __syncthreads_or(bad);
+        if (warp == 0 && lane < n) {
+            const float bl = lane >= p.n_ring ? tbeta : sb[lane];
+            if (!any_bad) sc[lane] = make_float4(bl, 1.f, 0.f, 0.f);
+        }
+        if (any_bad && warp == 0) {
+            __shared__ float bl_s[SS_MAX_WINDOW];
+            bl_s[lane] = lane < n ? (lane >= p.n_ring ? tbeta : sb[lane]) : 0.f;
+            __syncwarp();
+            scan_with_folds<FAM, K>(n, p.n_ring, nullptr, bl_s, kraw, graw, kd, ku, fin, sc, meta, lane);
+        } else if (warp == 0 && lane == 0) {
+            meta[0] = 0u;
+        }
+    }
+}
+
+template <int FAM, int K, int V>
+__global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __grid_constant__ FlushParams p, int rpad) {
+    using S = FS<K, V>;
+    constexpr int R = S::R, KB = S::KB, KD = S::KD;
+    extern __shared__ __align__(16) unsigned char smem[];
+
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int cgw = lane & 3, rb = lane >> 2;
+    const int c0 = warp * 16 + cgw * 4;          // first of this thread's 4 columns
+    const int row0 = rb * R;                     // first of this thread's R rows
+    const long long units = (long long)p.B * p.H;
+    const int n = p.n_ring + p.has_token;
+    const FlushLayout L = flush_layout(FAM, K, V, n, rpad);
+    const float* tile = reinterpret_cast<const float*>(smem + L.tile);
+    const float* kd = reinterpret_cast<const float*>(smem + L.kd);
+    const float* ku = reinterpret_cast<const float*>(smem + L.ku);
+    const float* fin = reinterpret_cast<const float*>(smem + L.fin);
+    const float4* sc = reinterpret_cast<const float4*>(smem + L.sc);
+    const unsigned* meta = reinterpret_cast<const unsigned*>(smem + L.meta);
+    uint64_t* tbar = reinterpret_cast<uint64_t*>(smem + L.bars);
+    uint64_t* wbar = tbar + 1;                   // the window
+    const bool stall = p.stall && blockIdx.x == 0;
+
+    // Only thread 0 issues copies; it tracks which barriers have copies in flight.
+    unsigned pending = 0;                        // bit 0: tile, bit 1: window
+    long long u = blockIdx.x;
+    if (t == 0) {
+        mbar_init(tbar, 1);
+        mbar_init(wbar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (t == 0 && u < units) {
+        mbar_expect_tx(tbar, K * V * 4);
+        bulk_g2s(smem + L.tile, p.state + u * (long long)(K * V), K * V * 4, tbar);
+        issue_window<FAM, K, V>(p, u, smem, L, wbar, stall ? 16u : 0u);
+        pending = 1u | 2u;
+    }
+
+    bool ok = true;
+    for (int k = 0; u < units; ++k, u += gridDim.x) {
+        const int h = int(u % p.H);
+        const long long b = u / p.H;
+        const long long un = u + gridDim.x;
+        float tgate = 0.f, tbeta = 0.f;                           // the token's scalar inputs
+        if (p.has_token && warp == 0) {
+            if (FAM != KDA) tgate = p.tok_gate[u];
+            if (FAM != MAMBA2) tbeta = p.tok_beta[u];
+        }
+        bool w_ok = mbar_wait(tbar, k & 1);
+        w_ok = mbar_wait(wbar, k & 1) && w_ok;
+        if (__syncthreads_or(!w_ok)) { ok = false; break; }       // (A) head u staged
+        if (t == 0) pending = 0;
+        unsigned char* sl = smem;
+
+        // 1. This thread's tile, pairs of adjacent columns.
+        float2 st[R][2];
+        {
+            const float* tb = tile + row0 * V + c0;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const float4 a = *reinterpret_cast<const float4*>(tb + i * V);
+                st[i][0] = make_float2(a.x, a.y);
+                st[i][1] = make_float2(a.z, a.w);
             }
         }
+
+        // 2. Per-head preparation: keys, decays, coefficients, extended basis.
+        const int r_h = p.do_sketch ? p.off[h + 1] - p.off[h] : 0;
+        const int next = r_h + p.has_token;                           // columns of [Omega_h | q]
+        const int nch = (next + 3) / 4;
+        prepare_head<FAM, K, V>(p, h, n, r_h, rpad, sl, L, smem, tgate, tbeta, t);
         __syncthreads();                                              // (B)
 
         // 3. The tile buffer is free: start the next head's state.
-        if (un < units) prefetch_tile<K, V>(p, un, tile, t);
-        cp_async_commit();
+        if (t == 0 && un < units) {
+            mbar_expect_tx(tbar, K * V * 4);
+            bulk_g2s(smem + L.tile, p.state + un * (long long)(K * V), K * V * 4, tbar);
+            pending |= 1u;
+        }
 
         // 4. Apply the updates.
         const unsigned mask = meta[0];
         const float* kdb = kd + rb * KB;
         const float* kub = ku + rb * KB;
-        for (int j = 0; j < n; ++j) {
-            const float4 scj = sc[j];
-            const bool fold = (mask >> j) & 1u;
-            if (fold) {
-                if (FAM == KDA) {
-#pragma unroll
-                    for (int i = 0; i < R; i += 2) {
-                        const float4 f = *reinterpret_cast<const float4*>(kub + j * KD + 2 * i);
-#pragma unroll
-                        for (int cp = 0; cp < 2; ++cp) {
-                            s[i][cp] = fmul2(s[i][cp], make_float2(f.x, f.y));
-                            s[i + 1][cp] = fmul2(s[i + 1][cp], make_float2(f.z, f.w));
-                        }
-                    }
-                } else {
-                    const float2 f = dup2(scj.z);
-#pragma unroll
-                    for (int i = 0; i < R; ++i)
-#pragma unroll
-                        for (int cp = 0; cp < 2; ++cp) s[i][cp] = fmul2(s[i][cp], f);
-                }
-            }
+        const uint16_t* vraw = reinterpret_cast<const uint16_t*>(sl + L.vraw);
+        auto update = [&](int j, float4 scj) {
             float2 kv[R];
 #pragma unroll
             for (int i = 0; i < R; i += 2) {
@@ -348,17 +398,23 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
             }
             float2 w2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
             if (FAM != MAMBA2) {
+                float2 w2b[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int i = 0; i < R; ++i)
+                for (int i = 0; i < R; i += 2)
 #pragma unroll
-                    for (int cp = 0; cp < 2; ++cp) w2[cp] = ffma2(kv[i], s[i][cp], w2[cp]);
+                    for (int cp = 0; cp < 2; ++cp) {
+                        w2[cp] = ffma2(kv[i], st[i][cp], w2[cp]);
+                        w2b[cp] = ffma2(kv[i + 1], st[i + 1][cp], w2b[cp]);
+                    }
 #pragma unroll
-                for (int cp = 0; cp < 2; ++cp)
+                for (int cp = 0; cp < 2; ++cp) {
+                    w2[cp] = make_float2(w2[cp].x + w2b[cp].x, w2[cp].y + w2b[cp].y);
 #pragma unroll
                     for (int m = 4; m <= 16; m <<= 1) {
                         w2[cp].x += __shfl_xor_sync(FULL, w2[cp].x, m);
                         w2[cp].y += __shfl_xor_sync(FULL, w2[cp].y, m);
                     }
+                }
             }
             const uint2 vv = *reinterpret_cast<const uint2*>(vraw + j * V + c0);
             const float2 v01 = make_float2(bf2f_lo(vv.x), bf2f_hi(vv.x));
@@ -372,7 +428,7 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
                 d2[0] = fmul2(dup2(scj.x), ffma2(ncw, w2[0], v01));
                 d2[1] = fmul2(dup2(scj.x), ffma2(ncw, w2[1], v23));
             }
-            if (FAM == KDA && !fold) {
+            if (FAM == KDA && !((mask >> j) & 1u)) {
 #pragma unroll
                 for (int i = 0; i < R; i += 2) {
                     const float4 f = *reinterpret_cast<const float4*>(kub + j * KD + 2 * i);
@@ -383,13 +439,44 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
 #pragma unroll
             for (int i = 0; i < R; ++i)
 #pragma unroll
-                for (int cp = 0; cp < 2; ++cp) s[i][cp] = ffma2(kv[i], d2[cp], s[i][cp]);
+                for (int cp = 0; cp < 2; ++cp) st[i][cp] = ffma2(kv[i], d2[cp], st[i][cp]);
+        };
+        if (mask == 0) {                                              // no folds (the common case)
+            constexpr int UNR = V == 64 ? 2 : 1;                      // dv = 128 has no registers to spare
+#pragma unroll UNR
+            for (int j = 0; j < n; ++j) update(j, sc[j]);
+        } else {
+            for (int j = 0; j < n; ++j) {
+                const float4 scj = sc[j];
+                if ((mask >> j) & 1u) {
+                    if (FAM == KDA) {
+#pragma unroll
+                        for (int i = 0; i < R; i += 2) {
+                            const float4 f = *reinterpret_cast<const float4*>(kub + j * KD + 2 * i);
+#pragma unroll
+                            for (int cp = 0; cp < 2; ++cp) {
+                                st[i][cp] = fmul2(st[i][cp], make_float2(f.x, f.y));
+                                st[i + 1][cp] = fmul2(st[i + 1][cp], make_float2(f.z, f.w));
+                            }
+                        }
+                    } else {
+                        const float2 f = dup2(scj.z);
+#pragma unroll
+                        for (int i = 0; i < R; ++i)
+#pragma unroll
+                            for (int cp = 0; cp < 2; ++cp) st[i][cp] = fmul2(st[i][cp], f);
+                    }
+                }
+                update(j, scj);
+            }
         }
-        __syncthreads();                                              // (C) window buffers read
+        __syncthreads();                                              // (C) window read
 
         // 5. The window buffers are free: start the next head's window.
-        if (un < units) prefetch_window<FAM, K, V>(p, un, smem, L, t);
-        cp_async_commit();
+        if (t == 0 && un < units) {
+            issue_window<FAM, K, V>(p, un, smem, L, wbar, 0u);
+            pending |= 2u;
+        }
 
         // 6. True state S = Diag(Gamma) S', written back.
         if (FAM == KDA) {
@@ -399,8 +486,8 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
                 const float4 f = *reinterpret_cast<const float4*>(g + 2 * i);
 #pragma unroll
                 for (int cp = 0; cp < 2; ++cp) {
-                    s[i][cp] = fmul2(s[i][cp], make_float2(f.x, f.y));
-                    s[i + 1][cp] = fmul2(s[i + 1][cp], make_float2(f.z, f.w));
+                    st[i][cp] = fmul2(st[i][cp], make_float2(f.x, f.y));
+                    st[i + 1][cp] = fmul2(st[i + 1][cp], make_float2(f.z, f.w));
                 }
             }
         } else {
@@ -408,17 +495,18 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
 #pragma unroll
             for (int i = 0; i < R; ++i)
 #pragma unroll
-                for (int cp = 0; cp < 2; ++cp) s[i][cp] = fmul2(s[i][cp], f);
+                for (int cp = 0; cp < 2; ++cp) st[i][cp] = fmul2(st[i][cp], f);
         }
-        float* st = p.state + u * (long long)(K * V) + row0 * V + c0;
+        float* sto = p.state + u * (long long)(K * V) + row0 * V + c0;
 #pragma unroll
         for (int i = 0; i < R; ++i)
-            __stcs(reinterpret_cast<float4*>(st + i * V), make_float4(s[i][0].x, s[i][0].y, s[i][1].x, s[i][1].y));
+            __stcs(reinterpret_cast<float4*>(sto + i * V), make_float4(st[i][0].x, st[i][0].y, st[i][1].x, st[i][1].y));
 
         // 7. Fused read-out against [Omega_h | q], 4 basis columns per pass; a
         //    3-level reduce-scatter over the row blocks leaves row block
         //    (b2 b1 b0) with basis column 4 ch + 2 b2 + b1 for the state
         //    columns c0 + 2 b0, c0 + 2 b0 + 1.
+        const float* pt = reinterpret_cast<const float*>(smem + L.pt);
         const int hb2 = (rb >> 2) & 1, hb1 = (rb >> 1) & 1, hb0 = rb & 1;
         for (int ch = 0; ch < nch; ++ch) {
             float2 acc[4][2];
@@ -433,7 +521,7 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
 #pragma unroll
                     for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-                        for (int cp = 0; cp < 2; ++cp) acc[e][cp] = ffma2(dup2(pe[ii]), s[i + ii][cp], acc[e][cp]);
+                        for (int cp = 0; cp < 2; ++cp) acc[e][cp] = ffma2(dup2(pe[ii]), st[i + ii][cp], acc[e][cp]);
                 }
             }
             float v8[2][4];                      // level 1 (lane bit 4 = rb bit 2): basis columns {0,1} | {2,3}
@@ -475,7 +563,12 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
             }
         }
     }
-    cp_async_wait_all();
+    if (!ok && t == 0) {                                              // a bounded wait ran out
+        report_timeout(p.status);
+        const int k_last = int((u - blockIdx.x) / gridDim.x);         // the head whose wait failed
+        if (pending & 1u) mbar_wait(tbar, k_last & 1);                // own copies: one more bounded wait
+        if (pending & 2u) mbar_wait(wbar, k_last & 1);
+    }
 }
 
 template <int FAM, int K, int V>

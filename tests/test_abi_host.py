@@ -63,7 +63,7 @@ def test_create_rejects_bad_shapes(L):
 def test_supported_rank_and_window_range(L):
     """The shared-memory limits stated for ss_create: every rank up to 64 at
     W <= 16 and up to 32 at W <= 32 is accepted, for every family, shape and
-    sketch type; rank 128 with dk = dv = 128 at W = 32 is not."""
+    sketch type; KDA with rank 128, dk = dv = 128 and W = 32 is not."""
     def ok(fam, dk, dv, W, r, sk):
         try:
             B.Plan(fam, 2, 2, dk, dv, W, [r, 1], sk)
@@ -76,7 +76,7 @@ def test_supported_rank_and_window_range(L):
             for sk in (B.SS_F32, B.SS_BF16):
                 assert ok(fam, dk, dv, 16, min(64, dk), sk)
                 assert ok(fam, dk, dv, 32, 32, sk)
-        assert not ok(fam, 128, 128, 32, 128, B.SS_F32)
+    assert not ok(B.SS_KDA, 128, 128, 32, 128, B.SS_F32)
 
 
 def test_buffer_sizes(L):

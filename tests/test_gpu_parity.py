@@ -233,7 +233,7 @@ def test_sweep_points_sampled(cuda_ok, batch, window, mean_rank):
         p.step(synth.step_inputs(wl, p.st, t), ring=False)
 
 
-@pytest.mark.parametrize("call", ["decode", "replay"])
+@pytest.mark.parametrize("call", ["decode", "replay", "flush"])
 def test_bounded_wait_reports_timeout(cuda_ok, call):
     """A launch whose bulk copies deliver fewer bytes than one CTA expects: that
     CTA's bounded wait runs out, it sets SS_DEVICE_TIMEOUT in the status word
@@ -248,8 +248,10 @@ def test_bounded_wait_reports_timeout(cuda_ok, call):
     tok = p.layer.token(synth.step_inputs(wl, p.st, 0))
     if call == "decode":
         p.layer.decode(tok)
-    else:
+    elif call == "replay":
         B.ss_replay_step(p.layer.plan, p.layer.bufs(False), p.layer.io(tok))
+    else:
+        p.layer.flush(None)                      # end-of-sequence flush of an empty window
     torch.cuda.synchronize()
     assert int(p.layer.status[0]) & B.SS_DEVICE_TIMEOUT
     # the context is still usable: a fresh session runs clean and matches the oracle
