@@ -84,12 +84,18 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// One bounded probe of an mbarrier phase: the thread may be suspended for up
+// to `hint_ns` (woken early when the phase completes), so a waiting warp
+// issues few instructions.
+#ifndef SS_WAIT_HINT_NS
+#define SS_WAIT_HINT_NS 2000
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned phase) {
     unsigned ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase)
+        : "r"(smem_u32(bar)), "r"(phase), "r"(SS_WAIT_HINT_NS)
         : "memory");
     return ok != 0;
 }
