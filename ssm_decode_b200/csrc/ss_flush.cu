@@ -594,10 +594,13 @@ cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream) {
+    if (family == MAMBA2) return launch_flush_mma(dk, dv, p, rmax, stream);
     SS_DISPATCH(flush_t, p, rmax, stream);
 }
 
+// rpad = rows of [Omega | q] rounded up to 4 (the CUDA-core kernel's read-out passes).
 int flush_smem_bytes(int family, int dk, int dv, int n, int rpad) {
+    if (family == MAMBA2) return flush_mma_smem_bytes(dk, dv, n, (rpad + 15) & ~15);
     return flush_layout(family, dk, dv, n, rpad).total;
 }
 

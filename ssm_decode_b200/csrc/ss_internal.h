@@ -64,6 +64,9 @@ struct StepParams {
 // `rmax` is the largest per-head rank taking part in the launch.
 cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int rmax,
                          cudaStream_t stream);
+// Mamba-2 flush on the tensor cores (any dk, dv in {64, 128}).
+cudaError_t launch_flush_mma(int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream);
+int flush_mma_smem_bytes(int dk, int dv, int n, int e16);
 cudaError_t launch_decode(int family, int dk, int dv, const StepParams& p, int rmax,
                           cudaStream_t stream);
 cudaError_t launch_replay(int family, int dk, int dv, const StepParams& p,
