@@ -593,6 +593,8 @@ cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
 
 }  // namespace
 
+// Mamba-2 runs on the tensor-core kernel (ss_flush_mma.cu); GDN and KDA on
+// the CUDA-core kernel above.
 cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream) {
     if (family == MAMBA2) return launch_flush_mma(dk, dv, p, rmax, stream);
     SS_DISPATCH(flush_t, p, rmax, stream);

@@ -25,47 +25,12 @@
 // to dv+4 floats (conflict-free fragment loads), the window by the same bulk
 // copies as the CUDA-core flush.  Waits are bounded and report
 // SS_DEVICE_TIMEOUT in the caller's status word.
-#include <cuda.h>   // CUtensorMap and its enums; the encoder is fetched from the driver at run time
-
 #include <mutex>
 
-#include "ss_common.cuh"
+#include "ss_mma.cuh"
 
 namespace ss {
 namespace {
-
-// x = hi + lo with hi = x truncated to tf32 (the low 13 mantissa bits
-// cleared) and lo = x - hi, exact in fp32; the MMA keeps lo's top bits, so
-// hi*b + lo*b is within 2^-20 |x b| of x*b.
-__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-    hi = __float_as_uint(x) & 0xffffe000u;
-    lo = __float_as_uint(x - __uint_as_float(hi));
-}
-// The same, kept where it is written: splitting the 64 accumulators of the
-// read-out once, ahead of its loop over basis tiles, would need 128 more
-// registers.
-__device__ __forceinline__ void split_tf32_here(float x, uint32_t& hi, uint32_t& lo) {
-    asm volatile("and.b32 %0, %1, 0xffffe000;\n" : "=r"(hi) : "r"(__float_as_uint(x)));
-    lo = __float_as_uint(x - __uint_as_float(hi));
-}
-
-// Tiled tensor copy of a 2-D box (x = column, y = row) into shared memory,
-// completing on an mbarrier.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// D += A B for one m16n8k8 tile (tf32 inputs, fp32 accumulators).
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 template <int K, int V>
 struct MS {
@@ -73,15 +38,6 @@ struct MS {
     static constexpr int NT = K / 8;             // 8-row blocks of the state
     static constexpr int KS = K + 8;             // padded key / basis row (floats)
 };
-
-// The state tile arrives as dv/32 boxes of dk rows x 32 floats (128 bytes)
-// with the 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
-// Byte offset of element (row, col):
-template <int K>
-__device__ __forceinline__ int tile_off(int row, int col) {
-    const int cc = col & 31;
-    return (col >> 5) * (K * 128) + row * 128 + ((((cc >> 2) ^ (row & 7)) << 4) | ((cc & 3) << 2));
-}
 
 // Per-CTA shared-memory layout (byte offsets).
 struct MmaLayout {
@@ -137,15 +93,6 @@ __device__ __forceinline__ void mma_issue_window(const FlushParams& p, long long
         bulk_g2s(smem + L.tq, p.tok_q + u * K, K * 2, bar);
     }
     if (r > 0) bulk_g2s(smem + L.braw, p.basis + (long long)p.off[h] * K, r * K * 4, bar);
-}
-
-// One thread: the state tile of head u, dv/32 swizzled boxes.
-template <int K, int V>
-__device__ __forceinline__ void mma_issue_tile(const CUtensorMap* map, long long u, unsigned char* base,
-                                               const MmaLayout& L, uint64_t* bar) {
-    mbar_expect_tx(bar, K * V * 4);
-#pragma unroll
-    for (int bx = 0; bx < V / 32; ++bx) tma_load_2d(base + L.tile + bx * K * 128, map, 32 * bx, int(u * K), bar);
 }
 
 // Per-head preparation: widened keys kt[j][row] (zero past the window),
@@ -266,7 +213,7 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
     }
     __syncthreads();
     if (u < units && t == 0) {
-        mma_issue_tile<K, V>(&tmap, u, smem, L, tbar);
+        issue_state_tile<K, V>(&tmap, u, smem + L.tile, tbar);
         mma_issue_window<K, V>(p, u, smem, L, wbar, stall ? 16u : 0u);
         pending = 3u;
     }
@@ -306,7 +253,7 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
 
         // 3. The tile buffer is free: start the next head's state.
         if (un < units && t == 0) {
-            mma_issue_tile<K, V>(&tmap, un, smem, L, tbar);
+            issue_state_tile<K, V>(&tmap, un, smem + L.tile, tbar);
             pending |= 1u;
         }
 
@@ -434,6 +381,31 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
     }
 }
 
+template <int K, int V>
+cudaError_t flush_mma_t(const FlushParams& p, int rmax, cudaStream_t stream) {
+    const int n = p.n_ring + p.has_token;
+    const int e16 = (((p.do_sketch ? rmax : 0) + p.has_token) + 15) & ~15;
+    const int bytes = mma_layout(K, V, n, e16).total;
+    if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
+    CUtensorMap map;
+    cudaError_t e = state_tensor_map(p.state, (long long)p.B * p.H * K, K, V, &map);
+    if (e != cudaSuccess) return e;
+    auto kern = flush_mma_kernel<K, V>;
+    static KernelCache kc;
+    e = ensure_smem(kern, kc, bytes);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cached_occupancy(kern, kc, MS<K, V>::T, bytes, &per_sm);
+    if (e != cudaSuccess) return e;
+    const long long units = (long long)p.B * p.H;
+    const long long cap = (long long)per_sm * sm_count();
+    const long long grid = units < cap ? units : cap;
+    kern<<<dim3(unsigned(grid)), dim3(MS<K, V>::T), bytes, stream>>>(p, map, e16);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
 // The driver's tensor-map encoder, fetched once through the runtime.
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -484,31 +456,6 @@ cudaError_t state_tensor_map(const float* state, long long rows, int K, int V, C
     *out = m;
     return cudaSuccess;
 }
-
-template <int K, int V>
-cudaError_t flush_mma_t(const FlushParams& p, int rmax, cudaStream_t stream) {
-    const int n = p.n_ring + p.has_token;
-    const int e16 = (((p.do_sketch ? rmax : 0) + p.has_token) + 15) & ~15;
-    const int bytes = mma_layout(K, V, n, e16).total;
-    if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
-    CUtensorMap map;
-    cudaError_t e = state_tensor_map(p.state, (long long)p.B * p.H * K, K, V, &map);
-    if (e != cudaSuccess) return e;
-    auto kern = flush_mma_kernel<K, V>;
-    static KernelCache kc;
-    e = ensure_smem(kern, kc, bytes);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cached_occupancy(kern, kc, MS<K, V>::T, bytes, &per_sm);
-    if (e != cudaSuccess) return e;
-    const long long units = (long long)p.B * p.H;
-    const long long cap = (long long)per_sm * sm_count();
-    const long long grid = units < cap ? units : cap;
-    kern<<<dim3(unsigned(grid)), dim3(MS<K, V>::T), bytes, stream>>>(p, map, e16);
-    return cudaGetLastError();
-}
-
-}  // namespace
 
 cudaError_t launch_flush_mma(int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream) {
     if (dk == 128 && dv == 64) return flush_mma_t<128, 64>(p, rmax, stream);
