@@ -253,7 +253,8 @@ def run_ours(args, rank, world):
     fl_b = fl["read_bytes"] + fl["write_bytes"]
     kernel_ms = sum(dec_t) + sum(fl_t)
     kernels = {}
-    for name, ts, nbytes in (("decode_kernel", dec_t, dec_b), ("flush_kernel", fl_t, fl_b)):
+    flush_name = "flush_mma_kernel" if wl.family == synth.MAMBA2 else "flush_kernel"
+    for name, ts, nbytes in (("decode_kernel", dec_t, dec_b), (flush_name, fl_t, fl_b)):
         if not ts:
             continue
         avg_s = sum(ts) / len(ts) / 1e3
