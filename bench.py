@@ -206,24 +206,32 @@ def run_ours(args, rank, world):
     def ev():
         return torch.cuda.Event(enable_timing=True)
 
-    def window(events, call=lambda lay, tok: lay.step(tok)):
+    def window(marks=None, call=lambda lay, tok: lay.step(tok), per_launch=None):
+        # marks = (start, decodes done, end) events on the launching stream:
+        # the window's decodes run between the first two, its flushes between
+        # the last two.  per_launch[p][l] = an event pair around one launch
+        # (a separate pass only: events between launches add gaps).
+        if marks:
+            marks[0].record(stream)
         for p in range(W):
+            if marks and p == W - 1:
+                marks[1].record(stream)
             for l, lay in enumerate(layers):
-                e0, e1 = events[p][l]
-                e0.record(stream)
+                if per_launch:
+                    per_launch[p][l][0].record(stream)
                 call(lay, toks[(p + l) % W])
-                e1.record(stream)
-
-    def new_events():
-        return [[(ev(), ev()) for _ in range(NL)] for _ in range(W)]
+                if per_launch:
+                    per_launch[p][l][1].record(stream)
+        if marks:
+            marks[2].record(stream)
 
     for lay in layers:
         lay.prime()
-    evs = [new_events() for _ in range(args.steps)]
+    marks = [(ev(), ev(), ev()) for _ in range(args.steps)]
     # clocks are sampled from the start of the warm-up through the timed windows
     with ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) as clk:
         for _ in range(args.warmup):
-            window(new_events())
+            window()
         torch.cuda.synchronize()
         barrier(dev)
         n0 = B.ss_launch_count()
@@ -231,14 +239,18 @@ def run_ours(args, rank, world):
         torch.cuda.synchronize()
         t_all0.record(stream)
         for k in range(args.steps):
-            window(evs[k])
+            window(marks[k])
         t_all1.record(stream)
         torch.cuda.synchronize()
         barrier(dev)
     launches = B.ss_launch_count() - n0
-    dec_t = [evs[k][p][l][0].elapsed_time(evs[k][p][l][1])
-             for k in range(args.steps) for p in range(W - 1) for l in range(NL)]
-    fl_t = [evs[k][W - 1][l][0].elapsed_time(evs[k][W - 1][l][1]) for k in range(args.steps) for l in range(NL)]
+    dec_ms = sum(m[0].elapsed_time(m[1]) for m in marks)
+    fl_ms = sum(m[1].elapsed_time(m[2]) for m in marks)
+    n_dec, n_fl = args.steps * NL * (W - 1), args.steps * NL
+    # per-position decode times, from a separate pass with events around each launch
+    per_launch = [[(ev(), ev()) for _ in range(NL)] for _ in range(W)]
+    window(per_launch=per_launch)
+    torch.cuda.synchronize()
     total_ms = t_all0.elapsed_time(t_all1)
     total_ms_max = reduce_max(total_ms, dev)
     value = weak_scaling_value(units * W * NL * args.steps, world, total_ms_max / 1e3)
@@ -251,22 +263,24 @@ def run_ours(args, rank, world):
     dec_b = sum(t["read_bytes"] + t["write_bytes"] for t in dec_bytes) / max(W - 1, 1)
     fl = B.ss_traffic_bytes(plan, B.SS_OP_FLUSH)
     fl_b = fl["read_bytes"] + fl["write_bytes"]
-    kernel_ms = sum(dec_t) + sum(fl_t)
+    kernel_ms = dec_ms + fl_ms
     kernels = {}
     flush_name = "flush_mma_kernel" if wl.family == synth.MAMBA2 else "flush_kernel"
-    for name, ts, nbytes in (("decode_kernel", dec_t, dec_b), (flush_name, fl_t, fl_b)):
-        if not ts:
+    for name, ms, count, nbytes in (("decode_kernel", dec_ms, n_dec, dec_b), (flush_name, fl_ms, n_fl, fl_b)):
+        if not count:
             continue
-        avg_s = sum(ts) / len(ts) / 1e3
+        avg_s = ms / count / 1e3
         ach = nbytes / avg_s / 1e9
         rec = kernel_traffic_record(name)
-        kernels[name] = {"launches": len(ts), "avg_us": avg_s * 1e6, "bytes_per_launch": nbytes,
-                         "achieved_gbs": ach, "frac": ach / peak, "share": sum(ts) / kernel_ms,
-                         "traffic": rec["dram_bytes_per_launch"] if rec else None}
+        kernels[name] = {"launches": count, "avg_us": avg_s * 1e6, "bytes_per_launch": nbytes,
+                         "achieved_gbs": ach, "frac": ach / peak, "share": ms / kernel_ms,
+                         "traffic": rec["dram_bytes_per_launch"] if rec else None,
+                         "timing": "events at window boundaries and around the flush group"}
     if W > 1:
         kernels["decode_kernel"]["by_phase_us"] = [
-            round(sum(evs[k][p][l][0].elapsed_time(evs[k][p][l][1]) for k in range(args.steps)
-                      for l in range(NL)) / (args.steps * NL) * 1e3, 2) for p in range(W - 1)]
+            round(sum(per_launch[p][l][0].elapsed_time(per_launch[p][l][1]) for l in range(NL)) / NL * 1e3, 2)
+            for p in range(W - 1)]
+        kernels["decode_kernel"]["by_phase_note"] = "one extra window with events around each launch"
     dom = max(kernels, key=lambda k: kernels[k]["share"])
     d = kernels[dom]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(d["achieved_gbs"], 1), "peak": peak,
@@ -279,10 +293,9 @@ def run_ours(args, rank, world):
                        ("replay", lambda lay, tok: lay.replay_step(tok))):
         ts = []
         for _ in range(2):
-            e = new_events()
             a, b = ev(), ev()
             a.record(stream)
-            window(e, call)
+            window(call=call)
             b.record(stream)
             torch.cuda.synchronize()
             ts.append(a.elapsed_time(b) / NL)
