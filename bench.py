@@ -173,6 +173,37 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
+def sketch_vs_exact(layers, toks, W, torch):
+    """Approximation metric of the sketched read: two layers start from the same
+    state; one takes the window's non-flush steps through ss_decode_step
+    (sketched read), the other through ss_replay_step (the exact windowed read
+    S0^T q~ + buffered term, same library); their outputs are compared per
+    (sequence, head): ||o^ - o||_2 / ||o||_2."""
+    a, b = layers[0], layers[1]
+    b.state.copy_(a.state)
+    a.prime()
+    b.prime()
+    errs, nums, dens = [], 0.0, 0.0
+    for p in range(W - 1):
+        a.decode(toks[p])
+        b.replay_step(toks[p])
+        num = (a.out - b.out).double().norm(dim=-1)
+        den = b.out.double().norm(dim=-1)
+        errs.append((num / den.clamp_min(1e-300)).flatten())
+        nums += float(num.sum())
+        dens += float(den.sum())
+    e = torch.cat(errs)
+    res = {"metric": "sketch-vs-exact relative error ||o^ - o||_2 / ||o||_2 per (sequence, head) "
+                      "over the non-flush steps of one window (sketched decode vs the exact replay read)",
+            "mean": float(e.mean()), "p99": float(torch.quantile(e.float(), 0.99)), "max": float(e.max()),
+            "aggregate": nums / max(dens, 1e-300),       # sum ||o^ - o|| / sum ||o||
+            "outputs": int(e.numel())}
+    # close the window so both layers are back at phase 0
+    a.flush(toks[W - 1])
+    b.replay_step(toks[W - 1])
+    return res
+
+
 def run_ours(args, rank, world):
     import torch
     from ssm_decode_b200 import binding as B
@@ -302,6 +333,7 @@ def run_ours(args, rank, world):
         t = min(ts)
         baselines[name] = {"ms_per_window": t, "value": units * W / (t / 1e3),
                            "sketch_speedup": t / (total_ms / (args.steps * NL))}
+    approx = sketch_vs_exact(layers, toks, W, torch) if NL >= 2 and W > 1 else None
     for lay in layers:
         lay.prime()
 
@@ -344,7 +376,7 @@ def run_ours(args, rank, world):
                    "l2": f"inputs larger than L2: {NL} layers rotated, back-to-back launches",
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline, "kernels": kernels, "baselines": baselines, "e2e": e2e,
-        "gpu_launches": launches, "clocks": clk.summary(),
+        "gpu_launches": launches, "clocks": clk.summary(), "approx": approx,
     }
     return result
 
@@ -410,6 +442,101 @@ def run_reference(args):
     }
 
 
+def run_sweep(args):
+    """The sweep on the Mamba-2 shape: batch x window x mean rank, sketched
+    flush + decode against the Standard and ReplaySSM steps of the same
+    library, with the decode / flush HBM GB/s and the sketch-vs-exact error.
+    One JSON line per point, then a markdown table."""
+    import torch
+    from ssm_decode_b200 import binding as B
+    from ssm_decode_b200 import synth
+    from ssm_decode_b200.layer import DecodeLayer
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peak = float(measured_peaks()[0]["hbm_gbs"])
+    rows = []
+    batches = [int(x) for x in args.sweep_batches.split(",")]
+    windows = [int(x) for x in args.sweep_windows.split(",")]
+    ranks = [int(x) for x in args.sweep_ranks.split(",")]
+    for batch in batches:
+        for W in windows:
+            for mr in ranks:
+                wl = synth.sweep_workload(batch, W, mr)
+                st = synth.static_inputs(wl)
+                # enough layers that the rotated inputs exceed L2 (126 MB), at least 2
+                per_layer = wl.units * wl.dk * wl.dv * 4
+                NL = max(2, min(8, -(-400_000_000 // per_layer)))
+                layers = []
+                for _ in range(NL):
+                    lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, B.SS_BF16, device=dev)
+                    lay.load(st.state, st.basis, st.coef, st.A)
+                    layers.append(lay)
+                toks = [layers[0].token(synth.step_inputs(wl, st, t)) for t in range(W)]
+                for lay in layers:
+                    lay.prime()
+
+                def run(call, marks=None):
+                    if marks:
+                        marks[0].record(stream)
+                    for p in range(W):
+                        if marks and p == W - 1:
+                            marks[1].record(stream)
+                        for l, lay in enumerate(layers):
+                            call(lay, toks[(p + l) % W])
+                    if marks:
+                        marks[2].record(stream)
+
+                ev = lambda: torch.cuda.Event(enable_timing=True)
+                res = {}
+                for name, call in (("sketch", lambda lay, tok: lay.step(tok)),
+                                   ("standard", lambda lay, tok: lay.exact_step(tok)),
+                                   ("replay", lambda lay, tok: lay.replay_step(tok))):
+                    run(call)                                  # warm-up window
+                    ms = []
+                    for _ in range(args.sweep_windows_timed):
+                        m = (ev(), ev(), ev())
+                        run(call, m)
+                        torch.cuda.synchronize()
+                        ms.append((m[0].elapsed_time(m[2]), m[0].elapsed_time(m[1]), m[1].elapsed_time(m[2])))
+                    best = min(ms)
+                    res[name] = best
+                    if name != "sketch":
+                        for lay in layers:
+                            lay.prime()
+                t_win, t_dec, t_fl = res["sketch"]
+                plan = layers[0].plan
+                dec_b = (sum(sum(B.ss_traffic_bytes(plan, B.SS_OP_DECODE, p)[k] for k in ("read_bytes", "write_bytes"))
+                             for p in range(W - 1)) / max(W - 1, 1))
+                fl = B.ss_traffic_bytes(plan, B.SS_OP_FLUSH)
+                fl_b = fl["read_bytes"] + fl["write_bytes"]
+                dec_us = t_dec / max(NL * (W - 1), 1) * 1e3
+                fl_us = t_fl / NL * 1e3
+                approx = sketch_vs_exact(layers, toks, W, torch) if W > 1 else None
+                row = {"batch": batch, "window": W, "mean_rank": mr, "layers": NL,
+                       "sketch_steps_per_s": wl.units * W * NL / (t_win / 1e3),
+                       "standard_steps_per_s": wl.units * W * NL / (res["standard"][0] / 1e3),
+                       "replay_steps_per_s": wl.units * W * NL / (res["replay"][0] / 1e3),
+                       "decode_us": dec_us, "decode_gbs": dec_b / (dec_us * 1e-6) / 1e9 if W > 1 else None,
+                       "flush_us": fl_us, "flush_gbs": fl_b / (fl_us * 1e-6) / 1e9,
+                       "err_mean": approx["mean"] if approx else 0.0, "err_max": approx["max"] if approx else 0.0}
+                rows.append(row)
+                print(json.dumps(row), flush=True)
+                del layers, toks
+                torch.cuda.empty_cache()
+    print("| batch | W | mean r | sketch steps/s | vs Standard | vs Replay | decode µs (GB/s) | flush µs (GB/s) | "
+          "sketch-vs-exact err mean / max |")
+    print("|---|---|---|---|---|---|---|---|---|")
+    for r in rows:
+        dec = f"{r['decode_us']:.1f} ({r['decode_gbs']:.0f})" if r["decode_gbs"] else "-"
+        print(f"| {r['batch']} | {r['window']} | {r['mean_rank']} | {r['sketch_steps_per_s']:.3g} | "
+              f"{r['sketch_steps_per_s'] / r['standard_steps_per_s']:.2f}x | "
+              f"{r['sketch_steps_per_s'] / r['replay_steps_per_s']:.2f}x | {dec} | "
+              f"{r['flush_us']:.1f} ({r['flush_gbs']:.0f}) | {r['err_mean']:.3g} / {r['err_max']:.3g} |")
+    print(f"(peak: measured {peak:.0f} GB/s)")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -422,9 +549,19 @@ def main():
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the batch x window x rank sweep on the Mamba-2 shape (1 GPU), instead of the bench line")
+    ap.add_argument("--sweep-batches", default="1,32,128,320,1024")
+    ap.add_argument("--sweep-windows", default="4,8,16,32")
+    ap.add_argument("--sweep-ranks", default="4,8,16")
+    ap.add_argument("--sweep-windows-timed", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+
+    if args.sweep:
+        run_sweep(args)
+        return
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
