@@ -86,6 +86,9 @@ typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_sketch_dtype;
  * to about one second; if a wait runs out the kernel sets SS_DEVICE_TIMEOUT
  * and returns without completing its outputs. */
 #define SS_DEVICE_TIMEOUT 1
+/* Set by ss_step_mixed when a fill count lies outside 0..W-1: that sequence
+ * is neither decoded nor flushed and its fill_out entry is left as it was. */
+#define SS_DEVICE_BAD_FILL 2
 
 typedef struct {
     int32_t family;          /* ss_family */
@@ -213,6 +216,22 @@ ss_status ss_exact_step(ss_plan* plan, const ss_buffers* bufs, const ss_step_io*
  * ss_flush with bufs->sketch == NULL. */
 ss_status ss_replay_step(ss_plan* plan, const ss_buffers* bufs, const ss_step_io* io,
                          ss_stream stream);
+
+/* One step of a batch whose sequences sit at different window positions
+ * (project page, "Per step"; paper §3.2 and §4.1 applied per sequence).
+ * fill_in[b] (device int32[batch], 4-byte aligned) is the number of tokens
+ * sequence b has buffered since its last flush, 0..W-1.  Sequences with
+ * fill_in[b] <= W-2 take the non-flush step of ss_decode_step at their own
+ * slot fill_in[b]; sequences with fill_in[b] == W-1 take ss_flush with this
+ * token and refresh their sketch rows.  fill_out[b] (device int32[batch],
+ * must not alias fill_in) receives (fill_in[b] + 1) mod W.  A value outside
+ * 0..W-1 sets SS_DEVICE_BAD_FILL in bufs->status; that sequence's outputs,
+ * ring, state and fill_out entry are left as they were.  Needs the plan at
+ * phase 0 with a valid sketch (ss_prime), bufs->state, sketch, basis, coef
+ * (and A for Mamba-2); the plan's phase is not used and stays 0.  Two
+ * kernels on `stream`; the fills are read on the device only. */
+ss_status ss_step_mixed(ss_plan* plan, const ss_buffers* bufs, const ss_step_io* io,
+                        const int32_t* fill_in, int32_t* fill_out, ss_stream stream);
 
 /* Traffic of one call for the whole batch (see ss_traffic).  tau = phase
  * before the call for SS_OP_DECODE / SS_OP_REPLAY / SS_OP_FLUSH_NO_TOKEN. */

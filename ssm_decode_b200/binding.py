@@ -17,6 +17,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "sketchssm.h")
 
 SS_OK, SS_ERR_INVALID_ARG, SS_ERR_ALIGNMENT, SS_ERR_UNSUPPORTED, SS_ERR_SCHEDULE, SS_ERR_CUDA = range(6)
 SS_DEVICE_TIMEOUT = 1
+SS_DEVICE_BAD_FILL = 2
 SS_MAMBA2, SS_GDN, SS_KDA = 0, 1, 2
 SS_F32, SS_BF16 = 0, 1
 (SS_OP_DECODE, SS_OP_FLUSH, SS_OP_FLUSH_NO_TOKEN, SS_OP_PRIME, SS_OP_EXACT, SS_OP_REPLAY,
@@ -79,6 +80,7 @@ def lib():
             "ss_flush": ([P, ctypes.POINTER(ss_buffers), ctypes.POINTER(ss_step_io), P], S),
             "ss_exact_step": ([P, ctypes.POINTER(ss_buffers), ctypes.POINTER(ss_step_io), P], S),
             "ss_replay_step": ([P, ctypes.POINTER(ss_buffers), ctypes.POINTER(ss_step_io), P], S),
+            "ss_step_mixed": ([P, ctypes.POINTER(ss_buffers), ctypes.POINTER(ss_step_io), P, P, P], S),
             "ss_traffic_bytes": ([P, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ss_traffic)], S),
             "ss_launch_count": ([], ctypes.c_uint64),
             "ss_debug_stall_next_copy": ([P, ctypes.c_int32], S),
@@ -225,6 +227,13 @@ def ss_exact_step(plan, bufs, io, stream=None):
 
 def ss_replay_step(plan, bufs, io, stream=None):
     _check(lib().ss_replay_step(plan.handle, ctypes.byref(bufs), ctypes.byref(io), _stream(stream)))
+
+
+def ss_step_mixed(plan, bufs, io, fill_in, fill_out, stream=None):
+    """fill_in / fill_out: device int32 tensors of `batch` entries (or raw pointers)."""
+    fi = fill_in if isinstance(fill_in, int) else fill_in.data_ptr()
+    fo = fill_out if isinstance(fill_out, int) else fill_out.data_ptr()
+    _check(lib().ss_step_mixed(plan.handle, ctypes.byref(bufs), ctypes.byref(io), fi, fo, _stream(stream)))
 
 
 def ss_traffic_bytes(plan, op, tau=0):

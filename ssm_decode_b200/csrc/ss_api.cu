@@ -335,6 +335,47 @@ ss_status ss_replay_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io,
     return ok();
 }
 
+ss_status ss_step_mixed(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, const int32_t* fill_in,
+                        int32_t* fill_out, ss_stream stream) {
+    if (pl == nullptr || b == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or bufs is NULL");
+    if (pl->phase != 0)
+        return fail(SS_ERR_SCHEDULE, "ss_step_mixed needs the plan at phase 0 (phase is %d)", pl->phase);
+    if (!pl->sketch_valid)
+        return fail(SS_ERR_SCHEDULE, "ss_step_mixed needs a current sketch (ss_prime first)");
+    if (fill_in == nullptr || fill_out == nullptr) return fail(SS_ERR_INVALID_ARG, "fill_in or fill_out is NULL");
+    if (reinterpret_cast<uintptr_t>(fill_in) % 4 || reinterpret_cast<uintptr_t>(fill_out) % 4)
+        return fail(SS_ERR_ALIGNMENT, "fill_in and fill_out must be 4-byte aligned");
+    if (static_cast<const void*>(fill_in) == static_cast<const void*>(fill_out))
+        return fail(SS_ERR_INVALID_ARG, "fill_out must not alias fill_in");
+    CHECK(check_ring(pl, b));
+    REQUIRE_PTR(b->state, "bufs->state");
+    REQUIRE_PTR(b->sketch, "bufs->sketch");
+    REQUIRE_PTR(b->basis, "bufs->basis");
+    REQUIRE_PTR(b->coef, "bufs->coef");
+    if (pl->cfg.family == SS_MAMBA2) REQUIRE_PTR(b->A, "bufs->A");
+    CHECK(check_io(pl, io));
+    CHECK(check_status(b));
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int stall = take_stall(pl);
+    const int W = pl->cfg.window;
+    if (W > 1) {                              // sequences with fill < W-1: a non-flush step
+        ss::StepParams p = step_params(pl, b, io);
+        p.p = W - 2;                          // staging is sized for the longest window
+        p.fill_in = fill_in;
+        p.fill_out = fill_out;
+        p.stall = stall;
+        CHECK(launched(ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax, st), "mixed decode"));
+    }
+    ss::FlushParams f = flush_params(pl, b, io);   // sequences with fill == W-1: the flush
+    f.n_ring = W - 1;
+    f.has_token = 1;
+    f.do_sketch = 1;
+    f.fill_in = fill_in;
+    f.fill_out = fill_out;
+    CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, f, pl->rmax, st), "mixed flush"));
+    return ok();
+}
+
 ss_status ss_traffic_bytes(const ss_plan* pl, int32_t op, int32_t tau, ss_traffic* out) {
     if (pl == nullptr || out == nullptr) return fail(SS_ERR_INVALID_ARG, "plan or out is NULL");
     const ss_config& c = pl->cfg;

@@ -115,6 +115,67 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned phase) {
     return true;
 }
 
+// A mixed step (fill_in set) flushes only the units whose sequence sits at
+// the window's last slot, fill_in[b] == W-1.  Each CTA of the flush keeps a
+// queue of its own such units in shared memory: its candidates are
+// blockIdx.x, blockIdx.x + gridDim.x, ...; warp 0 compacts them 32 at a time
+// with a ballot whenever the queue runs dry, so the fill counts are read once
+// per candidate and the next unit is a shared-memory read.  The refill also
+// writes fill_out[b] = 0 for each flushing sequence (from its head-0 unit).
+constexpr int FQ_CAP = 64;
+struct FlushQueue {
+    long long pos;           // next candidate to test
+    long long next;          // the unit handed out last (all threads read it)
+    int head, count;         // unit[head..count) are queued
+    int unit[FQ_CAP];
+};
+constexpr int FQ_BYTES = (int(sizeof(FlushQueue)) + 15) & ~15;
+
+__device__ __forceinline__ void fq_init(FlushQueue* q) {          // one thread
+    q->pos = blockIdx.x;
+    q->next = 0;
+    q->head = q->count = 0;
+}
+
+// Called by the whole of warp 0: the next unit this CTA flushes (`units`
+// when none is left); lane 0 also publishes it in q->next.
+__device__ __forceinline__ long long fq_next(const FlushParams& p, FlushQueue* q, long long units) {
+    const int lane = threadIdx.x & 31;
+    const bool refill = q->head == q->count;
+    __syncwarp();                                       // every lane has read head/count
+    if (refill) {
+        long long pos = q->pos;
+        int n = 0;
+        while (pos < units && n <= FQ_CAP - 32) {
+            const long long c = pos + (long long)lane * gridDim.x;
+            const bool hit = c < units && p.fill_in[c / p.H] == p.W - 1;
+            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            if (hit) {
+                q->unit[n + __popc(m & ((1u << lane) - 1u))] = int(c);
+                if (c % p.H == 0) p.fill_out[c / p.H] = 0;   // the sequence's new fill, once per sequence
+            }
+            n += __popc(m);
+            pos += 32LL * gridDim.x;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            q->pos = pos;
+            q->head = 0;
+            q->count = n;
+        }
+        __syncwarp();
+    }
+    const int h = q->head;
+    const long long u = h < q->count ? (long long)q->unit[h] : units;
+    __syncwarp();                                       // every lane has read head
+    if (lane == 0) {
+        if (h < q->count) q->head = h + 1;
+        q->next = u;
+    }
+    __syncwarp();
+    return u;
+}
+
 __device__ __forceinline__ void report_timeout(int32_t* status) {
     if (status != nullptr) atomicOr(status, SS_DEVICE_TIMEOUT);
 }

@@ -302,7 +302,7 @@ __device__ __forceinline__ void prepare_head(const FlushParams& p, int h, int n,
     }
 }
 
-template <int FAM, int K, int V>
+template <int FAM, int K, int V, bool MIXED>
 __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __grid_constant__ FlushParams p, int rpad) {
     using S = FS<K, V>;
     constexpr int R = S::R, KB = S::KB, KD = S::KD;
@@ -327,13 +327,21 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
 
     // Only thread 0 issues copies; it tracks which barriers have copies in flight.
     unsigned pending = 0;                        // bit 0: tile, bit 1: window
+    __shared__ FlushQueue fq_s;                      // mixed steps only
+    FlushQueue* const fq = &fq_s;
     long long u = blockIdx.x;
     if (t == 0) {
         mbar_init(tbar, 1);
         mbar_init(wbar, 1);
         fence_mbar_init();
+        if (MIXED) fq_init(fq);
     }
     __syncthreads();
+    if constexpr (MIXED) {
+        if (warp == 0) fq_next(p, fq, units);
+        __syncthreads();
+        u = fq->next;
+    }
     if (t == 0 && u < units) {
         mbar_expect_tx(tbar, K * V * 4);
         bulk_g2s(smem + L.tile, p.state + u * (long long)(K * V), K * V * 4, tbar);
@@ -342,10 +350,10 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
     }
 
     bool ok = true;
-    for (int k = 0; u < units; ++k, u += gridDim.x) {
+    int k_fail = 0;                                   // mixed steps: the head whose wait ran out
+    for (int k = 0; u < units; ++k, u = MIXED ? fq->next : u + gridDim.x) {
         const int h = int(u % p.H);
         const long long b = u / p.H;
-        const long long un = u + gridDim.x;
         float tgate = 0.f, tbeta = 0.f;                           // the token's scalar inputs
         if (p.has_token && warp == 0) {
             if (FAM != KDA) tgate = p.tok_gate[u];
@@ -353,7 +361,15 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
         }
         bool w_ok = mbar_wait(tbar, k & 1);
         w_ok = mbar_wait(wbar, k & 1) && w_ok;
-        if (__syncthreads_or(!w_ok)) { ok = false; break; }       // (A) head u staged
+        if (__syncthreads_or(!w_ok)) {                              // (A) head u staged
+            ok = false;
+            if (MIXED) k_fail = k;
+            break;
+        }
+        if constexpr (MIXED) {
+            // After (A) every thread has read the previous q->next: queue the next unit.
+            if (warp == 0) fq_next(p, fq, units);
+        }
         if (t == 0) pending = 0;
         unsigned char* sl = smem;
 
@@ -377,10 +393,13 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
         __syncthreads();                                              // (B)
 
         // 3. The tile buffer is free: start the next head's state.
-        if (t == 0 && un < units) {
-            mbar_expect_tx(tbar, K * V * 4);
-            bulk_g2s(smem + L.tile, p.state + un * (long long)(K * V), K * V * 4, tbar);
-            pending |= 1u;
+        {
+            const long long un = MIXED ? fq->next : u + gridDim.x;
+            if (t == 0 && un < units) {
+                mbar_expect_tx(tbar, K * V * 4);
+                bulk_g2s(smem + L.tile, p.state + un * (long long)(K * V), K * V * 4, tbar);
+                pending |= 1u;
+            }
         }
 
         // 4. Apply the updates.
@@ -473,9 +492,12 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
         __syncthreads();                                              // (C) window read
 
         // 5. The window buffers are free: start the next head's window.
-        if (t == 0 && un < units) {
-            issue_window<FAM, K, V>(p, un, smem, L, wbar, 0u);
-            pending |= 2u;
+        {
+            const long long un = MIXED ? fq->next : u + gridDim.x;
+            if (t == 0 && un < units) {
+                issue_window<FAM, K, V>(p, un, smem, L, wbar, 0u);
+                pending |= 2u;
+            }
         }
 
         // 6. True state S = Diag(Gamma) S', written back.
@@ -565,19 +587,19 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
     }
     if (!ok && t == 0) {                                              // a bounded wait ran out
         report_timeout(p.status);
-        const int k_last = int((u - blockIdx.x) / gridDim.x);         // the head whose wait failed
+        const int k_last = MIXED ? k_fail : int((u - blockIdx.x) / gridDim.x);   // the head whose wait failed
         if (pending & 1u) mbar_wait(tbar, k_last & 1);                // own copies: one more bounded wait
         if (pending & 2u) mbar_wait(wbar, k_last & 1);
     }
 }
 
-template <int FAM, int K, int V>
-cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
+template <int FAM, int K, int V, bool MIXED>
+cudaError_t flush_launch(const FlushParams& p, int rmax, cudaStream_t stream) {
     const int n = p.n_ring + p.has_token;
     const int rpad = ((p.do_sketch ? rmax : 0) + p.has_token + 3) & ~3;
     const int bytes = flush_layout(FAM, K, V, n, rpad).total;
     if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
-    auto kern = flush_kernel<FAM, K, V>;
+    auto kern = flush_kernel<FAM, K, V, MIXED>;
     static KernelCache kc;
     cudaError_t e = ensure_smem(kern, kc, bytes);
     if (e != cudaSuccess) return e;
@@ -589,6 +611,13 @@ cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
     const long long grid = units < cap ? units : cap;
     kern<<<dim3(unsigned(grid)), dim3(FS<K, V>::T), bytes, stream>>>(p, rpad);
     return cudaGetLastError();
+}
+
+// A mixed step (fill_in set) runs its own instance, so the uniform kernel
+// carries no unit selection.
+template <int FAM, int K, int V>
+cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
+    return p.fill_in ? flush_launch<FAM, K, V, true>(p, rmax, stream) : flush_launch<FAM, K, V, false>(p, rmax, stream);
 }
 
 }  // namespace

@@ -180,7 +180,7 @@ __device__ __forceinline__ void mma_prepare(const FlushParams& p, int h, int n, 
     }
 }
 
-template <int K, int V>
+template <int K, int V, bool MIXED>
 __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const __grid_constant__ FlushParams p,
                                                                          const __grid_constant__ CUtensorMap tmap,
                                                                          int e16) {
@@ -205,13 +205,21 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
     const bool stall = p.stall && blockIdx.x == 0;
 
     unsigned pending = 0;                            // thread 0: bit 0 tile, bit 1 window in flight
+    __shared__ FlushQueue fq_s;                      // mixed steps only
+    FlushQueue* const fq = &fq_s;
     long long u = blockIdx.x;
     if (t == 0) {
         mbar_init(tbar, 1);
         mbar_init(wbar, 1);
         fence_mbar_init();
+        if (MIXED) fq_init(fq);
     }
     __syncthreads();
+    if constexpr (MIXED) {
+        if (warp == 0) fq_next(p, fq, units);
+        __syncthreads();
+        u = fq->next;
+    }
     if (u < units && t == 0) {
         issue_state_tile<K, V>(&tmap, u, smem + L.tile, tbar);
         mma_issue_window<K, V>(p, u, smem, L, wbar, stall ? 16u : 0u);
@@ -219,14 +227,22 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
     }
 
     bool ok = true;
-    for (int k = 0; u < units; ++k, u += gridDim.x) {
+    int k_fail = 0;                                   // mixed steps: the head whose wait ran out
+    for (int k = 0; u < units; ++k, u = MIXED ? fq->next : u + gridDim.x) {
         const int h = int(u % p.H);
         const long long b = u / p.H;
-        const long long un = u + gridDim.x;
         const float tgate = (p.has_token && warp == 0) ? p.tok_gate[u] : 0.f;
         bool w_ok = mbar_wait(tbar, k & 1);
         w_ok = mbar_wait(wbar, k & 1) && w_ok;
-        if (__syncthreads_or(!w_ok)) { ok = false; break; }       // (A) head u staged
+        if (__syncthreads_or(!w_ok)) {                              // (A) head u staged
+            ok = false;
+            if (MIXED) k_fail = k;
+            break;
+        }
+        if constexpr (MIXED) {
+            // After (A) every thread has read the previous q->next: queue the next unit.
+            if (warp == 0) fq_next(p, fq, units);
+        }
         if (t == 0) pending = 0;
 
         // 1. S'^T in accumulator layout: acc[nb] covers rows 8 nb .. 8 nb + 7.
@@ -252,9 +268,12 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
         __syncthreads();                                              // (B)
 
         // 3. The tile buffer is free: start the next head's state.
-        if (un < units && t == 0) {
-            issue_state_tile<K, V>(&tmap, un, smem + L.tile, tbar);
-            pending |= 1u;
+        {
+            const long long un = MIXED ? fq->next : u + gridDim.x;
+            if (un < units && t == 0) {
+                issue_state_tile<K, V>(&tmap, un, smem + L.tile, tbar);
+                pending |= 1u;
+            }
         }
 
         // 4. The window's updates, 8 at a time: S'^T += A K with
@@ -297,9 +316,12 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
         __syncthreads();                                              // (C) window read
 
         // 5. The window buffers are free: start the next head's window.
-        if (t == 0 && un < units) {
-            mma_issue_window<K, V>(p, un, smem, L, wbar, 0u);
-            pending |= 2u;
+        {
+            const long long un = MIXED ? fq->next : u + gridDim.x;
+            if (t == 0 && un < units) {
+                mma_issue_window<K, V>(p, un, smem, L, wbar, 0u);
+                pending |= 2u;
+            }
         }
 
         // 6. True state S = Gamma_n S', written back (8 consecutive columns
@@ -375,14 +397,14 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
     }
     if (!ok && t == 0) {                                              // a bounded wait ran out
         report_timeout(p.status);
-        const int k_last = int((u - blockIdx.x) / gridDim.x);
+        const int k_last = MIXED ? k_fail : int((u - blockIdx.x) / gridDim.x);   // the head whose wait failed
         if (pending & 1u) mbar_wait(tbar, k_last & 1);                // own copies: one more bounded wait
         if (pending & 2u) mbar_wait(wbar, k_last & 1);
     }
 }
 
-template <int K, int V>
-cudaError_t flush_mma_t(const FlushParams& p, int rmax, cudaStream_t stream) {
+template <int K, int V, bool MIXED>
+cudaError_t flush_mma_launch(const FlushParams& p, int rmax, cudaStream_t stream) {
     const int n = p.n_ring + p.has_token;
     const int e16 = (((p.do_sketch ? rmax : 0) + p.has_token) + 15) & ~15;
     const int bytes = mma_layout(K, V, n, e16).total;
@@ -390,7 +412,7 @@ cudaError_t flush_mma_t(const FlushParams& p, int rmax, cudaStream_t stream) {
     CUtensorMap map;
     cudaError_t e = state_tensor_map(p.state, (long long)p.B * p.H * K, K, V, &map);
     if (e != cudaSuccess) return e;
-    auto kern = flush_mma_kernel<K, V>;
+    auto kern = flush_mma_kernel<K, V, MIXED>;
     static KernelCache kc;
     e = ensure_smem(kern, kc, bytes);
     if (e != cudaSuccess) return e;
@@ -402,6 +424,13 @@ cudaError_t flush_mma_t(const FlushParams& p, int rmax, cudaStream_t stream) {
     const long long grid = units < cap ? units : cap;
     kern<<<dim3(unsigned(grid)), dim3(MS<K, V>::T), bytes, stream>>>(p, map, e16);
     return cudaGetLastError();
+}
+
+// A mixed step (fill_in set) runs its own instance: the unit selection would
+// otherwise cost the uniform kernel registers it has none to spare for.
+template <int K, int V>
+cudaError_t flush_mma_t(const FlushParams& p, int rmax, cudaStream_t stream) {
+    return p.fill_in ? flush_mma_launch<K, V, true>(p, rmax, stream) : flush_mma_launch<K, V, false>(p, rmax, stream);
 }
 
 }  // namespace

@@ -32,6 +32,10 @@ struct FlushParams {
     int B, H, W, Wg, R;
     int n_ring, has_token, do_sketch, sketch_bf16;
     int stall;               // testing hook: extra bytes expected by the first bulk wait
+    // Mixed-phase steps (ss_step_mixed): only sequences b with fill_in[b] ==
+    // W-1 flush; each writes fill_out[b] = 0.  Null for a uniform batch.
+    const int32_t* fill_in;
+    int32_t* fill_out;
     int off[SS_MAX_HEADS + 1];
 };
 
@@ -57,6 +61,12 @@ struct StepParams {
     int B, H, W, Wg, R;
     int p, sketch_bf16;
     int stall;               // testing hook: extra bytes expected by the first bulk wait
+    // Mixed-phase steps (ss_step_mixed): sequence b appends at slot fill_in[b]
+    // (p is then the largest slot, W-2, which sizes the staging); sequences
+    // with fill_in[b] == W-1 are left to the flush; each other sequence
+    // writes fill_out[b] = fill_in[b] + 1.  Null for a uniform batch.
+    const int32_t* fill_in;
+    int32_t* fill_out;
     int off[SS_MAX_HEADS + 1];
 };
 

@@ -58,13 +58,12 @@ __device__ __forceinline__ unsigned unit_bytes(int P, int ubytes) {
     return n;
 }
 
-// Issue (one lane) the bulk copies of one unit: its live ring slots 0..p-1,
+// Issue (one lane) the bulk copies of one unit: its live ring slots 0..P-1,
 // `ubytes` of sketch rows from `usrc` (0 for replay) and the step's token.
 template <int FAM, int K, int V>
-__device__ __forceinline__ void stage_unit_bulk(const StepParams& p, long long unit, unsigned char* sh,
+__device__ __forceinline__ void stage_unit_bulk(const StepParams& p, long long unit, int P, unsigned char* sh,
                                                 const UnitSmem& L, const void* usrc, int ubytes,
                                                 uint64_t* bar, unsigned extra) {
-    const int P = p.p;
     mbar_expect_tx(bar, unit_bytes<FAM, K, V>(P, ubytes) + extra);
     const long long ring_row = unit * p.W;
     if (P > 0) {
@@ -530,7 +529,7 @@ __device__ __forceinline__ void axpy(float a, const float (&x)[E], float (&y)[E]
     for (int e = 0; e < E; ++e) y[e] = fmaf(a, x[e], y[e]);
 }
 
-template <int FAM, int K, int V, bool UB16>
+template <int FAM, int K, int V, bool UB16, bool MIXED>
 __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_constant__ StepParams p,
                                                                int rmax, int ns, int stage_bytes) {
     constexpr int G = dec_gl(FAM), UPW = 32 / G;
@@ -561,8 +560,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         const int s = it % ns;
         if (l == 0) {
             const int b = grp * UPW + g;
-            if (b < p.B)
-                stage_unit_bulk<FAM, K, V>(p, (long long)b * p.H + h, wbase + s * stage_bytes + 16 + g * L.total, L,
+            const int Pb = MIXED && b < p.B ? p.fill_in[b] : P;
+            if (b < p.B && Pb >= 0 && Pb < p.W - 1)
+                stage_unit_bulk<FAM, K, V>(p, (long long)b * p.H + h, Pb, wbase + s * stage_bytes + 16 + g * L.total, L,
                                            static_cast<const char*>(p.sketch) + (b * (long long)p.R + off) * (V * ESZ),
                                            r * V * ESZ, bar(s), (stall && it == 0 && g == 0) ? 16u : 0u);
             else
@@ -580,15 +580,19 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         if (r > 0) bulk_g2s(smem, p.coef + (long long)off * K, r * K * 4, cbar);
     }
     if (g0 >= ngroups) return;                              // warp 0 always has a group
-    for (int it = 0; it < ns - 1; ++it) issue(it);
+    for (int it = 0; it < ns; ++it) issue(it);              // before C arrives: the two latencies overlap
     bool ok = __all_sync(FULL, mbar_wait(cbar, 0));
     unsigned phases = 0;       // bit s: parity of the next phase of stage s
     int it = 0;
     for (int grp = g0; ok && grp < ngroups; ++it, grp += gstride) {
         const int s = it % ns;
-        issue(it + ns - 1);                                    // its stage was freed by the last group
+        if (it > 0) issue(it + ns - 1);                        // its stage was freed by the last group
         const int b = grp * UPW + g;
-        const bool active = b < p.B;
+        // this unit's ring position; in a mixed step, units at W-1 flush elsewhere
+        const int Pu = MIXED ? (b < p.B ? p.fill_in[b] : 0) : P;
+        const bool active = b < p.B && Pu >= 0 && Pu < p.W - 1;
+        if (MIXED && b < p.B && (Pu < 0 || Pu > p.W - 1) && h == 0 && l == 0 && p.status)
+            atomicOr(p.status, SS_DEVICE_BAD_FILL);              // neither decoded nor flushed
         const long long u = (long long)b * p.H + h;
         float tgate = 0.f, tbeta = 0.f;
         if (active) {
@@ -610,14 +614,15 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         const uint16_t* tv = reinterpret_cast<const uint16_t*>(sh + L.tv);
         const float* tg = reinterpret_cast<const float*>(sh + L.tg);
 
-        // 1. Append the token at ring slot P, bit for bit.
+        // 1. Append the token at ring slot Pu, bit for bit.
         if (active) {
-            const long long slot = u * p.W + P;
+            const long long slot = u * p.W + Pu;
             copy_row_bf16<K, G>(p.ring_k + slot * K, tk, l);
             copy_row_bf16<V, G>(p.ring_v + slot * V, tv, l);
             if (FAM == KDA) copy_row_f32<K, G>(p.ring_gate + slot * K, tg, l);
-            else if (l == 0) p.ring_gate[u * p.Wg + P] = tgate;
-            if (FAM != MAMBA2 && l == 0) p.ring_beta[u * p.Wg + P] = tbeta;
+            else if (l == 0) p.ring_gate[u * p.Wg + Pu] = tgate;
+            if (FAM != MAMBA2 && l == 0) p.ring_beta[u * p.Wg + Pu] = tbeta;
+            if (MIXED && h == 0 && l == 0) p.fill_out[b] = Pu + 1;
         }
 
         // 2. Backward sweep from the token (j = P) to slot 0: x_P = q,
@@ -628,7 +633,119 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         row_bf16<V, G>(tv, l, vj);
 #pragma unroll
         for (int e = 0; e < EV; ++e) ob[e] = 0.f;
-        if constexpr (FAM == MAMBA2) {
+        if constexpr (MIXED && FAM == MAMBA2) {
+            // The uniform sweep below, 4 rows at a time, walked to the warp's
+            // largest ring position: rows at or past this unit's own position
+            // read as zero with unit decay (dt = 0).
+            const int Pw = int(__reduce_max_sync(FULL, unsigned(active ? Pu : 0)));
+            axpy<EV>(tgate * gsum<G>(dot<EK>(kj, x)), vj, ob);
+            float gam = expf(A * tgate);
+            int j = Pw - 1;
+            for (; j >= 3; j -= 4) {
+                float d[4], a[4], dt[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float kk[EK];
+#pragma unroll
+                    for (int e = 0; e < EK; ++e) kk[e] = 0.f;
+                    dt[q] = 0.f;
+                    if (j - q < Pu) {
+                        row_bf16<K, G>(kraw + (j - q) * K, l, kk);
+                        dt[q] = gs[j - q];
+                    }
+                    d[q] = dot<EK>(kk, x);
+                    a[q] = expf(A * dt[q]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) d[q] = gsum<G>(d[q]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float vv[EV];
+#pragma unroll
+                    for (int e = 0; e < EV; ++e) vv[e] = 0.f;
+                    if (j - q < Pu) row_bf16<V, G>(vraw + (j - q) * V, l, vv);
+                    axpy<EV>(dt[q] * gam * d[q], vv, ob);
+                    gam *= a[q];
+                }
+            }
+            for (; j >= 0; --j) {
+#pragma unroll
+                for (int e = 0; e < EK; ++e) kj[e] = 0.f;
+#pragma unroll
+                for (int e = 0; e < EV; ++e) vj[e] = 0.f;
+                float dt = 0.f;
+                if (j < Pu) {
+                    row_bf16<K, G>(kraw + j * K, l, kj);
+                    row_bf16<V, G>(vraw + j * V, l, vj);
+                    dt = gs[j];
+                }
+                const float dj = gsum<G>(dot<EK>(kj, x));
+                axpy<EV>(dt * gam * dj, vj, ob);
+                gam *= expf(A * dt);
+            }
+#pragma unroll
+            for (int e = 0; e < EK; ++e) x[e] *= gam;
+        } else if constexpr (MIXED) {
+            // Units of one warp sit at different ring positions: every group
+            // walks to the warp's largest position, rows past its own are
+            // identities (zero key and value, unit decay).
+            const int Pw = int(__reduce_max_sync(FULL, unsigned(active ? Pu : 0)));
+            float gam = 1.f, aj[EK];
+            {
+                const float d = gsum<G>(dot<EK>(kj, x));
+                if constexpr (FAM == MAMBA2) {
+                    axpy<EV>(tgate * d, vj, ob);
+                    gam = expf(A * tgate);
+                } else {
+                    const float t = tbeta * d;
+                    axpy<EV>(t, vj, ob);
+                    if constexpr (FAM == GDN) {
+                        axpy<EK>(-t, kj, x);
+                        gam = tgate;
+                    } else {
+                        row_f32<K, G>(tg, l, aj);
+#pragma unroll
+                        for (int e = 0; e < EK; ++e) x[e] = aj[e] * fmaf(-t, kj[e], x[e]);
+                    }
+                }
+            }
+            for (int j = Pw - 1; j >= 0; --j) {
+                const bool own = j < Pu;
+#pragma unroll
+                for (int e = 0; e < EK; ++e) kj[e] = 0.f;
+#pragma unroll
+                for (int e = 0; e < EV; ++e) vj[e] = 0.f;
+                float gj = FAM == MAMBA2 ? 0.f : 1.f, bj = 0.f;
+                if (own) {
+                    row_bf16<K, G>(kraw + j * K, l, kj);
+                    row_bf16<V, G>(vraw + j * V, l, vj);
+                    if (FAM != KDA) gj = gs[j];
+                    if (FAM != MAMBA2) bj = bs[j];
+                }
+                const float d = gsum<G>(dot<EK>(kj, x));
+                if constexpr (FAM == MAMBA2) {
+                    axpy<EV>(gj * gam * d, vj, ob);            // gj = dt_j
+                    gam *= expf(A * gj);
+                } else if constexpr (FAM == GDN) {
+                    const float t = bj * d;
+                    axpy<EV>(gam * t, vj, ob);
+                    axpy<EK>(-t, kj, x);
+                    gam *= gj;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EK; ++e) aj[e] = 1.f;
+                    if (own) row_f32<K, G>(graw + j * K, l, aj);
+                    const float t = bj * d;
+                    axpy<EV>(t, vj, ob);
+#pragma unroll
+                    for (int e = 0; e < EK; ++e) x[e] = aj[e] * fmaf(-t, kj[e], x[e]);
+                }
+            }
+            if constexpr (FAM != KDA) {
+#pragma unroll
+                for (int e = 0; e < EK; ++e) x[e] *= gam;
+            }
+        } else if constexpr (FAM == MAMBA2) {
             // No erase term: every read uses q, scaled by the later decays
             // (gam = prod_{i > j} a_i).  The rows are independent, so they
             // are taken 4 at a time: loads, dots and reductions overlap.
@@ -801,7 +918,7 @@ __global__ void __launch_bounds__(128) replay_kernel(const __grid_constant__ Ste
         if (lane == 0) {
             mbar_init(bar, 1);
             fence_mbar_init();
-            stage_unit_bulk<FAM, K, V>(p, unit, sh, L, nullptr, 0, bar, p.stall && unit == 0 ? 16u : 0u);
+            stage_unit_bulk<FAM, K, V>(p, unit, p.p, sh, L, nullptr, 0, bar, p.stall && unit == 0 ? 16u : 0u);
         }
         const float tgate = FAM != KDA ? p.tok_gate[unit] : 0.f;
         const float tbeta = FAM != MAMBA2 ? p.tok_beta[unit] : 0.f;
@@ -852,7 +969,7 @@ int decode_stage(int fam, int K, int V, int P, int rmax, int esz) {
     return dec_stage_bytes(fam, K, V, P, rmax * V * esz);
 }
 
-template <int FAM, int K, int V, bool UB16>
+template <int FAM, int K, int V, bool UB16, bool MIXED>
 cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
     constexpr int esz = UB16 ? 2 : 4, upw = 32 / dec_gl(FAM);
     const int stage = decode_stage(FAM, K, V, p.p, rmax, esz);
@@ -861,7 +978,7 @@ cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
     int wpc = DEC_WARPS;
     while (wpc > 1 && cpart + wpc * stage > SMEM_LIMIT) --wpc;
     const int bytes = cpart + wpc * stage;
-    auto kern = decode_kernel<FAM, K, V, UB16>;
+    auto kern = decode_kernel<FAM, K, V, UB16, MIXED>;
     static KernelCache kc;
     cudaError_t e = ensure_smem(kern, kc, bytes);
     if (e != cudaSuccess) return e;
@@ -873,8 +990,11 @@ cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
 
 template <int FAM, int K, int V>
 cudaError_t decode_t(const StepParams& p, int rmax, cudaStream_t stream) {
-    return p.sketch_bf16 ? decode_launch<FAM, K, V, true>(p, rmax, stream)
-                         : decode_launch<FAM, K, V, false>(p, rmax, stream);
+    if (p.fill_in)
+        return p.sketch_bf16 ? decode_launch<FAM, K, V, true, true>(p, rmax, stream)
+                             : decode_launch<FAM, K, V, false, true>(p, rmax, stream);
+    return p.sketch_bf16 ? decode_launch<FAM, K, V, true, false>(p, rmax, stream)
+                         : decode_launch<FAM, K, V, false, false>(p, rmax, stream);
 }
 
 template <int FAM, int K, int V>

@@ -128,6 +128,12 @@ class DecodeLayer:
     def exact_step(self, tok, out=None, stream=None):
         B.ss_exact_step(self.plan, self.bufs(False), self.io(tok, out), stream)
 
+    def step_mixed(self, tok, fill_in, fill_out, out=None, stream=None):
+        """One step with a window position per sequence (int32 device tensors
+        of `batch` entries): sequences at W-1 flush, the rest decode;
+        fill_out receives (fill_in + 1) mod W."""
+        B.ss_step_mixed(self.plan, self.bufs(), self.io(tok, out), fill_in, fill_out, stream)
+
     def replay_step(self, tok, out=None, stream=None):
         if self.phase == self.window - 1:
             self.flush(tok, with_sketch=False, out=out, stream=stream)
