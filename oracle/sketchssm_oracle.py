@@ -39,8 +39,15 @@ Readings of points the pages leave open:
     KDA:     M_t = (I - beta_t k_t k_t^T) Diag(a_t), a_t in (0,1)^dk, b_t = beta_t.
 * P2 update-then-read: ``o_t = S_t^T q_t`` (the flush computes its output
   from the updated state, App. B).
-* P4 the coefficient map is a fixed per-head matrix C (the workloads use
-  C = P^T); the state-dependent map of §A.2.1 is not part of this oracle.
+* P4 the coefficient map is either a fixed per-head matrix C (the workloads
+  use C = P^T) or the state-dependent map of the project page ("Per window ·
+  Flush: Sketch & coefficient map", C = (U^T U)^+ U^T S0^T; paper §A.2.1),
+  refreshed with the sketch at every flush.  The pages call the map "exact
+  regularized" without giving the regulariser; this oracle takes a ridge
+  relative to the Gram matrix's mean diagonal, lambda = rho * tr(U^T U) / r,
+  so that rho = 0 is the pseudoinverse form for a full-column-rank U.  With a
+  bf16 sketch the map is built from the stored (rounded) U and is itself
+  stored rounded to bf16 ("reads the BF16 sketch and coefficient map", §D).
 * P7 a bf16 sketch is the fp64 sketch rounded once to bf16 (nearest, ties
   to even).
 
@@ -174,9 +181,28 @@ def sketch(S, P):
 
 
 def sketched_output(U, C, q_tilde, o_buf):
-    """o^ = U (C q~) + o_buf (project page, "Coefficient vector & readout")."""
-    c = np.einsum("rk,...k->...r", C, q_tilde)
+    """o^ = U (C q~) + o_buf (project page, "Coefficient vector & readout").
+    C is [r, K] (fixed, shared by the batch) or [..., r, K] (state-dependent)."""
+    c = np.einsum("...rk,...k->...r", C, q_tilde)
     return np.einsum("...vr,...r->...v", U, c) + o_buf
+
+
+def coefficient_map(U, S, rho=0.0):
+    """State-dependent coefficient map C = (U^T U + lambda I)^{-1} U^T S^T
+    (project page, "Per window · Flush: Sketch & coefficient map"; paper
+    §A.2.1): the map whose c = C q~ minimises ||S^T q~ - U c||_2 (plus
+    lambda ||c||^2).  lambda = rho * tr(U^T U) / r.
+    U [..., V, r], S [..., K, V] -> C [..., r, K]."""
+    U = np.asarray(U, dtype=np.float64)
+    S = np.asarray(S, dtype=np.float64)
+    r = U.shape[-1]
+    if r == 0:
+        return np.zeros(U.shape[:-2] + (0, S.shape[-2]))
+    G = np.einsum("...vr,...vs->...rs", U, U)              # U^T U
+    Z = np.einsum("...vr,...kv->...rk", U, S)              # U^T S^T
+    lam = rho * np.trace(G, axis1=-2, axis2=-1) / r
+    A = G + lam[..., None, None] * np.eye(r)
+    return np.linalg.solve(A, Z)
 
 
 def flush(family: int, S0, tokens, q=None):
@@ -200,7 +226,7 @@ class Session:
     """
 
     def __init__(self, family, state, window, A=None, basis=None, coef=None,
-                 offsets=None, sketch_bf16=False):
+                 offsets=None, sketch_bf16=False, state_map=False, rho=0.0):
         self.family = family
         self.S = np.asarray(state, dtype=np.float64).copy()     # [B, H, K, V]
         self.B, self.H, self.K, self.V = self.S.shape
@@ -214,8 +240,10 @@ class Session:
             self.P = [basis[self.offsets[h]:self.offsets[h + 1]].T for h in range(self.H)]
             self.C = [coef[self.offsets[h]:self.offsets[h + 1]] for h in range(self.H)]
         self.sketch_bf16 = sketch_bf16
+        self.state_map, self.rho = state_map, rho
         self.ring = []
         self.U = None
+        self.Cs = None             # state-dependent maps, list over heads of [B, r_h, K]
 
     # -- inputs -------------------------------------------------------------
     def token(self, inp):
@@ -237,6 +265,17 @@ class Session:
         if self.sketch_bf16:
             U = [round_bf16(u) for u in U]
         self.U = U
+        if self.state_map:
+            Cs = [coefficient_map(U[h], self.S[:, h], self.rho) for h in range(self.H)]
+            self.Cs = [round_bf16(c) for c in Cs] if self.sketch_bf16 else Cs
+
+    def coef(self, h):
+        """The coefficient map head h's reads use: [r, K] or [B, r, K]."""
+        return self.Cs[h] if self.state_map else self.C[h]
+
+    def packed_map(self):
+        """State-dependent maps in the library's packed layout [B][R][K]."""
+        return np.concatenate(self.Cs, axis=1)
 
     def packed_sketch(self):
         """Sketch in the library's packed layout [B][R][V] (row = u_i)."""
@@ -257,8 +296,10 @@ class Session:
         o_hat = np.empty((self.B, self.H, self.V))
         self.last_coefficients = []
         for h in range(self.H):
-            o_hat[:, h] = sketched_output(self.U[h], self.C[h], qt[:, h], o_buf[:, h])
-            self.last_coefficients.append(np.einsum("rk,bk->br", self.C[h], qt[:, h]))
+            C = self.coef(h)
+            o_hat[:, h] = sketched_output(self.U[h], C, qt[:, h], o_buf[:, h])
+            self.last_coefficients.append(np.einsum("brk,bk->br" if C.ndim == 3 else "rk,bk->br",
+                                                    C, qt[:, h]))
         return o_hat, read(self.S, qt) + o_buf
 
     def flush(self, inp=None, with_sketch=True):
@@ -273,7 +314,7 @@ class Session:
         if with_sketch:
             self._make_sketch()
         else:
-            self.U = None
+            self.U = self.Cs = None
         return o
 
     def step(self, inp):

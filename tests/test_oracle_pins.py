@@ -331,6 +331,93 @@ def test_synth_ranks_and_basis():
 
 
 # ----------------------------------------------------------------------------
+# 9b. state-dependent coefficient map (project page, "Per window · Flush:
+#     Sketch & coefficient map", C = (U^T U)^+ U^T S0^T; paper §A.2.1: the
+#     coefficients minimise ||S0^T q~ - U c||_2)
+# ----------------------------------------------------------------------------
+def _map_case(seed, n=4, K=12, V=20, r=5):
+    rng = np.random.default_rng(seed)
+    S = rng.standard_normal((n, K, V))
+    P = np.linalg.qr(rng.standard_normal((K, K)))[0][:, :r]
+    q = rng.standard_normal((n, K))
+    return S, P, orc.sketch(S, P), q
+
+
+def test_coefficient_map_is_least_squares():
+    """c = C q~ is numpy's least-squares solution of min_c ||S^T q~ - U c||."""
+    S, P, U, q = _map_case(1)
+    C = orc.coefficient_map(U, S)
+    for i in range(len(S)):
+        c_ls = np.linalg.lstsq(U[i], S[i].T @ q[i], rcond=None)[0]
+        assert relerr(C[i] @ q[i], c_ls) < 1e-10
+
+
+def test_coefficient_map_residual_is_orthogonal_to_sketch():
+    """Normal equations: the readout error S^T q~ - U C q~ is orthogonal to every u_i."""
+    S, P, U, q = _map_case(2, K=16, V=9, r=6)
+    C = orc.coefficient_map(U, S)
+    res = np.einsum("nkv,nk->nv", S, q) - np.einsum("nvr,nrk,nk->nv", U, C, q)
+    assert np.abs(np.einsum("nvr,nv->nr", U, res)).max() < 1e-10 * np.abs(res).max()
+
+
+def test_coefficient_map_full_rank_is_identity():
+    """r = K <= V with a square orthogonal basis P: U = S^T P has full column
+    rank, so C = (P^T S S^T P)^{-1} P^T S S^T = P^T and every read is exact."""
+    S, P, U, q = _map_case(3, K=8, V=20, r=8)
+    C = orc.coefficient_map(U, S)
+    assert relerr(C, np.broadcast_to(P.T, C.shape)) < 1e-10
+    o = np.einsum("nkv,nk->nv", S, q)
+    assert relerr(orc.sketched_output(U, C, q, 0.0), o) < 1e-10
+
+
+def test_coefficient_map_ridge_is_augmented_least_squares():
+    """With the ridge, c = C q~ solves min ||S^T q~ - U c||^2 + lambda ||c||^2,
+    lambda = rho tr(U^T U) / r: the stacked system [U; sqrt(lambda) I] c ~ [S^T q~; 0]."""
+    S, P, U, q = _map_case(4)
+    rho = 0.3
+    C = orc.coefficient_map(U, S, rho)
+    r = U.shape[-1]
+    for i in range(len(S)):
+        lam = rho * np.sum(U[i] * U[i]) / r
+        A = np.vstack([U[i], np.sqrt(lam) * np.eye(r)])
+        y = np.concatenate([S[i].T @ q[i], np.zeros(r)])
+        assert relerr(C[i] @ q[i], np.linalg.lstsq(A, y, rcond=None)[0]) < 1e-10
+
+
+def test_state_map_never_worse_than_fixed_map():
+    """The least-squares map reads at least as well as the fixed C = P^T."""
+    S, P, U, q = _map_case(5, K=32, V=16, r=6)
+    o = np.einsum("nkv,nk->nv", S, q)
+    e_state = np.linalg.norm(o - orc.sketched_output(U, orc.coefficient_map(U, S), q, 0.0), axis=-1)
+    e_fixed = np.linalg.norm(o - orc.sketched_output(U, P.T, q, 0.0), axis=-1)
+    assert (e_state <= e_fixed * (1 + 1e-12)).all() and (e_state < e_fixed).any()
+
+
+@pytest.mark.parametrize("family", FAMS)
+def test_session_state_map_identity_basis_reads_exactly(family):
+    """Session with the state map and P = I (r = K <= V): every sketched read
+    equals the exact windowed read (C = I)."""
+    from ssm_decode_b200 import synth
+    rng = np.random.default_rng(6)
+    B, H, K, V, W = 2, 2, 4, 6, 4
+    S0 = rng.standard_normal((B, H, K, V))
+    offsets = np.arange(H + 1) * K
+    basis = np.tile(np.eye(K), (H, 1))
+    A = -np.exp(rng.uniform(0, 1, H))
+    sess = orc.Session(family, S0, W, A, basis, basis, offsets, state_map=True)
+    sess.prime()
+    for _ in range(W - 1):
+        inp = {"q": synth.f32_to_bf16_bits(rng.standard_normal((B, H, K))),
+               "k": synth.f32_to_bf16_bits(rng.standard_normal((B, H, K)) / 2),
+               "v": synth.f32_to_bf16_bits(rng.standard_normal((B, H, V))),
+               "gate": (rng.uniform(0.2, 0.9, (B, H, K)) if family == orc.KDA
+                        else rng.uniform(0.2, 0.9, (B, H))),
+               "beta": rng.uniform(0.1, 0.9, (B, H))}
+        o_hat, o = sess.decode(inp)
+        assert relerr(o_hat, o) < 1e-9
+
+
+# ----------------------------------------------------------------------------
 # 10. planted mistakes must fail a pin
 # ----------------------------------------------------------------------------
 def _run_pins():
@@ -350,6 +437,41 @@ def _run_pins():
     except AssertionError:
         return False
     return True
+
+
+def _run_map_pins():
+    try:
+        test_coefficient_map_is_least_squares()
+        test_coefficient_map_residual_is_orthogonal_to_sketch()
+        test_coefficient_map_full_rank_is_identity()
+        test_coefficient_map_ridge_is_augmented_least_squares()
+        test_state_map_never_worse_than_fixed_map()
+    except AssertionError:
+        return False
+    return True
+
+
+ORIG_MAP = orc.coefficient_map
+
+
+def _mut_map_no_ridge(U, S, rho=0.0):
+    return ORIG_MAP(U, S, 0.0)
+
+
+def _mut_map_sign(U, S, rho=0.0):
+    return -ORIG_MAP(U, S, rho)
+
+
+def _mut_map_gram_only(U, S, rho=0.0):
+    # skips the Gram solve: C = U^T S^T
+    return np.einsum("...vr,...kv->...rk", U, S)
+
+
+@pytest.mark.parametrize("mutant", [_mut_map_no_ridge, _mut_map_sign, _mut_map_gram_only])
+def test_planted_map_mistakes_are_caught(monkeypatch, mutant):
+    assert _run_map_pins()
+    monkeypatch.setattr(orc, "coefficient_map", mutant)
+    assert not _run_map_pins(), "a mistake planted in coefficient_map went unnoticed"
 
 
 def _mut_erase_sign(family, x, k, a, b):
