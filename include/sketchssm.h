@@ -44,6 +44,8 @@
  *   sketch     float or bf16 [B][R][dv]       row off_h + i is u_i = S^T omega_i of head h
  *   basis      float    [R][dk]               row off_h + i is omega_i of head h (shared by the batch)
  *   coef       float    [R][dk]               rows off_h .. off_h + r_h - 1 are head h's map C
+ *   coef_state float or bf16 [B][R][dk]       SS_COEF_STATE: sequence b's map rows of head h at
+ *                                             off_h .. off_h + r_h - 1 (dtype of the sketch)
  *   A          float    [H]                   Mamba-2 decay rates (A_h < 0 for decay)
  *   q, k       uint16_t [B][H][dk] bf16;  v uint16_t [B][H][dv] bf16
  *   gate       float    [B][H] (Mamba-2 dt, GDN a) or [B][H][dk] (KDA a)
@@ -89,6 +91,22 @@ typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_sketch_dtype;
 /* Set by ss_step_mixed when a fill count lies outside 0..W-1: that sequence
  * is neither decoded nor flushed and its fill_out entry is left as it was. */
 #define SS_DEVICE_BAD_FILL 2
+/* Set by a flush in SS_COEF_STATE mode when a head's Gram matrix
+ * U^T U + lambda I is not numerically positive definite (a Cholesky pivot
+ * <= 0 or not finite, e.g. an all-zero state with rho = 0): that head's map
+ * rows are written as zeros. */
+#define SS_DEVICE_SINGULAR_MAP 4
+
+/* Which coefficient map the non-flush read c = C q~ uses (project page,
+ * "Per step · Non-flush: Coefficient vector & readout"). */
+typedef enum {
+    SS_COEF_FIXED = 0,       /* C = bufs->coef: one fp32 [R][dk] map shared by the batch */
+    SS_COEF_STATE = 1        /* per (sequence, head) map C = (U^T U + lambda I)^-1 U^T S^T,
+                              * lambda = rho tr(U^T U) / r (project page, "Per window ·
+                              * Flush: Sketch & coefficient map"; paper §A.2.1), rebuilt
+                              * by every flush from the new state and sketch, fused into
+                              * it (no second state read); stored in bufs->coef_state */
+} ss_coef_mode;
 
 typedef struct {
     int32_t family;          /* ss_family */
@@ -99,6 +117,8 @@ typedef struct {
     int32_t window;          /* W: steps per flush window */
     const int32_t* ranks;    /* host [heads]: sketch rank r_h of each head; copied */
     int32_t sketch_dtype;    /* ss_sketch_dtype of the stored sketch U */
+    int32_t coef_mode;       /* ss_coef_mode; 0 (zero-initialised) = SS_COEF_FIXED */
+    float coef_ridge;        /* rho >= 0 of SS_COEF_STATE (ignored otherwise) */
 } ss_config;
 
 typedef struct ss_plan ss_plan;
@@ -106,6 +126,7 @@ typedef struct ss_plan ss_plan;
 typedef struct {
     size_t state, ring_k, ring_v, ring_gate, ring_beta, sketch, basis, coef, A;
     size_t q, k, v, gate, beta, out;
+    size_t coef_state;       /* SS_COEF_STATE: [B][R][dk] in the sketch dtype; else 0 */
     int32_t total_rank;      /* R = sum of ranks */
     int32_t gate_stride;     /* Wg (scalar-gate families) or W * dk (KDA), floats per (b, h) */
 } ss_sizes;
@@ -121,6 +142,10 @@ typedef struct {
     const float* coef;       /* needed by ss_decode_step */
     const float* A;          /* needed for Mamba-2 */
     int32_t* status;         /* optional device int32 (4-byte aligned), see SS_DEVICE_TIMEOUT; NULL: no report */
+    void* coef_state;        /* SS_COEF_STATE only: device [B][R][dk] in the sketch dtype, the
+                              * per-(sequence, head) maps (head h's rows at the rank offset,
+                              * like the sketch); written by ss_prime / ss_flush with a sketch,
+                              * read by ss_decode_step; bufs->coef is then unused */
 } ss_buffers;
 
 typedef struct {
@@ -166,8 +191,10 @@ typedef struct {
  * warp, the window's ring slots and sketch rows plus the head's map C
  * (rmax x dk fp32), so very large ranks with long windows may not fit (KDA
  * with rank 128, dk = dv = 128 and W = 32 does not).  Every rank up to 64 at W <= 16,
- * and up to 32 at W <= 32, is supported.  The plan starts at phase 0
- * with no valid sketch. */
+ * and up to 32 at W <= 32, is supported.  SS_COEF_STATE needs every rank
+ * <= dv (U^T U must be invertible) and a finite coef_ridge >= 0; its flushes
+ * run on the CUDA-core flush kernel for every family.  The plan starts at
+ * phase 0 with no valid sketch. */
 ss_status ss_create(const ss_config* cfg, ss_plan** out);
 ss_status ss_destroy(ss_plan* plan);
 

@@ -202,7 +202,16 @@ def coefficient_map(U, S, rho=0.0):
     Z = np.einsum("...vr,...kv->...rk", U, S)              # U^T S^T
     lam = rho * np.trace(G, axis1=-2, axis2=-1) / r
     A = G + lam[..., None, None] * np.eye(r)
-    return np.linalg.solve(A, Z)
+    # A Gram matrix that is not positive definite (e.g. an all-zero state
+    # with rho = 0) has no such map; the library then stores zeros.
+    C = np.zeros(Z.shape)
+    for idx in np.ndindex(A.shape[:-2]):
+        try:
+            np.linalg.cholesky(A[idx])
+        except np.linalg.LinAlgError:
+            continue
+        C[idx] = np.linalg.solve(A[idx], Z[idx])
+    return C
 
 
 def flush(family: int, S0, tokens, q=None):
@@ -293,6 +302,7 @@ class Session:
         q, tok = self.token(inp)
         self.ring.append(tok)
         qt, o_buf = effective_query(self.family, self.ring, q)
+        self.last_q_tilde, self.last_o_buf = qt, o_buf
         o_hat = np.empty((self.B, self.H, self.V))
         self.last_coefficients = []
         for h in range(self.H):

@@ -18,6 +18,8 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "sketchssm.h")
 SS_OK, SS_ERR_INVALID_ARG, SS_ERR_ALIGNMENT, SS_ERR_UNSUPPORTED, SS_ERR_SCHEDULE, SS_ERR_CUDA = range(6)
 SS_DEVICE_TIMEOUT = 1
 SS_DEVICE_BAD_FILL = 2
+SS_DEVICE_SINGULAR_MAP = 4
+SS_COEF_FIXED, SS_COEF_STATE = 0, 1
 SS_MAMBA2, SS_GDN, SS_KDA = 0, 1, 2
 SS_F32, SS_BF16 = 0, 1
 (SS_OP_DECODE, SS_OP_FLUSH, SS_OP_FLUSH_NO_TOKEN, SS_OP_PRIME, SS_OP_EXACT, SS_OP_REPLAY,
@@ -27,20 +29,21 @@ SS_F32, SS_BF16 = 0, 1
 class ss_config(ctypes.Structure):
     _fields_ = [("family", ctypes.c_int32), ("batch", ctypes.c_int32), ("heads", ctypes.c_int32),
                 ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("window", ctypes.c_int32),
-                ("ranks", ctypes.POINTER(ctypes.c_int32)), ("sketch_dtype", ctypes.c_int32)]
+                ("ranks", ctypes.POINTER(ctypes.c_int32)), ("sketch_dtype", ctypes.c_int32),
+                ("coef_mode", ctypes.c_int32), ("coef_ridge", ctypes.c_float)]
 
 
 class ss_sizes(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("state", "ring_k", "ring_v", "ring_gate", "ring_beta", "sketch", "basis", "coef", "A",
-                 "q", "k", "v", "gate", "beta", "out")] + \
+                 "q", "k", "v", "gate", "beta", "out", "coef_state")] + \
                [("total_rank", ctypes.c_int32), ("gate_stride", ctypes.c_int32)]
 
 
 class ss_buffers(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("state", "ring_k", "ring_v", "ring_gate", "ring_beta", "sketch", "basis", "coef", "A",
-                 "status")]
+                 "status", "coef_state")]
 
 
 class ss_step_io(ctypes.Structure):
@@ -138,7 +141,7 @@ def _dt():
 
 
 def make_buffers(state=None, ring_k=None, ring_v=None, ring_gate=None, ring_beta=None, sketch=None,
-                 basis=None, coef=None, A=None, status=None):
+                 basis=None, coef=None, A=None, status=None, coef_state=None):
     import torch
     d = _dt()
     return ss_buffers(_ptr(state, "state", d["f32"]), _ptr(ring_k, "ring_k", d["bf16"]),
@@ -146,7 +149,8 @@ def make_buffers(state=None, ring_k=None, ring_v=None, ring_gate=None, ring_beta
                       _ptr(ring_beta, "ring_beta", d["f32"]),
                       _ptr(sketch, "sketch", d["f32"] + d["bf16"]), _ptr(basis, "basis", d["f32"]),
                       _ptr(coef, "coef", d["f32"]), _ptr(A, "A", d["f32"]),
-                      _ptr(status, "status", (torch.int32,)))
+                      _ptr(status, "status", (torch.int32,)),
+                      _ptr(coef_state, "coef_state", d["f32"] + d["bf16"]))
 
 
 def make_step_io(q, k, v, gate, beta, out):
@@ -171,15 +175,18 @@ def _stream(stream):
 class Plan:
     """Owns an ss_plan*; destroyed with the object."""
 
-    def __init__(self, family, batch, heads, dk, dv, window, ranks, sketch_dtype=SS_F32):
+    def __init__(self, family, batch, heads, dk, dv, window, ranks, sketch_dtype=SS_F32,
+                 coef_mode=SS_COEF_FIXED, coef_ridge=0.0):
         self.ranks = (ctypes.c_int32 * heads)(*[int(r) for r in ranks])
         cfg = ss_config(family, batch, heads, dk, dv, window,
-                        ctypes.cast(self.ranks, ctypes.POINTER(ctypes.c_int32)), sketch_dtype)
+                        ctypes.cast(self.ranks, ctypes.POINTER(ctypes.c_int32)), sketch_dtype,
+                        coef_mode, coef_ridge)
         h = ctypes.c_void_p()
         _check(lib().ss_create(ctypes.byref(cfg), ctypes.byref(h)))
         self.handle = h
         self.family, self.batch, self.heads, self.dk, self.dv, self.window = family, batch, heads, dk, dv, window
         self.sketch_dtype = sketch_dtype
+        self.coef_mode, self.coef_ridge = coef_mode, coef_ridge
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -188,8 +195,9 @@ class Plan:
             self.handle = None
 
 
-def ss_create(family, batch, heads, dk, dv, window, ranks, sketch_dtype=SS_F32):
-    return Plan(family, batch, heads, dk, dv, window, ranks, sketch_dtype)
+def ss_create(family, batch, heads, dk, dv, window, ranks, sketch_dtype=SS_F32, coef_mode=SS_COEF_FIXED,
+              coef_ridge=0.0):
+    return Plan(family, batch, heads, dk, dv, window, ranks, sketch_dtype, coef_mode, coef_ridge)
 
 
 def ss_buffer_sizes(plan):

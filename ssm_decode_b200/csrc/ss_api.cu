@@ -11,8 +11,9 @@
 #include "ss_internal.h"
 
 namespace ss {
-int flush_smem_bytes(int family, int dk, int dv, int n, int rpad);
-int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz);
+int flush_smem_bytes(int family, int dk, int dv, int n, int rpad, bool smap);
+int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz, bool smap);
+bool flush_map_fits(int dk, int dv, int r);
 }  // namespace ss
 
 struct ss_plan {
@@ -67,6 +68,14 @@ ss_status check_status(const ss_buffers* b) {
     return SS_OK;
 }
 
+bool state_map(const ss_plan* pl) { return pl->cfg.coef_mode == SS_COEF_STATE; }
+
+// The map buffer a flush that refreshes the sketch must also refresh.
+ss_status check_map(const ss_plan* pl, const ss_buffers* b) {
+    if (state_map(pl)) REQUIRE_PTR(b->coef_state, "bufs->coef_state");
+    return SS_OK;
+}
+
 // Consume the testing hook: the stall applies to one launch only.
 int take_stall(ss_plan* pl) {
     const int s = pl->stall_next;
@@ -113,6 +122,10 @@ ss::FlushParams flush_params(const ss_plan* pl, const ss_buffers* b, const ss_st
     p.status = b->status;
     p.B = pl->cfg.batch; p.H = pl->cfg.heads; p.W = pl->cfg.window; p.Wg = pl->Wg; p.R = pl->R;
     p.sketch_bf16 = pl->cfg.sketch_dtype == SS_BF16;
+    if (state_map(pl) && b->sketch != nullptr) {
+        p.cmap = b->coef_state;
+        p.ridge = pl->cfg.coef_ridge;
+    }
     std::memcpy(p.off, pl->off, sizeof(int32_t) * (pl->cfg.heads + 1));
     return p;
 }
@@ -127,6 +140,7 @@ ss::StepParams step_params(const ss_plan* pl, const ss_buffers* b, const ss_step
     p.B = pl->cfg.batch; p.H = pl->cfg.heads; p.W = pl->cfg.window; p.Wg = pl->Wg; p.R = pl->R;
     p.p = pl->phase;
     p.sketch_bf16 = pl->cfg.sketch_dtype == SS_BF16;
+    if (state_map(pl)) p.cmap = b->coef_state;
     std::memcpy(p.off, pl->off, sizeof(int32_t) * (pl->cfg.heads + 1));
     return p;
 }
@@ -159,6 +173,10 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
     if (c.sketch_dtype != SS_F32 && c.sketch_dtype != SS_BF16)
         return fail(SS_ERR_INVALID_ARG, "unknown sketch dtype %d", c.sketch_dtype);
     if (c.ranks == nullptr) return fail(SS_ERR_INVALID_ARG, "ranks is NULL");
+    if (c.coef_mode != SS_COEF_FIXED && c.coef_mode != SS_COEF_STATE)
+        return fail(SS_ERR_INVALID_ARG, "unknown coef_mode %d", c.coef_mode);
+    if (c.coef_mode == SS_COEF_STATE && !(c.coef_ridge >= 0.f && c.coef_ridge < 3.0e38f))
+        return fail(SS_ERR_INVALID_ARG, "coef_ridge must be finite and >= 0");
     if ((long long)c.batch * c.heads > (1ll << 31) / 2)
         return fail(SS_ERR_UNSUPPORTED, "batch * heads too large");
     ss_plan* pl = new (std::nothrow) ss_plan;
@@ -174,6 +192,11 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
             delete pl;
             return fail(SS_ERR_INVALID_ARG, "ranks[%d] = %d outside 0..dk", h, r);
         }
+        if (c.coef_mode == SS_COEF_STATE && !ss::flush_map_fits(c.dk, c.dv, r)) {
+            delete pl;
+            return fail(SS_ERR_UNSUPPORTED, "ranks[%d] = %d: the state-dependent map needs rank <= dv and "
+                        "room for U and its Gram matrix in the flush's tile buffer", h, r);
+        }
         pl->ranks[h] = r;
         pl->off[h + 1] = pl->off[h] + r;
         if (r > pl->rmax) pl->rmax = r;
@@ -182,8 +205,9 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
     pl->Wg = (c.window + 3) & ~3;
     // Every launch must fit one head (flush) or one warp (decode) in shared memory.
     const int rpad = (pl->rmax + 1 + 3) & ~3;
-    const int fl = ss::flush_smem_bytes(c.family, c.dk, c.dv, c.window, rpad);
-    const int dec = ss::decode_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax, esize(pl));
+    const bool smap = c.coef_mode == SS_COEF_STATE;
+    const int fl = ss::flush_smem_bytes(c.family, c.dk, c.dv, c.window, rpad, smap);
+    const int dec = ss::decode_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax, esize(pl), smap);
     if (fl > kSmemLimit || dec > kSmemLimit) {
         const int rmax = pl->rmax;
         delete pl;
@@ -219,6 +243,7 @@ ss_status ss_buffer_sizes(const ss_plan* pl, ss_sizes* out) {
     out->gate = (c.family == SS_KDA ? BH * K : BH) * 4;
     out->beta = c.family == SS_MAMBA2 ? 0 : BH * 4;
     out->out = BH * V * 4;
+    out->coef_state = state_map(pl) ? size_t(c.batch) * pl->R * K * esize(pl) : 0;
     out->total_rank = pl->R;
     out->gate_stride = c.family == SS_KDA ? c.window * c.dk : pl->Wg;
     return ok();
@@ -247,6 +272,7 @@ ss_status ss_prime(ss_plan* pl, const ss_buffers* b, ss_stream stream) {
     REQUIRE_PTR(b->state, "bufs->state");
     REQUIRE_PTR(b->sketch, "bufs->sketch");
     REQUIRE_PTR(b->basis, "bufs->basis");
+    CHECK(check_map(pl, b));
     CHECK(check_status(b));
     ss::FlushParams p = flush_params(pl, b, nullptr);
     p.n_ring = 0; p.has_token = 0; p.do_sketch = 1;
@@ -266,7 +292,8 @@ ss_status ss_decode_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io,
         return fail(SS_ERR_SCHEDULE, "ss_decode_step needs a current sketch (ss_prime or ss_flush first)");
     CHECK(check_ring(pl, b));
     REQUIRE_PTR(b->sketch, "bufs->sketch");
-    REQUIRE_PTR(b->coef, "bufs->coef");
+    if (state_map(pl)) CHECK(check_map(pl, b));
+    else REQUIRE_PTR(b->coef, "bufs->coef");
     CHECK(check_io(pl, io));
     CHECK(check_status(b));
     ss::StepParams p = step_params(pl, b, io);
@@ -288,6 +315,7 @@ ss_status ss_flush(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_st
     if (sk) {
         REQUIRE_PTR(b->sketch, "bufs->sketch");
         REQUIRE_PTR(b->basis, "bufs->basis");
+        CHECK(check_map(pl, b));
     }
     CHECK(check_status(b));
     ss::FlushParams p = flush_params(pl, b, io);
@@ -351,7 +379,8 @@ ss_status ss_step_mixed(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
     REQUIRE_PTR(b->state, "bufs->state");
     REQUIRE_PTR(b->sketch, "bufs->sketch");
     REQUIRE_PTR(b->basis, "bufs->basis");
-    REQUIRE_PTR(b->coef, "bufs->coef");
+    if (state_map(pl)) CHECK(check_map(pl, b));
+    else REQUIRE_PTR(b->coef, "bufs->coef");
     if (pl->cfg.family == SS_MAMBA2) REQUIRE_PTR(b->A, "bufs->A");
     CHECK(check_io(pl, io));
     CHECK(check_status(b));
@@ -397,26 +426,28 @@ ss_status ss_traffic_bytes(const ss_plan* pl, int32_t op, int32_t tau, ss_traffi
     const double bh = B * H;
     const double basis_bytes = R * K * 4;                // once per head per launch
     const double sketch_bytes = B * R * V * sk;          // U of every sequence
+    const bool smap = c.coef_mode == SS_COEF_STATE;
+    const double map_bytes = smap ? B * R * K * sk : 0;  // per-sequence maps (SS_COEF_STATE)
     const double paper_tg = B * R * (K + V) * 2 + (m2 ? 0 : B * R * W * 2);
     switch (op) {
         case SS_OP_DECODE:
-            rd = bh * (tok + tau * slot) + sketch_bytes + basis_bytes + A;
+            rd = bh * (tok + tau * slot) + sketch_bytes + (smap ? map_bytes : basis_bytes) + A;
             wr = bh * (slot + 4 * V);
             prd = paper_tg;
             break;
         case SS_OP_FLUSH:
             rd = bh * (D + (W - 1) * slot + tok) + basis_bytes + A;
-            wr = bh * (D + 4 * V) + sketch_bytes;
+            wr = bh * (D + 4 * V) + sketch_bytes + map_bytes;
             prd = bh * D; pwr = bh * D;
             break;
         case SS_OP_FLUSH_NO_TOKEN:
             rd = bh * (D + tau * slot) + basis_bytes + A;
-            wr = bh * D + sketch_bytes;
+            wr = bh * D + sketch_bytes + map_bytes;
             prd = bh * D; pwr = bh * D;
             break;
         case SS_OP_PRIME:
             rd = bh * D + basis_bytes;
-            wr = sketch_bytes;
+            wr = sketch_bytes + map_bytes;
             prd = bh * D;
             break;
         case SS_OP_EXACT:

@@ -302,7 +302,158 @@ __device__ __forceinline__ void prepare_head(const FlushParams& p, int h, int n,
     }
 }
 
-template <int FAM, int K, int V, bool MIXED>
+// Whether the coefficient map of a rank-r head fits the flush's scratch: the
+// tile buffer (dk x dv floats) holds U (r x dv), then per-warp partial sums of
+// at least one map row (dv/16 warps x dk) and later the Gram matrix (r x r).
+__host__ __device__ inline bool map_fits(int K, int V, int r) {
+    const int free_floats = K * V - r * V;
+    return r <= V && free_floats >= (V / 16) * K && free_floats >= r * r;
+}
+
+// State-dependent coefficient map of one head (project page, "Per window ·
+// Flush: Sketch & coefficient map"; paper §A.2.1):
+//     C = (U^T U + lambda I)^-1 U^T S^T,  lambda = ridge * tr(U^T U) / r,
+// from the updated state S (this thread's R x 4 tile in `st`) and the sketch
+// U as stored (r x dv in the tile buffer, written by the read-out).  No
+// second pass over HBM: the state is still in registers.
+//   1. Z = U^T S^T (r x dk): each thread contracts its 4 columns, a 2-level
+//      reduce-scatter over the 4 column lanes leaves R/4 rows per lane, and
+//      the dv/16 warps' partials are summed through shared memory, EC rows
+//      of Z at a time.  Z lands in the extended-basis buffer (free now).
+//   2. G = U^T U (lower triangle) in the tile buffer; warp 0 factors
+//      G + lambda I = L L^T (Cholesky, column by column).
+//   3. Thread k solves L L^T c = Z[:, k] for column k in place; the columns
+//      are C's, written in the sketch dtype.  A pivot that is not positive
+//      and finite zeroes the head's map and sets SS_DEVICE_SINGULAR_MAP.
+template <int K, int V>
+__device__ __forceinline__ void build_map(const FlushParams& p, const float2 (&st)[K / 8][2], int r,
+                                          long long b, int h, unsigned char* smem, const FlushLayout& L,
+                                          int t) {
+    using S = FS<K, V>;
+    constexpr int T = S::T, R = S::R, NW = T / 32;
+    const int lane = t & 31, warp = t >> 5;
+    const int cgw = lane & 3, rb = lane >> 2;
+    const int c0 = warp * 16 + cgw * 4, row0 = rb * R;
+    const int b0 = cgw & 1, b1 = (cgw >> 1) & 1;
+    float* umap = reinterpret_cast<float*>(smem + L.tile);     // [r][V]
+    float* zp = umap + r * V;                                  // [EC][NW][K], then G [r][r]
+    float* zs = reinterpret_cast<float*>(smem + L.pt);         // [r][K]: Z, then C
+    __shared__ int map_ok;
+    const int EC = min(r, (K * V - r * V) / (NW * K));
+    __syncthreads();                                           // (D) U written, basis rows read
+
+    // 1. Z = U^T S^T
+    for (int e0 = 0; e0 < r; e0 += EC) {
+        const int ne = min(EC, r - e0);
+        for (int el = 0; el < ne; ++el) {
+            const float4 uu = *reinterpret_cast<const float4*>(umap + (e0 + el) * V + c0);
+            float z[R];
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                float2 pp = fmul2(st[i][0], make_float2(uu.x, uu.y));
+                pp = ffma2(st[i][1], make_float2(uu.z, uu.w), pp);
+                z[i] = pp.x + pp.y;
+            }
+            float z2[R / 2];                                   // lane bit 0: which half of the rows
+#pragma unroll
+            for (int i = 0; i < R / 2; ++i) {
+                const float keep = b0 ? z[i + R / 2] : z[i], send = b0 ? z[i] : z[i + R / 2];
+                z2[i] = keep + __shfl_xor_sync(FULL, send, 1);
+            }
+            float z4[R / 4];                                   // lane bit 1: which quarter
+#pragma unroll
+            for (int i = 0; i < R / 4; ++i) {
+                const float keep = b1 ? z2[i + R / 4] : z2[i], send = b1 ? z2[i] : z2[i + R / 4];
+                z4[i] = keep + __shfl_xor_sync(FULL, send, 2);
+            }
+            float* dst = zp + (el * NW + warp) * K + row0 + b0 * (R / 2) + b1 * (R / 4);
+#pragma unroll
+            for (int i = 0; i < R / 4; ++i) dst[i] = z4[i];
+        }
+        __syncthreads();
+        for (int idx = t; idx < ne * K; idx += T) {
+            const int el = idx / K, k = idx - el * K;
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) sum += zp[(el * NW + w) * K + k];
+            zs[(e0 + el) * K + k] = sum;
+        }
+        __syncthreads();
+    }
+
+    // 2. G = U^T U (lower triangle), then G + lambda I = L L^T in place
+    float* g = zp;
+    for (int idx = t; idx < r * r; idx += T) {
+        const int e = idx / r, f = idx - e * r;
+        if (f > e) continue;
+        const float* ue = umap + e * V;
+        const float* uf = umap + f * V;
+        float sum = 0.f;
+        for (int v = 0; v < V; v += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(ue + v);
+            const float4 c = *reinterpret_cast<const float4*>(uf + v);
+            sum = fmaf(a.x, c.x, sum);
+            sum = fmaf(a.y, c.y, sum);
+            sum = fmaf(a.z, c.z, sum);
+            sum = fmaf(a.w, c.w, sum);
+        }
+        g[e * r + f] = sum;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        float tr = 0.f;
+        for (int e = lane; e < r; e += 32) tr += g[e * r + e];
+        const float lam = p.ridge * warp_sum(tr) / float(r);
+        bool good = true;
+        for (int j = 0; j < r && good; ++j) {
+            float part = 0.f;
+            for (int k = lane; k < j; k += 32) part = fmaf(g[j * r + k], g[j * r + k], part);
+            const float piv = g[j * r + j] + lam - warp_sum(part);
+            good = piv > 0.f && piv < INFINITY;                // the same value in every lane
+            if (!good) break;
+            const float d = sqrtf(piv);
+            __syncwarp();
+            for (int i = j + 1 + lane; i < r; i += 32) {
+                float acc = g[i * r + j];
+                for (int k = 0; k < j; ++k) acc = fmaf(-g[i * r + k], g[j * r + k], acc);
+                g[i * r + j] = acc / d;
+            }
+            __syncwarp();
+            if (lane == 0) g[j * r + j] = d;
+            __syncwarp();
+        }
+        if (lane == 0) {
+            map_ok = good;
+            if (!good && p.status != nullptr) atomicOr(p.status, SS_DEVICE_SINGULAR_MAP);
+        }
+    }
+    __syncthreads();
+
+    // 3. C = L^-T L^-1 Z, one column of dk per thread, then stored
+    const bool good = map_ok != 0;
+    for (int k = t; k < K; k += T) {
+        if (good) {
+            for (int e = 0; e < r; ++e) {
+                float acc = zs[e * K + k];
+                for (int f = 0; f < e; ++f) acc = fmaf(-g[e * r + f], zs[f * K + k], acc);
+                zs[e * K + k] = acc / g[e * r + e];
+            }
+            for (int e = r - 1; e >= 0; --e) {
+                float acc = zs[e * K + k];
+                for (int f = e + 1; f < r; ++f) acc = fmaf(-g[f * r + e], zs[f * K + k], acc);
+                zs[e * K + k] = acc / g[e * r + e];
+            }
+        }
+        const long long row = b * p.R + p.off[h];
+        for (int e = 0; e < r; ++e) {
+            const float c = good ? zs[e * K + k] : 0.f;
+            if (p.sketch_bf16) static_cast<uint16_t*>(p.cmap)[(row + e) * K + k] = f2bf(c);
+            else static_cast<float*>(p.cmap)[(row + e) * K + k] = c;
+        }
+    }
+}
+
+template <int FAM, int K, int V, bool MIXED, bool MAP>
 __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __grid_constant__ FlushParams p, int rpad) {
     using S = FS<K, V>;
     constexpr int R = S::R, KB = S::KB, KD = S::KD;
@@ -392,8 +543,9 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
         prepare_head<FAM, K, V>(p, h, n, r_h, rpad, sl, L, smem, tgate, tbeta, t);
         __syncthreads();                                              // (B)
 
-        // 3. The tile buffer is free: start the next head's state.
-        {
+        // 3. The tile buffer is free: start the next head's state (with the
+        //    coefficient map the buffer is scratch until the map is built).
+        if constexpr (!MAP) {
             const long long un = MIXED ? fq->next : u + gridDim.x;
             if (t == 0 && un < units) {
                 mbar_expect_tx(tbar, K * V * 4);
@@ -573,15 +725,29 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
             const int col = c0 + hb0 * 2;
             if (e < r_h) {
                 const long long row = b * p.R + p.off[h] + e;
+                float2 us = make_float2(v2[0], v2[1]);                // U as stored
                 if (p.sketch_bf16) {
+                    const uint16_t h0 = f2bf(v2[0]), h1 = f2bf(v2[1]);
                     *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.sketch) + row * V + col) =
-                        uint32_t(f2bf(v2[0])) | (uint32_t(f2bf(v2[1])) << 16);
+                        uint32_t(h0) | (uint32_t(h1) << 16);
+                    us = make_float2(bf2f(h0), bf2f(h1));
                 } else {
-                    *reinterpret_cast<float2*>(static_cast<float*>(p.sketch) + row * V + col) =
-                        make_float2(v2[0], v2[1]);
+                    *reinterpret_cast<float2*>(static_cast<float*>(p.sketch) + row * V + col) = us;
                 }
+                if (MAP) *reinterpret_cast<float2*>(reinterpret_cast<float*>(smem + L.tile) + e * V + col) = us;
             } else if (e == r_h && p.has_token) {
                 *reinterpret_cast<float2*>(p.out + u * V + col) = make_float2(v2[0], v2[1]);
+            }
+        }
+        if constexpr (MAP) {
+            if (r_h > 0) build_map<K, V>(p, st, r_h, b, h, smem, L, t);
+            __syncthreads();                                          // (E) scratch read
+            // 3'. The tile buffer is free again: start the next head's state.
+            const long long un = MIXED ? fq->next : u + gridDim.x;
+            if (t == 0 && un < units) {
+                mbar_expect_tx(tbar, K * V * 4);
+                bulk_g2s(smem + L.tile, p.state + un * (long long)(K * V), K * V * 4, tbar);
+                pending |= 1u;
             }
         }
     }
@@ -593,13 +759,14 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
     }
 }
 
-template <int FAM, int K, int V, bool MIXED>
+template <int FAM, int K, int V, bool MIXED, bool MAP>
 cudaError_t flush_launch(const FlushParams& p, int rmax, cudaStream_t stream) {
     const int n = p.n_ring + p.has_token;
     const int rpad = ((p.do_sketch ? rmax : 0) + p.has_token + 3) & ~3;
     const int bytes = flush_layout(FAM, K, V, n, rpad).total;
     if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
-    auto kern = flush_kernel<FAM, K, V, MIXED>;
+    if (MAP && !map_fits(K, V, rmax)) return cudaErrorInvalidConfiguration;
+    auto kern = flush_kernel<FAM, K, V, MIXED, MAP>;
     static KernelCache kc;
     cudaError_t e = ensure_smem(kern, kc, bytes);
     if (e != cudaSuccess) return e;
@@ -617,21 +784,29 @@ cudaError_t flush_launch(const FlushParams& p, int rmax, cudaStream_t stream) {
 // carries no unit selection.
 template <int FAM, int K, int V>
 cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
-    return p.fill_in ? flush_launch<FAM, K, V, true>(p, rmax, stream) : flush_launch<FAM, K, V, false>(p, rmax, stream);
+    if (p.cmap && p.do_sketch)
+        return p.fill_in ? flush_launch<FAM, K, V, true, true>(p, rmax, stream)
+                         : flush_launch<FAM, K, V, false, true>(p, rmax, stream);
+    return p.fill_in ? flush_launch<FAM, K, V, true, false>(p, rmax, stream)
+                     : flush_launch<FAM, K, V, false, false>(p, rmax, stream);
 }
 
 }  // namespace
 
-// Mamba-2 runs on the tensor-core kernel (ss_flush_mma.cu); GDN and KDA on
-// the CUDA-core kernel above.
+// Mamba-2 runs on the tensor-core kernel (ss_flush_mma.cu); GDN and KDA, and
+// every family when the flush also builds the state-dependent coefficient
+// map, on the CUDA-core kernel above.
 cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream) {
-    if (family == MAMBA2) return launch_flush_mma(dk, dv, p, rmax, stream);
+    if (family == MAMBA2 && !(p.cmap && p.do_sketch)) return launch_flush_mma(dk, dv, p, rmax, stream);
     SS_DISPATCH(flush_t, p, rmax, stream);
 }
 
-// rpad = rows of [Omega | q] rounded up to 4 (the CUDA-core kernel's read-out passes).
-int flush_smem_bytes(int family, int dk, int dv, int n, int rpad) {
-    if (family == MAMBA2) return flush_mma_smem_bytes(dk, dv, n, (rpad + 15) & ~15);
+bool flush_map_fits(int dk, int dv, int r) { return map_fits(dk, dv, r); }
+
+// rpad = rows of [Omega | q] rounded up to 4 (the CUDA-core kernel's read-out
+// passes); smap: the flush builds the state-dependent map (CUDA-core kernel).
+int flush_smem_bytes(int family, int dk, int dv, int n, int rpad, bool smap) {
+    if (family == MAMBA2 && !smap) return flush_mma_smem_bytes(dk, dv, n, (rpad + 15) & ~15);
     return flush_layout(family, dk, dv, n, rpad).total;
 }
 

@@ -36,6 +36,11 @@ struct FlushParams {
     // W-1 flush; each writes fill_out[b] = 0.  Null for a uniform batch.
     const int32_t* fill_in;
     int32_t* fill_out;
+    // State-dependent coefficient map (SS_COEF_STATE): when set, the flush
+    // also writes C = (U^T U + lambda I)^-1 U^T S^T, lambda = ridge tr(U^T U)/r,
+    // for every head it sketches, as [B][R][dk] in the sketch dtype.
+    void* cmap;
+    float ridge;
     int off[SS_MAX_HEADS + 1];
 };
 
@@ -67,6 +72,9 @@ struct StepParams {
     // writes fill_out[b] = fill_in[b] + 1.  Null for a uniform batch.
     const int32_t* fill_in;
     int32_t* fill_out;
+    // SS_COEF_STATE: per-unit maps [B][R][dk] in the sketch dtype, staged with
+    // each unit instead of the shared `coef` (decode only).
+    const void* cmap;
     int off[SS_MAX_HEADS + 1];
 };
 

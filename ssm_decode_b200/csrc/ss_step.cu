@@ -63,8 +63,9 @@ __device__ __forceinline__ unsigned unit_bytes(int P, int ubytes) {
 template <int FAM, int K, int V>
 __device__ __forceinline__ void stage_unit_bulk(const StepParams& p, long long unit, int P, unsigned char* sh,
                                                 const UnitSmem& L, const void* usrc, int ubytes,
-                                                uint64_t* bar, unsigned extra) {
-    mbar_expect_tx(bar, unit_bytes<FAM, K, V>(P, ubytes) + extra);
+                                                uint64_t* bar, unsigned extra, const void* csrc = nullptr,
+                                                int cbytes = 0) {
+    mbar_expect_tx(bar, unit_bytes<FAM, K, V>(P, ubytes + cbytes) + extra);
     const long long ring_row = unit * p.W;
     if (P > 0) {
         const int P4 = (P + 3) & ~3;
@@ -75,6 +76,7 @@ __device__ __forceinline__ void stage_unit_bulk(const StepParams& p, long long u
         if (FAM != MAMBA2) bulk_g2s(sh + L.bs, p.ring_beta + unit * p.Wg, P4 * 4, bar);
     }
     if (ubytes > 0) bulk_g2s(sh + L.ush, usrc, ubytes, bar);
+    if (cbytes > 0) bulk_g2s(sh + L.ush + ubytes, csrc, cbytes, bar);     // the unit's own map rows
     bulk_g2s(sh + L.tq, p.tok_q + unit * K, K * 2, bar);
     bulk_g2s(sh + L.tk, p.tok_k + unit * K, K * 2, bar);
     bulk_g2s(sh + L.tv, p.tok_v + unit * V, V * 2, bar);
@@ -544,8 +546,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
     const int g0 = blockIdx.x * wpc + warp;
     const int off = p.off[h], r = p.off[h + 1] - off;
     const int P = p.p;
-    const UnitSmem L = unit_smem(FAM, K, V, P, rmax * V * ESZ);
-    const int cbytes = align16(rmax * K * 4);
+    // With the state-dependent map each unit stages its own C rows (r x dk,
+    // sketch dtype) after its sketch rows; otherwise the CTA stages the
+    // head's shared fp32 C once.
+    const bool smap = p.cmap != nullptr;
+    const UnitSmem L = unit_smem(FAM, K, V, P, rmax * (V + (smap ? K : 0)) * ESZ);
+    const int cbytes = smap ? 0 : align16(rmax * K * 4);
     const float* csm = reinterpret_cast<const float*>(smem);
     uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + cbytes);
     unsigned char* wbase = smem + cbytes + 16 + warp * ns * stage_bytes;
@@ -564,7 +570,10 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
             if (b < p.B && Pb >= 0 && Pb < p.W - 1)
                 stage_unit_bulk<FAM, K, V>(p, (long long)b * p.H + h, Pb, wbase + s * stage_bytes + 16 + g * L.total, L,
                                            static_cast<const char*>(p.sketch) + (b * (long long)p.R + off) * (V * ESZ),
-                                           r * V * ESZ, bar(s), (stall && it == 0 && g == 0) ? 16u : 0u);
+                                           r * V * ESZ, bar(s), (stall && it == 0 && g == 0) ? 16u : 0u,
+                                           smap ? static_cast<const char*>(p.cmap) + (b * (long long)p.R + off) * (K * ESZ)
+                                                : nullptr,
+                                           smap ? r * K * ESZ : 0);
             else
                 mbar_arrive(bar(s));
         }
@@ -576,8 +585,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
     fence_mbar_init();
     __syncthreads();                                        // the only block barrier
     if (threadIdx.x == 0) {
-        mbar_expect_tx(cbar, r * K * 4);
-        if (r > 0) bulk_g2s(smem, p.coef + (long long)off * K, r * K * 4, cbar);
+        mbar_expect_tx(cbar, smap ? 0 : r * K * 4);
+        if (!smap && r > 0) bulk_g2s(smem, p.coef + (long long)off * K, r * K * 4, cbar);
     }
     if (g0 >= ngroups) return;                              // warp 0 always has a group
     for (int it = 0; it < ns; ++it) issue(it);              // before C arrives: the two latencies overlap
@@ -837,13 +846,18 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         // 3. Coefficients c = C q~ and the sketched read o = U c + term,
         //    4 rows of C at a time.
         const unsigned char* us = sh + L.ush;
+        const unsigned char* cmu = us + r * V * ESZ;          // this unit's map rows (smap)
+        auto crow = [&](int i, float (&ci)[EK]) {
+            if (smap) row_any<K, G, UB16>(cmu + i * K * ESZ, l, ci);
+            else row_f32<K, G>(csm + i * K, l, ci);
+        };
         int i = 0;
         for (; i + 4 <= r; i += 4) {
             float c[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 float ci[EK];
-                row_f32<K, G>(csm + (i + q) * K, l, ci);
+                crow(i + q, ci);
                 c[q] = dot<EK>(ci, x);
             }
 #pragma unroll
@@ -857,7 +871,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         }
         for (; i < r; ++i) {
             float ci[EK], ui[EV];
-            row_f32<K, G>(csm + i * K, l, ci);
+            crow(i, ci);
             const float c = gsum<G>(dot<EK>(ci, x));
             row_any<V, G, UB16>(us + i * V * ESZ, l, ui);
             axpy<EV>(c, ui, ob);
@@ -965,15 +979,21 @@ __global__ void __launch_bounds__(128) replay_kernel(const __grid_constant__ Ste
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-int decode_stage(int fam, int K, int V, int P, int rmax, int esz) {
-    return dec_stage_bytes(fam, K, V, P, rmax * V * esz);
+// One warp's staging buffer; with the state-dependent map (`smap`) each unit
+// also stages its own map rows.
+int decode_stage(int fam, int K, int V, int P, int rmax, int esz, bool smap) {
+    return dec_stage_bytes(fam, K, V, P, rmax * (V + (smap ? K : 0)) * esz);
 }
+
+// The CTA-wide part: the head's shared C (fixed map only) and its mbarrier.
+int decode_cpart(int K, int rmax, bool smap) { return (smap ? 0 : align16(rmax * K * 4)) + 16; }
 
 template <int FAM, int K, int V, bool UB16, bool MIXED>
 cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
     constexpr int esz = UB16 ? 2 : 4, upw = 32 / dec_gl(FAM);
-    const int stage = decode_stage(FAM, K, V, p.p, rmax, esz);
-    const int cpart = align16(rmax * K * 4) + 16;
+    const bool smap = p.cmap != nullptr;
+    const int stage = decode_stage(FAM, K, V, p.p, rmax, esz, smap);
+    const int cpart = decode_cpart(K, rmax, smap);
     if (cpart + stage > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
     int wpc = DEC_WARPS;
     while (wpc > 1 && cpart + wpc * stage > SMEM_LIMIT) --wpc;
@@ -1023,8 +1043,8 @@ cudaError_t launch_replay(int family, int dk, int dv, const StepParams& p, cudaS
     SS_DISPATCH(replay_t, p, stream);
 }
 
-int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz) {
-    return align16(rmax * dk * 4) + 16 + decode_stage(family, dk, dv, P, rmax, esz);
+int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz, bool smap) {
+    return decode_cpart(dk, rmax, smap) + decode_stage(family, dk, dv, P, rmax, esz, smap);
 }
 
 }  // namespace ss

@@ -36,9 +36,9 @@ class DecodeLayer:
     """Plan plus caller-owned device buffers for one linear-attention layer."""
 
     def __init__(self, family, batch, heads, dk, dv, window, ranks, sketch_dtype=B.SS_F32,
-                 device="cuda"):
+                 device="cuda", coef_mode=B.SS_COEF_FIXED, coef_ridge=0.0):
         import torch
-        self.plan = B.Plan(family, batch, heads, dk, dv, window, ranks, sketch_dtype)
+        self.plan = B.Plan(family, batch, heads, dk, dv, window, ranks, sketch_dtype, coef_mode, coef_ridge)
         self.family, self.batch, self.heads, self.dk, self.dv, self.window = family, batch, heads, dk, dv, window
         self.device = device
         sz = B.ss_buffer_sizes(self.plan)
@@ -55,6 +55,9 @@ class DecodeLayer:
         self.sketch = torch.zeros((batch, max(self.R, 1), dv), dtype=sk_dtype, device=device)
         self.basis = z(max(self.R, 1), dk)
         self.coef = z(max(self.R, 1), dk)
+        # per-(sequence, head) coefficient maps of SS_COEF_STATE, sketch dtype
+        self.coef_state = (torch.zeros((batch, max(self.R, 1), dk), dtype=sk_dtype, device=device)
+                           if coef_mode == B.SS_COEF_STATE else None)
         self.A = z(heads)
         self.out = z(batch, heads, dv)
         self.status = torch.zeros(4, dtype=torch.int32, device=device)   # device status word (+ padding)
@@ -88,7 +91,7 @@ class DecodeLayer:
     def _make_bufs(self, with_sketch):
         return B.make_buffers(self.state, self.ring_k, self.ring_v, self.ring_gate, self.ring_beta,
                               self.sketch if with_sketch else None, self.basis, self.coef, self.A,
-                              self.status)
+                              self.status, self.coef_state)
 
     def io(self, tok, out=None):
         cache = getattr(tok, "_io", None) if out is None else None

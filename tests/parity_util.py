@@ -59,21 +59,24 @@ class Pair:
     compare sampled sequences); the GPU always runs the whole batch.
     """
 
-    def __init__(self, wl, st=None, sketch_dtype=B.SS_F32, sel=None):
+    def __init__(self, wl, st=None, sketch_dtype=B.SS_F32, sel=None, state_map=False, rho=0.0):
         import torch
         self.wl = wl
         self.st = st if st is not None else synth.static_inputs(wl)
         self.sel = np.arange(wl.batch) if sel is None else np.asarray(sel)
+        self.state_map = state_map
         self.layer = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, wl.window,
-                                 self.st.ranks, sketch_dtype)
+                                 self.st.ranks, sketch_dtype,
+                                 coef_mode=B.SS_COEF_STATE if state_map else B.SS_COEF_FIXED,
+                                 coef_ridge=rho)
         self.layer.load(self.st.state, self.st.basis, self.st.coef, self.st.A)
         self.sess = orc.Session(wl.family, self.st.state[self.sel], wl.window, self.st.A,
                                 self.st.basis, self.st.coef, self.st.offsets,
-                                sketch_bf16=sketch_dtype == B.SS_BF16)
+                                sketch_bf16=sketch_dtype == B.SS_BF16, state_map=state_map, rho=rho)
         self.bf16 = sketch_dtype == B.SS_BF16
         self.ring_k = np.zeros((wl.batch, wl.heads, wl.window, wl.dk), np.uint16)
         self.ring_v = np.zeros((wl.batch, wl.heads, wl.window, wl.dv), np.uint16)
-        self.worst = {"out": 0.0, "sketched": 0.0, "state": 0.0, "sketch": 0.0}
+        self.worst = {"out": 0.0, "sketched": 0.0, "state": 0.0, "sketch": 0.0, "map": 0.0}
         torch.cuda.synchronize()
 
     # -- checks ------------------------------------------------------------------
@@ -103,6 +106,43 @@ class Pair:
                 self.worst["sketch"] = max(self.worst["sketch"], err)
                 assert err <= TOL, f"sketch head {h} relerr {err:.3e}"
 
+    def gpu_sketch_heads(self):
+        """The GPU's stored sketch per head, widened: list of [b, V, r_h]."""
+        u = to_np(self.layer.sketch)[self.sel]
+        offs = self.st.offsets
+        return [np.transpose(u[:, offs[h]:offs[h + 1]], (0, 2, 1)) for h in range(self.wl.heads)]
+
+    def check_map(self):
+        """State-dependent maps: per head, max|gpu - oracle| / max|oracle| within
+        1e-4 (fp32).  With a bf16 sketch the map is a function of the stored U,
+        whose entries may sit one bf16 ulp from the oracle's rounding (fp32 vs
+        fp64 straddling a tie), and the solve amplifies that; so the reference
+        map is the oracle's map of the GPU's own stored U (reading P7), rounded
+        to bf16, and each entry must lie within one bf16 ulp of it plus 1e-4
+        of the head's largest entry."""
+        if not self.state_map:
+            return
+        g = to_np(self.layer.coef_state)[self.sel]
+        if self.bf16:
+            Ug = self.gpu_sketch_heads()
+            ref = np.concatenate([orc.round_bf16(orc.coefficient_map(Ug[h], self.sess.S[:, h], self.sess.rho))
+                                  for h in range(self.wl.heads)], axis=1)
+        else:
+            ref = self.sess.packed_map()
+        offs = self.st.offsets
+        for h in range(self.wl.heads):
+            if offs[h + 1] == offs[h]:
+                continue
+            gh, rh = g[:, offs[h]:offs[h + 1]], ref[:, offs[h]:offs[h + 1]]
+            if self.bf16:
+                allow = bf16_ulp(rh) + TOL * np.abs(rh).max(axis=(1, 2), keepdims=True)
+                ok = np.abs(gh - rh) <= allow * (1 + 1e-9)
+                assert ok.all(), f"map head {h}: {(~ok).sum()} entries beyond one bf16 ulp + allowance"
+            else:
+                err = head_relerr(gh, rh)
+                self.worst["map"] = max(self.worst["map"], err)
+                assert err <= TOL, f"map head {h} relerr {err:.3e}"
+
     def check_ring(self):
         ph = self.layer.phase
         gk = to_np(self.layer.ring_k)
@@ -127,6 +167,7 @@ class Pair:
         self.layer.prime()
         self.sess.prime()
         self.check_sketch()
+        self.check_map()
 
     def _sub(self, inp):
         return {k: v[self.sel] for k, v in inp.items()}
@@ -148,9 +189,22 @@ class Pair:
             assert err <= TOL, f"flush output relerr {err:.3e}"
             self.check_state()
             self.check_sketch()
+            self.check_map()
         else:
             o_hat, _ = self.sess.decode(self._sub(inp))
-            if self.bf16:
+            if self.bf16 and self.state_map:
+                # the GPU's stored bf16 U and map applied to the oracle's q~ and buffered term
+                Cg = to_np(self.layer.coef_state)[self.sel]
+                Ug = self.gpu_sketch_heads()
+                offs = self.st.offsets
+                ref = np.empty_like(o_hat)
+                for h in range(self.wl.heads):
+                    c = np.einsum("brk,bk->br", Cg[:, offs[h]:offs[h + 1]], self.sess.last_q_tilde[:, h])
+                    ref[:, h] = np.einsum("bvr,br->bv", Ug[h], c) + self.sess.last_o_buf[:, h]
+                err = vec_relerr(g, ref)
+                self.worst["sketched"] = max(self.worst["sketched"], err)
+                assert err <= TOL, f"sketched output (stored bf16 U and map) relerr {err:.3e} at phase {ph}"
+            elif self.bf16:
                 ref_u = self.sess.packed_sketch()
                 allow_u = self._sketch_allowance(ref_u)
                 bound = np.broadcast_to(TOL * np.abs(o_hat).max(-1, keepdims=True), o_hat.shape).copy()

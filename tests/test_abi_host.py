@@ -148,6 +148,51 @@ def test_schedule_and_argument_errors(L):
     assert B.ss_launch_count() == 0
 
 
+def test_state_map_config_sizes_and_traffic(L):
+    """SS_COEF_STATE: the per-sequence map buffer, its validation and its bytes."""
+    p = B.Plan(B.SS_GDN, 3, 2, 128, 64, 6, [5, 7], B.SS_BF16, B.SS_COEF_STATE, 0.25)
+    s = B.ss_buffer_sizes(p)
+    assert s["coef_state"] == 3 * 12 * 128 * 2
+    assert B.ss_buffer_sizes(B.Plan(B.SS_GDN, 3, 2, 128, 64, 6, [5, 7], B.SS_BF16))["coef_state"] == 0
+    fixed = B.Plan(B.SS_GDN, 3, 2, 128, 64, 6, [5, 7], B.SS_BF16)
+    d_s, d_f = B.ss_traffic_bytes(p, B.SS_OP_DECODE, 2), B.ss_traffic_bytes(fixed, B.SS_OP_DECODE, 2)
+    # per-sequence maps replace the shared fp32 map read once per head
+    assert d_s["read_bytes"] - d_f["read_bytes"] == 3 * 12 * 128 * 2 - 12 * 128 * 4
+    f_s, f_f = B.ss_traffic_bytes(p, B.SS_OP_FLUSH), B.ss_traffic_bytes(fixed, B.SS_OP_FLUSH)
+    assert f_s["write_bytes"] - f_f["write_bytes"] == 3 * 12 * 128 * 2
+    assert f_s["paper_read_bytes"] == f_f["paper_read_bytes"]
+    for mode, ridge in ((7, 0.0), (B.SS_COEF_STATE, -1.0), (B.SS_COEF_STATE, float("nan")),
+                        (B.SS_COEF_STATE, float("inf"))):
+        with pytest.raises(B.SSError) as e:
+            B.Plan(B.SS_GDN, 1, 1, 64, 64, 4, [4], B.SS_F32, mode, ridge)
+        assert e.value.status == B.SS_ERR_INVALID_ARG
+    # the map needs U, per-warp partial sums and U^T U in the flush's tile buffer
+    with pytest.raises(B.SSError) as e:
+        B.Plan(B.SS_KDA, 1, 1, 64, 64, 4, [64], B.SS_F32, B.SS_COEF_STATE)
+    assert e.value.status == B.SS_ERR_UNSUPPORTED
+    for K, V in ((64, 64), (64, 128), (128, 64), (128, 128)):
+        B.Plan(B.SS_MAMBA2, 1, 1, K, V, 16, [min(K, V) // 2], B.SS_BF16, B.SS_COEF_STATE)
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="fake-pointer validation tests run on CPU hosts only")
+def test_state_map_needs_its_buffer(L):
+    p = B.Plan(B.SS_KDA, 2, 2, 64, 64, 4, [2, 3], B.SS_F32, B.SS_COEF_STATE, 0.0)
+    st = ctypes.c_void_p(0)
+    io = _fake_io()
+    B.ss_set_phase(p, 1, True)
+    b = _fake_bufs(null="coef_state")
+    assert L.ss_decode_step(p.handle, ctypes.byref(b), ctypes.byref(io), st) == B.SS_ERR_INVALID_ARG
+    assert "coef_state" in B.ss_last_error_string()
+    b = _fake_bufs(bad="coef_state")
+    assert L.ss_decode_step(p.handle, ctypes.byref(b), ctypes.byref(io), st) == B.SS_ERR_ALIGNMENT
+    B.ss_set_phase(p, 0, False)
+    assert L.ss_prime(p.handle, ctypes.byref(_fake_bufs(null="coef_state")), st) == B.SS_ERR_INVALID_ARG
+    B.ss_set_phase(p, 3, True)
+    assert L.ss_flush(p.handle, ctypes.byref(_fake_bufs(null="coef_state")), ctypes.byref(io), st) == \
+        B.SS_ERR_INVALID_ARG
+    assert B.ss_launch_count() == 0
+
+
 def _ratio(family, dk, dv, rank, W, heads=4, batch=3):
     p = B.Plan(family, batch, heads, dk, dv, W, [rank] * heads, B.SS_BF16)
     ex = B.ss_traffic_bytes(p, B.SS_OP_EXACT)

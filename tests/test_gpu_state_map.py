@@ -1,0 +1,165 @@
+"""GPU parity of the state-dependent coefficient map (SS_COEF_STATE).
+
+Every flush (and ss_prime) also builds, per (sequence, head), the map
+C = (U^T U + lambda I)^-1 U^T S^T from the new state and sketch (project page,
+"Per window · Flush: Sketch & coefficient map"; paper §A.2.1), and every
+non-flush step reads c = C q~ with that map.  The fp64 oracle session does the
+same with numpy's solve; maps, sketched outputs, states and sketches are
+compared after every step (tolerances in tests/parity_util.py).
+
+Conditioning: after a window of decaying updates the state is dominated by
+its last few updates, so U^T U is badly conditioned (median condition number
+~1e7 on these inputs after one flush, against ~2.4 before any update).  The
+map's fp32 accuracy is bounded through cond(U^T U + lambda I) <= 1 + r/rho,
+so the tests that cross a flush use rho = 0.1 (<= 161 at r = 16), where fp32
+meets the 1e-4 bar against fp64; rho = 0 is tested where it is well posed
+(ss_prime's map and the first window's reads).
+"""
+import numpy as np
+import pytest
+
+from oracle import sketchssm_oracle as orc
+from ssm_decode_b200 import binding as B
+from ssm_decode_b200 import synth
+from ssm_decode_b200.layer import DecodeLayer
+from tests.parity_util import TOL, Pair, head_relerr, to_np, vec_relerr
+from tests.test_gpu_mixed import _one, _put_ring
+
+pytestmark = pytest.mark.gpu
+
+FAM = {"mamba2": synth.MAMBA2, "gdn": synth.GDN, "kda": synth.KDA}
+RHO = 0.1
+
+
+def small(family, dk=128, dv=128, batch=3, heads=5, window=16, mean_rank=8, seed=77):
+    return synth.Workload(f"map_{family}", family, batch, heads, dk, dv, window, 0, mean_rank, seed)
+
+
+def run(pair, steps):
+    pair.prime()
+    for t in range(steps):
+        pair.step(synth.step_inputs(pair.wl, pair.st, t))
+    return pair.worst
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (128, 64), (64, 128), (64, 64)])
+def test_state_map_families_and_shapes(cuda_ok, family, dk, dv):
+    wl = small(FAM[family], dk, dv, seed=1500 + dk + dv)
+    w = run(Pair(wl, state_map=True, rho=RHO), 20)
+    assert w["map"] <= TOL and w["sketched"] <= TOL
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+@pytest.mark.parametrize("sketch_dtype", [B.SS_F32, B.SS_BF16])
+def test_state_map_unregularized_first_window(cuda_ok, family, sketch_dtype):
+    """rho = 0 (the pseudoinverse form): ss_prime's map and every read of the
+    first window, before a flush makes U^T U ill-conditioned."""
+    wl = small(FAM[family], 128, 128, seed=1550)
+    run(Pair(wl, sketch_dtype=sketch_dtype, state_map=True, rho=0.0), wl.window - 1)
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+def test_state_map_bf16(cuda_ok, family):
+    wl = small(FAM[family], 128, 64, seed=1600)
+    run(Pair(wl, sketch_dtype=B.SS_BF16, state_map=True, rho=RHO), 20)
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+def test_state_map_ridge(cuda_ok, family):
+    wl = small(FAM[family], 128, 128, seed=1700)
+    run(Pair(wl, state_map=True, rho=0.5), 18)
+
+
+@pytest.mark.parametrize("window", [1, 3, 32])
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+def test_state_map_windows(cuda_ok, family, window):
+    wl = small(FAM[family], 128, 64, batch=2, heads=3, window=window, seed=1800 + window)
+    run(Pair(wl, state_map=True, rho=RHO), 2 * window + 3)
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+def test_state_map_ragged_ranks_with_zero_and_one(cuda_ok, family):
+    wl = small(FAM[family], 128, 64, heads=4, seed=1900)
+    st = synth.static_inputs(wl)
+    ranks = np.array([0, 1, 16, 7], np.int32)
+    offs = np.concatenate([[0], np.cumsum(ranks)]).astype(np.int32)
+    rng = np.random.default_rng(19)
+    basis = np.concatenate([np.linalg.qr(rng.standard_normal((wl.dk, wl.dk)))[0][:, :r].T
+                            for r in ranks]).astype(np.float32)
+    st.ranks, st.offsets, st.basis, st.coef = ranks, offs, basis, basis.copy()
+    run(Pair(wl, st=st, state_map=True, rho=RHO), 18)
+
+
+def test_state_map_of_zero_state_is_singular(cuda_ok):
+    """An all-zero state has U = 0: no positive-definite Gram matrix.  The
+    flush flags SS_DEVICE_SINGULAR_MAP and stores a zero map (as the oracle
+    does), so the next reads return the exact buffered term alone."""
+    wl = small(synth.GDN, 128, 64, batch=2, heads=3, window=4, seed=2000)
+    st = synth.static_inputs(wl)
+    st.state = np.zeros_like(st.state)
+    p = Pair(wl, st=st, state_map=True)
+    p.prime()
+    assert int(p.layer.status[0].item()) & B.SS_DEVICE_SINGULAR_MAP
+    assert not to_np(p.layer.coef_state).any()
+    for t in range(2):
+        p.step(synth.step_inputs(wl, st, t))
+    p.layer.status.zero_()
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn"])
+def test_state_map_full_size_sampled(cuda_ok, family):
+    """The full workload (Mamba-2 batch 320 x 128 heads, or GDN 256 x 32) in
+    state-map mode for one window plus a flush, outputs and maps compared on
+    three sampled sequences."""
+    wl = synth.WORKLOADS["mamba2_b320" if family == "mamba2" else "gdn_b256"]
+    p = Pair(wl, sketch_dtype=B.SS_BF16, sel=[0, wl.batch // 2, wl.batch - 1], state_map=True, rho=RHO)
+    run(p, wl.window + 1)
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+def test_state_map_mixed_positions(cuda_ok, family):
+    """ss_step_mixed with the state map: sequences at their own positions,
+    each checked against its own oracle session (map included)."""
+    import torch
+    W, batch = 5, 7
+    wl = synth.Workload(f"mixmap_{family}", FAM[family], batch, 3, 128, 64, W, 0, 8, 2100)
+    st = synth.static_inputs(wl)
+    layer = DecodeLayer(wl.family, batch, 3, 128, 64, W, st.ranks, coef_mode=B.SS_COEF_STATE, coef_ridge=RHO)
+    layer.load(st.state, st.basis, st.coef, st.A)
+    sess = [orc.Session(wl.family, st.state[b:b + 1], W, st.A, st.basis, st.coef, st.offsets, state_map=True,
+                        rho=RHO) for b in range(batch)]
+    layer.prime()
+    for s in sess:
+        s.prime()
+    fills = (np.arange(batch) % W).astype(np.int32)
+    for j in range(W - 1):
+        inp = synth.step_inputs(wl, st, 700 + j)
+        for b in range(batch):
+            if j < fills[b]:
+                _put_ring(layer, inp, b, j)
+                sess[b].decode(_one(inp, b))
+    fin = torch.from_numpy(fills).cuda()
+    fout = torch.empty_like(fin)
+    fill = fills.copy()
+    for t in range(W + 2):
+        inp = synth.step_inputs(wl, st, t)
+        layer.step_mixed(layer.token(inp), fin, fout)
+        torch.cuda.synchronize()
+        g = to_np(layer.out)
+        cm = to_np(layer.coef_state)
+        for b, s in enumerate(sess):
+            if fill[b] == W - 1:
+                o = s.flush(_one(inp, b))
+                assert vec_relerr(g[b:b + 1], o) <= TOL
+                ref = s.packed_map()
+                for h in range(3):
+                    lo, hi = st.offsets[h], st.offsets[h + 1]
+                    if hi > lo:
+                        assert head_relerr(cm[b:b + 1, lo:hi], ref[:, lo:hi]) <= TOL
+            else:
+                o_hat, _ = s.decode(_one(inp, b))
+                assert vec_relerr(g[b:b + 1], o_hat) <= TOL, f"seq {b} fill {fill[b]}"
+        fill = (fill + 1) % W
+        fin, fout = fout, fin
+    assert int(layer.status[0].item()) == 0

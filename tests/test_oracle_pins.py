@@ -393,6 +393,14 @@ def test_state_map_never_worse_than_fixed_map():
     assert (e_state <= e_fixed * (1 + 1e-12)).all() and (e_state < e_fixed).any()
 
 
+def test_coefficient_map_of_zero_state_is_zero():
+    """No positive-definite Gram matrix (U = 0): the map is zero, so the
+    sketched read returns only the exact buffered term."""
+    S = np.zeros((2, 8, 6))
+    P = np.eye(8)[:, :3]
+    assert not orc.coefficient_map(orc.sketch(S, P), S, 0.5).any()
+
+
 @pytest.mark.parametrize("family", FAMS)
 def test_session_state_map_identity_basis_reads_exactly(family):
     """Session with the state map and P = I (r = K <= V): every sketched read
