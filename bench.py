@@ -150,15 +150,18 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def kernel_traffic_record(name):
-    """ncu-measured DRAM bytes per launch, if taken on the current kernel source."""
+def kernel_traffic_record(name, workload, coef="fixed"):
+    """ncu-measured DRAM bytes per launch, if taken on the current kernel source
+    for this workload (the records are of the fixed-map mode)."""
+    if coef != "fixed":
+        return None
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
         sha = kernel_source_sha()
         r = rec.get(name)
-        if r and r.get("source_sha") == sha:
+        if r and r.get("source_sha") == sha and r.get("workload") == workload:
             return r
     except (OSError, ValueError):
         pass
@@ -217,11 +220,13 @@ def run_ours(args, rank, world):
     if args.batch:
         wl = dataclasses.replace(wl, name=f"{wl.name}@batch{args.batch}", batch=args.batch)
     skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
+    smap = args.coef == "state"
     W, NL = wl.window, args.layers
     st = synth.static_inputs(wl)
     layers = []
     for _ in range(NL):
-        lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev)
+        lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev,
+                          coef_mode=B.SS_COEF_STATE if smap else B.SS_COEF_FIXED, coef_ridge=args.ridge)
         lay.load(st.state, st.basis, st.coef, st.A)
         layers.append(lay)
     st.state = None
@@ -296,13 +301,14 @@ def run_ours(args, rank, world):
     fl_b = fl["read_bytes"] + fl["write_bytes"]
     kernel_ms = dec_ms + fl_ms
     kernels = {}
-    flush_name = "flush_mma_kernel" if wl.family == synth.MAMBA2 else "flush_kernel"
+    # Mamba-2's flush runs on the tensor cores unless it also builds the state-dependent map
+    flush_name = "flush_mma_kernel" if wl.family == synth.MAMBA2 and not smap else "flush_kernel"
     for name, ms, count, nbytes in (("decode_kernel", dec_ms, n_dec, dec_b), (flush_name, fl_ms, n_fl, fl_b)):
         if not count:
             continue
         avg_s = ms / count / 1e3
         ach = nbytes / avg_s / 1e9
-        rec = kernel_traffic_record(name)
+        rec = kernel_traffic_record(name, wl.name, args.coef)
         kernels[name] = {"launches": count, "avg_us": avg_s * 1e6, "bytes_per_launch": nbytes,
                          "achieved_gbs": ach, "frac": ach / peak, "share": ms / kernel_ms,
                          "traffic": rec["dram_bytes_per_launch"] if rec else None,
@@ -372,6 +378,7 @@ def run_ours(args, rank, world):
         "config": {"workload": wl.name, "family": synth.FAMILY_NAMES[wl.family], "batch": wl.batch,
                    "heads": wl.heads, "dk": wl.dk, "dv": wl.dv, "window": W, "mean_rank": wl.mean_rank,
                    "layers": NL, "sketch": args.sketch_dtype, "inputs": "bf16 q/k/v, fp32 state",
+                   "coef": (f"state-dependent map, rho = {args.ridge}" if smap else "fixed C = P^T"),
                    "step": f"one window of {W} tokens through {NL} independent layers",
                    "l2": f"inputs larger than L2: {NL} layers rotated, back-to-back launches",
                    "parallelism": f"replicas x{world}"},
@@ -549,6 +556,10 @@ def main():
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--coef", default="fixed", choices=["fixed", "state"],
+                    help="coefficient map: the fixed C = P^T of the workloads, or the state-dependent "
+                         "least-squares map rebuilt by every flush")
+    ap.add_argument("--ridge", type=float, default=0.01, help="rho of the state-dependent map")
     ap.add_argument("--sweep", action="store_true",
                     help="the batch x window x rank sweep on the Mamba-2 shape (1 GPU), instead of the bench line")
     ap.add_argument("--sweep-batches", default="1,32,128,320,1024")

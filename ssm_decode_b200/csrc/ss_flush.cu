@@ -303,10 +303,12 @@ __device__ __forceinline__ void prepare_head(const FlushParams& p, int h, int n,
 }
 
 // Whether the coefficient map of a rank-r head fits the flush's scratch: the
-// tile buffer (dk x dv floats) holds U (r x dv), then per-warp partial sums of
-// at least one map row (dv/16 warps x dk) and later the Gram matrix (r x r).
+// tile buffer (dk x dv floats) holds U (r rows of dv + 4 floats; the pad puts
+// consecutive rows on different banks), then per-warp partial sums of at least
+// one map row (dv/16 warps x dk) and later the Gram matrix (r x r).
+__host__ __device__ constexpr int umap_stride(int V) { return V + 4; }
 __host__ __device__ inline bool map_fits(int K, int V, int r) {
-    const int free_floats = K * V - r * V;
+    const int free_floats = K * V - r * umap_stride(V);
     return r <= V && free_floats >= (V / 16) * K && free_floats >= r * r;
 }
 
@@ -320,11 +322,12 @@ __host__ __device__ inline bool map_fits(int K, int V, int r) {
 //      reduce-scatter over the 4 column lanes leaves R/4 rows per lane, and
 //      the dv/16 warps' partials are summed through shared memory, EC rows
 //      of Z at a time.  Z lands in the extended-basis buffer (free now).
-//   2. G = U^T U (lower triangle) in the tile buffer; warp 0 factors
-//      G + lambda I = L L^T (Cholesky, column by column).
-//   3. Thread k solves L L^T c = Z[:, k] for column k in place; the columns
-//      are C's, written in the sketch dtype.  A pivot that is not positive
-//      and finite zeroes the head's map and sets SS_DEVICE_SINGULAR_MAP.
+//   2. M = U^T U + lambda I in the tile buffer; warp 0 inverts it in place
+//      (Gauss-Jordan, one column per lane: the row updates of a step are
+//      independent, unlike the dependent chains of a Cholesky solve).
+//   3. Thread k forms column k of C = M^-1 Z with independent accumulators
+//      and stores it in the sketch dtype.  A pivot that is not positive and
+//      finite zeroes the head's map and sets SS_DEVICE_SINGULAR_MAP.
 template <int K, int V>
 __device__ __forceinline__ void build_map(const FlushParams& p, const float2 (&st)[K / 8][2], int r,
                                           long long b, int h, unsigned char* smem, const FlushLayout& L,
@@ -335,40 +338,53 @@ __device__ __forceinline__ void build_map(const FlushParams& p, const float2 (&s
     const int cgw = lane & 3, rb = lane >> 2;
     const int c0 = warp * 16 + cgw * 4, row0 = rb * R;
     const int b0 = cgw & 1, b1 = (cgw >> 1) & 1;
-    float* umap = reinterpret_cast<float*>(smem + L.tile);     // [r][V]
-    float* zp = umap + r * V;                                  // [EC][NW][K], then G [r][r]
+    constexpr int US = umap_stride(V);
+    float* umap = reinterpret_cast<float*>(smem + L.tile);     // [r][US]
+    float* zp = umap + r * US;                                 // [EC][NW][K], then G [r][r]
     float* zs = reinterpret_cast<float*>(smem + L.pt);         // [r][K]: Z, then C
     __shared__ int map_ok;
-    const int EC = min(r, (K * V - r * V) / (NW * K));
+    const int EC = min(r, (K * V - r * US) / (NW * K));
     __syncthreads();                                           // (D) U written, basis rows read
 
     // 1. Z = U^T S^T
     for (int e0 = 0; e0 < r; e0 += EC) {
         const int ne = min(EC, r - e0);
-        for (int el = 0; el < ne; ++el) {
-            const float4 uu = *reinterpret_cast<const float4*>(umap + (e0 + el) * V + c0);
-            float z[R];
+        for (int el0 = 0; el0 < ne; el0 += 2) {              // two map rows per pass
+            float z[2][R];
 #pragma unroll
-            for (int i = 0; i < R; ++i) {
-                float2 pp = fmul2(st[i][0], make_float2(uu.x, uu.y));
-                pp = ffma2(st[i][1], make_float2(uu.z, uu.w), pp);
-                z[i] = pp.x + pp.y;
+            for (int d = 0; d < 2; ++d) {
+                const int el = min(el0 + d, ne - 1);
+                const float4 uu = *reinterpret_cast<const float4*>(umap + (e0 + el) * US + c0);
+#pragma unroll
+                for (int i = 0; i < R; ++i) {
+                    float2 pp = fmul2(st[i][0], make_float2(uu.x, uu.y));
+                    pp = ffma2(st[i][1], make_float2(uu.z, uu.w), pp);
+                    z[d][i] = pp.x + pp.y;
+                }
             }
-            float z2[R / 2];                                   // lane bit 0: which half of the rows
+            float z2[2][R / 2];                                // lane bit 0: which half of the rows
 #pragma unroll
-            for (int i = 0; i < R / 2; ++i) {
-                const float keep = b0 ? z[i + R / 2] : z[i], send = b0 ? z[i] : z[i + R / 2];
-                z2[i] = keep + __shfl_xor_sync(FULL, send, 1);
+            for (int d = 0; d < 2; ++d)
+#pragma unroll
+                for (int i = 0; i < R / 2; ++i) {
+                    const float keep = b0 ? z[d][i + R / 2] : z[d][i], send = b0 ? z[d][i] : z[d][i + R / 2];
+                    z2[d][i] = keep + __shfl_xor_sync(FULL, send, 1);
+                }
+            float z4[2][R / 4];                                // lane bit 1: which quarter
+#pragma unroll
+            for (int d = 0; d < 2; ++d)
+#pragma unroll
+                for (int i = 0; i < R / 4; ++i) {
+                    const float keep = b1 ? z2[d][i + R / 4] : z2[d][i], send = b1 ? z2[d][i] : z2[d][i + R / 4];
+                    z4[d][i] = keep + __shfl_xor_sync(FULL, send, 2);
+                }
+#pragma unroll
+            for (int d = 0; d < 2; ++d) {
+                if (el0 + d >= ne) break;
+                float* dst = zp + ((el0 + d) * NW + warp) * K + row0 + b0 * (R / 2) + b1 * (R / 4);
+#pragma unroll
+                for (int i = 0; i < R / 4; ++i) dst[i] = z4[d][i];
             }
-            float z4[R / 4];                                   // lane bit 1: which quarter
-#pragma unroll
-            for (int i = 0; i < R / 4; ++i) {
-                const float keep = b1 ? z2[i + R / 4] : z2[i], send = b1 ? z2[i] : z2[i + R / 4];
-                z4[i] = keep + __shfl_xor_sync(FULL, send, 2);
-            }
-            float* dst = zp + (el * NW + warp) * K + row0 + b0 * (R / 2) + b1 * (R / 4);
-#pragma unroll
-            for (int i = 0; i < R / 4; ++i) dst[i] = z4[i];
         }
         __syncthreads();
         for (int idx = t; idx < ne * K; idx += T) {
@@ -381,45 +397,68 @@ __device__ __forceinline__ void build_map(const FlushParams& p, const float2 (&s
         __syncthreads();
     }
 
-    // 2. G = U^T U (lower triangle), then G + lambda I = L L^T in place
+    // 2. M = U^T U + lambda I, inverted in place by warp 0
     float* g = zp;
     for (int idx = t; idx < r * r; idx += T) {
         const int e = idx / r, f = idx - e * r;
         if (f > e) continue;
-        const float* ue = umap + e * V;
-        const float* uf = umap + f * V;
-        float sum = 0.f;
+        const float* ue = umap + e * US;
+        const float* uf = umap + f * US;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;       // four independent chains
+#pragma unroll 4
         for (int v = 0; v < V; v += 4) {
             const float4 a = *reinterpret_cast<const float4*>(ue + v);
             const float4 c = *reinterpret_cast<const float4*>(uf + v);
-            sum = fmaf(a.x, c.x, sum);
-            sum = fmaf(a.y, c.y, sum);
-            sum = fmaf(a.z, c.z, sum);
-            sum = fmaf(a.w, c.w, sum);
+            s0 = fmaf(a.x, c.x, s0);
+            s1 = fmaf(a.y, c.y, s1);
+            s2 = fmaf(a.z, c.z, s2);
+            s3 = fmaf(a.w, c.w, s3);
         }
+        const float sum = (s0 + s1) + (s2 + s3);
         g[e * r + f] = sum;
+        g[f * r + e] = sum;
     }
     __syncthreads();
     if (warp == 0) {
         float tr = 0.f;
         for (int e = lane; e < r; e += 32) tr += g[e * r + e];
         const float lam = p.ridge * warp_sum(tr) / float(r);
+        __syncwarp();
+        for (int e = lane; e < r; e += 32) g[e * r + e] += lam;
+        __syncwarp();
+        // Gauss-Jordan without pivoting (M is symmetric positive definite, so
+        // every pivot is a positive Schur complement); lane c owns column c.
         bool good = true;
-        for (int j = 0; j < r && good; ++j) {
-            float part = 0.f;
-            for (int k = lane; k < j; k += 32) part = fmaf(g[j * r + k], g[j * r + k], part);
-            const float piv = g[j * r + j] + lam - warp_sum(part);
+        for (int j = 0; j < r; ++j) {
+            const float piv = g[j * r + j];
             good = piv > 0.f && piv < INFINITY;                // the same value in every lane
             if (!good) break;
-            const float d = sqrtf(piv);
+            const float pinv = 1.f / piv;
             __syncwarp();
-            for (int i = j + 1 + lane; i < r; i += 32) {
-                float acc = g[i * r + j];
-                for (int k = 0; k < j; ++k) acc = fmaf(-g[i * r + k], g[j * r + k], acc);
-                g[i * r + j] = acc / d;
+            for (int c = lane; c < r; c += 32)
+                if (c != j) g[j * r + c] *= pinv;              // row j
+            __syncwarp();
+            for (int c = lane; c < r; c += 32) {               // rows i != j, columns c != j
+                if (c == j) continue;
+                const float mjc = g[j * r + c];
+                for (int i0 = 0; i0 < r; i0 += 8) {            // 8 rows' loads ahead of their stores
+                    float mij[8], mic[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int i = min(i0 + q, r - 1);
+                        mij[q] = g[i * r + j];
+                        mic[q] = g[i * r + c];
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int i = i0 + q;
+                        if (i < r && i != j) g[i * r + c] = fmaf(-mij[q], mjc, mic[q]);
+                    }
+                }
             }
             __syncwarp();
-            if (lane == 0) g[j * r + j] = d;
+            for (int i = lane; i < r; i += 32)                 // column j last
+                g[i * r + j] = i == j ? pinv : -g[i * r + j] * pinv;
             __syncwarp();
         }
         if (lane == 0) {
@@ -429,26 +468,33 @@ __device__ __forceinline__ void build_map(const FlushParams& p, const float2 (&s
     }
     __syncthreads();
 
-    // 3. C = L^-T L^-1 Z, one column of dk per thread, then stored
+    // 3. C = M^-1 Z, one column of dk per thread, four map rows at a time,
+    //    stored straight to HBM in the sketch dtype
     const bool good = map_ok != 0;
+    const long long row = b * p.R + p.off[h];
     for (int k = t; k < K; k += T) {
-        if (good) {
-            for (int e = 0; e < r; ++e) {
-                float acc = zs[e * K + k];
-                for (int f = 0; f < e; ++f) acc = fmaf(-g[e * r + f], zs[f * K + k], acc);
-                zs[e * K + k] = acc / g[e * r + e];
+        for (int e0 = 0; e0 < r; e0 += 4) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (good) {
+                const float* m0 = g + min(e0, r - 1) * r;
+                const float* m1 = g + min(e0 + 1, r - 1) * r;
+                const float* m2 = g + min(e0 + 2, r - 1) * r;
+                const float* m3 = g + min(e0 + 3, r - 1) * r;
+                for (int f = 0; f < r; ++f) {
+                    const float z = zs[f * K + k];
+                    acc[0] = fmaf(m0[f], z, acc[0]);
+                    acc[1] = fmaf(m1[f], z, acc[1]);
+                    acc[2] = fmaf(m2[f], z, acc[2]);
+                    acc[3] = fmaf(m3[f], z, acc[3]);
+                }
             }
-            for (int e = r - 1; e >= 0; --e) {
-                float acc = zs[e * K + k];
-                for (int f = e + 1; f < r; ++f) acc = fmaf(-g[f * r + e], zs[f * K + k], acc);
-                zs[e * K + k] = acc / g[e * r + e];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (e0 + q >= r) break;
+                const long long o = (row + e0 + q) * K + k;
+                if (p.sketch_bf16) static_cast<uint16_t*>(p.cmap)[o] = f2bf(acc[q]);
+                else static_cast<float*>(p.cmap)[o] = acc[q];
             }
-        }
-        const long long row = b * p.R + p.off[h];
-        for (int e = 0; e < r; ++e) {
-            const float c = good ? zs[e * K + k] : 0.f;
-            if (p.sketch_bf16) static_cast<uint16_t*>(p.cmap)[(row + e) * K + k] = f2bf(c);
-            else static_cast<float*>(p.cmap)[(row + e) * K + k] = c;
         }
     }
 }
@@ -734,7 +780,7 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
                 } else {
                     *reinterpret_cast<float2*>(static_cast<float*>(p.sketch) + row * V + col) = us;
                 }
-                if (MAP) *reinterpret_cast<float2*>(reinterpret_cast<float*>(smem + L.tile) + e * V + col) = us;
+                if (MAP) *reinterpret_cast<float2*>(reinterpret_cast<float*>(smem + L.tile) + e * umap_stride(V) + col) = us;
             } else if (e == r_h && p.has_token) {
                 *reinterpret_cast<float2*>(p.out + u * V + col) = make_float2(v2[0], v2[1]);
             }
