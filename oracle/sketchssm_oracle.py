@@ -235,7 +235,7 @@ class Session:
     """
 
     def __init__(self, family, state, window, A=None, basis=None, coef=None,
-                 offsets=None, sketch_bf16=False, state_map=False, rho=0.0):
+                 offsets=None, sketch_bf16=False, state_map=False, rho=0.0, dense=None):
         self.family = family
         self.S = np.asarray(state, dtype=np.float64).copy()     # [B, H, K, V]
         self.B, self.H, self.K, self.V = self.S.shape
@@ -248,6 +248,13 @@ class Session:
             coef = np.asarray(coef, dtype=np.float64)
             self.P = [basis[self.offsets[h]:self.offsets[h + 1]].T for h in range(self.H)]
             self.C = [coef[self.offsets[h]:self.offsets[h + 1]] for h in range(self.H)]
+        # Dense-fallback heads (paper App. D: they "read a BF16 state copy"):
+        # the sketch of P = I is that copy (u_k = S0^T e_k = row k of S0), and
+        # the read is S0^T q~ through the identity map.
+        self.dense = np.zeros(self.H, bool) if dense is None else np.asarray(dense, bool)
+        for h in np.flatnonzero(self.dense):
+            self.P[h] = np.eye(self.K)
+            self.C[h] = np.eye(self.K)
         self.sketch_bf16 = sketch_bf16
         self.state_map, self.rho = state_map, rho
         self.ring = []
@@ -275,16 +282,18 @@ class Session:
             U = [round_bf16(u) for u in U]
         self.U = U
         if self.state_map:
-            Cs = [coefficient_map(U[h], self.S[:, h], self.rho) for h in range(self.H)]
-            self.Cs = [round_bf16(c) for c in Cs] if self.sketch_bf16 else Cs
+            Cs = [None if self.dense[h] else coefficient_map(U[h], self.S[:, h], self.rho)
+                  for h in range(self.H)]
+            self.Cs = [c if c is None or not self.sketch_bf16 else round_bf16(c) for c in Cs]
 
     def coef(self, h):
         """The coefficient map head h's reads use: [r, K] or [B, r, K]."""
-        return self.Cs[h] if self.state_map else self.C[h]
+        return self.Cs[h] if self.state_map and not self.dense[h] else self.C[h]
 
     def packed_map(self):
-        """State-dependent maps in the library's packed layout [B][R][K]."""
-        return np.concatenate(self.Cs, axis=1)
+        """State-dependent maps in the library's packed layout [B][R][K]
+        (a dense head's rows, which the library never writes, as zeros)."""
+        return np.concatenate([np.zeros((self.B, self.K, self.K)) if c is None else c for c in self.Cs], axis=1)
 
     def packed_sketch(self):
         """Sketch in the library's packed layout [B][R][V] (row = u_i)."""

@@ -30,7 +30,8 @@ class ss_config(ctypes.Structure):
     _fields_ = [("family", ctypes.c_int32), ("batch", ctypes.c_int32), ("heads", ctypes.c_int32),
                 ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("ranks", ctypes.POINTER(ctypes.c_int32)), ("sketch_dtype", ctypes.c_int32),
-                ("coef_mode", ctypes.c_int32), ("coef_ridge", ctypes.c_float)]
+                ("coef_mode", ctypes.c_int32), ("coef_ridge", ctypes.c_float),
+                ("dense_heads", ctypes.POINTER(ctypes.c_uint8))]
 
 
 class ss_sizes(ctypes.Structure):
@@ -176,11 +177,14 @@ class Plan:
     """Owns an ss_plan*; destroyed with the object."""
 
     def __init__(self, family, batch, heads, dk, dv, window, ranks, sketch_dtype=SS_F32,
-                 coef_mode=SS_COEF_FIXED, coef_ridge=0.0):
+                 coef_mode=SS_COEF_FIXED, coef_ridge=0.0, dense_heads=None):
         self.ranks = (ctypes.c_int32 * heads)(*[int(r) for r in ranks])
+        self.dense_heads = None if dense_heads is None else (ctypes.c_uint8 * heads)(*[int(bool(d)) for d in dense_heads])
         cfg = ss_config(family, batch, heads, dk, dv, window,
                         ctypes.cast(self.ranks, ctypes.POINTER(ctypes.c_int32)), sketch_dtype,
-                        coef_mode, coef_ridge)
+                        coef_mode, coef_ridge,
+                        None if self.dense_heads is None
+                        else ctypes.cast(self.dense_heads, ctypes.POINTER(ctypes.c_uint8)))
         h = ctypes.c_void_p()
         _check(lib().ss_create(ctypes.byref(cfg), ctypes.byref(h)))
         self.handle = h

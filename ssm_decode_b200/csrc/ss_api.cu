@@ -12,7 +12,7 @@
 
 namespace ss {
 int flush_smem_bytes(int family, int dk, int dv, int n, int rpad, bool smap);
-int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz, bool smap);
+int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz, bool smap, bool dense_any);
 bool flush_map_fits(int dk, int dv, int r);
 }  // namespace ss
 
@@ -20,7 +20,9 @@ struct ss_plan {
     ss_config cfg;
     int32_t ranks[SS_MAX_HEADS];
     int32_t off[SS_MAX_HEADS + 1];
-    int32_t R, rmax, Wg;
+    int32_t R, rmax, Wg;      // rmax: largest rank of a sketched (not dense) head
+    uint32_t dense[SS_MAX_HEADS / 32];
+    int32_t n_dense;
     int32_t phase;
     int32_t sketch_valid;
     int32_t stall_next;
@@ -126,6 +128,7 @@ ss::FlushParams flush_params(const ss_plan* pl, const ss_buffers* b, const ss_st
         p.cmap = b->coef_state;
         p.ridge = pl->cfg.coef_ridge;
     }
+    std::memcpy(p.dense, pl->dense, sizeof p.dense);
     std::memcpy(p.off, pl->off, sizeof(int32_t) * (pl->cfg.heads + 1));
     return p;
 }
@@ -141,6 +144,8 @@ ss::StepParams step_params(const ss_plan* pl, const ss_buffers* b, const ss_step
     p.p = pl->phase;
     p.sketch_bf16 = pl->cfg.sketch_dtype == SS_BF16;
     if (state_map(pl)) p.cmap = b->coef_state;
+    std::memcpy(p.dense, pl->dense, sizeof p.dense);
+    p.dense_any = pl->n_dense > 0;
     std::memcpy(p.off, pl->off, sizeof(int32_t) * (pl->cfg.heads + 1));
     return p;
 }
@@ -153,6 +158,12 @@ ss_status launched(cudaError_t e, const char* what) {
 }
 
 int esize(const ss_plan* pl) { return pl->cfg.sketch_dtype == SS_BF16 ? 2 : 4; }
+
+// After a flush that sketches: the dense-fallback heads' state copies.
+ss_status dense_copies(const ss_plan* pl, const ss::FlushParams& p, cudaStream_t st) {
+    if (pl->n_dense == 0 || !p.do_sketch) return SS_OK;
+    return launched(ss::launch_dense_copy(pl->cfg.dk, pl->cfg.dv, p, st), "dense copy");
+}
 
 }  // namespace
 
@@ -184,6 +195,7 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
     std::memset(pl, 0, sizeof *pl);
     pl->cfg = c;
     pl->cfg.ranks = nullptr;
+    pl->cfg.dense_heads = nullptr;
     pl->off[0] = 0;
     pl->rmax = 0;
     for (int h = 0; h < c.heads; ++h) {
@@ -191,6 +203,18 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
         if (r < 0 || r > c.dk) {
             delete pl;
             return fail(SS_ERR_INVALID_ARG, "ranks[%d] = %d outside 0..dk", h, r);
+        }
+        const bool dense = c.dense_heads != nullptr && c.dense_heads[h] != 0;
+        if (dense) {
+            if (r != c.dk) {
+                delete pl;
+                return fail(SS_ERR_INVALID_ARG, "dense head %d needs rank dk = %d (has %d)", h, c.dk, r);
+            }
+            pl->dense[h >> 5] |= 1u << (h & 31);
+            pl->n_dense += 1;
+            pl->ranks[h] = r;
+            pl->off[h + 1] = pl->off[h] + r;
+            continue;
         }
         if (c.coef_mode == SS_COEF_STATE && !ss::flush_map_fits(c.dk, c.dv, r)) {
             delete pl;
@@ -207,7 +231,8 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
     const int rpad = (pl->rmax + 1 + 3) & ~3;
     const bool smap = c.coef_mode == SS_COEF_STATE;
     const int fl = ss::flush_smem_bytes(c.family, c.dk, c.dv, c.window, rpad, smap);
-    const int dec = ss::decode_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax, esize(pl), smap);
+    const int dec = ss::decode_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax, esize(pl), smap,
+                                          pl->n_dense > 0);
     if (fl > kSmemLimit || dec > kSmemLimit) {
         const int rmax = pl->rmax;
         delete pl;
@@ -279,6 +304,7 @@ ss_status ss_prime(ss_plan* pl, const ss_buffers* b, ss_stream stream) {
     p.stall = take_stall(pl);
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
                                     reinterpret_cast<cudaStream_t>(stream)), "prime"));
+    CHECK(dense_copies(pl, p, reinterpret_cast<cudaStream_t>(stream)));
     pl->sketch_valid = 1;
     return ok();
 }
@@ -325,6 +351,7 @@ ss_status ss_flush(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_st
     p.stall = take_stall(pl);
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
                                     reinterpret_cast<cudaStream_t>(stream)), "flush"));
+    CHECK(dense_copies(pl, p, reinterpret_cast<cudaStream_t>(stream)));
     pl->phase = 0;
     pl->sketch_valid = sk;
     return ok();
@@ -402,6 +429,7 @@ ss_status ss_step_mixed(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
     f.fill_in = fill_in;
     f.fill_out = fill_out;
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, f, pl->rmax, st), "mixed flush"));
+    CHECK(dense_copies(pl, f, st));
     return ok();
 }
 
@@ -424,29 +452,34 @@ ss_status ss_traffic_bytes(const ss_plan* pl, int32_t op, int32_t tau, ss_traffi
     double R = pl->R;   // sum of ranks over heads
     double rd = 0, wr = 0, prd = 0, pwr = 0;
     const double bh = B * H;
-    const double basis_bytes = R * K * 4;                // once per head per launch
     const double sketch_bytes = B * R * V * sk;          // U of every sequence
     const bool smap = c.coef_mode == SS_COEF_STATE;
-    const double map_bytes = smap ? B * R * K * sk : 0;  // per-sequence maps (SS_COEF_STATE)
-    const double paper_tg = B * R * (K + V) * 2 + (m2 ? 0 : B * R * W * 2);
+    // Dense-fallback heads: their dk sketch rows are the state copy; no
+    // basis, coef or map rows of theirs are read, and each flush that
+    // sketches reads their new state once more to write the copy.
+    const double nd = pl->n_dense, Rs = R - nd * K;      // ranks of the sketched heads
+    const double basis_s = Rs * K * 4;                   // basis / fixed map rows actually read
+    const double copy_rd = B * nd * D;
+    const double map_bytes = smap ? B * Rs * K * sk : 0; // per-sequence maps (SS_COEF_STATE)
+    const double paper_tg = B * Rs * (K + V) * 2 + (m2 ? 0 : B * Rs * W * 2) + B * nd * K * V * 2;
     switch (op) {
         case SS_OP_DECODE:
-            rd = bh * (tok + tau * slot) + sketch_bytes + (smap ? map_bytes : basis_bytes) + A;
+            rd = bh * (tok + tau * slot) + sketch_bytes + (smap ? map_bytes : basis_s) + A;
             wr = bh * (slot + 4 * V);
             prd = paper_tg;
             break;
         case SS_OP_FLUSH:
-            rd = bh * (D + (W - 1) * slot + tok) + basis_bytes + A;
+            rd = bh * (D + (W - 1) * slot + tok) + basis_s + copy_rd + A;
             wr = bh * (D + 4 * V) + sketch_bytes + map_bytes;
             prd = bh * D; pwr = bh * D;
             break;
         case SS_OP_FLUSH_NO_TOKEN:
-            rd = bh * (D + tau * slot) + basis_bytes + A;
+            rd = bh * (D + tau * slot) + basis_s + copy_rd + A;
             wr = bh * D + sketch_bytes + map_bytes;
             prd = bh * D; pwr = bh * D;
             break;
         case SS_OP_PRIME:
-            rd = bh * D + basis_bytes;
+            rd = bh * D + basis_s + copy_rd;
             wr = sketch_bytes + map_bytes;
             prd = bh * D;
             break;

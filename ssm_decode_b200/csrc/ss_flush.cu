@@ -110,7 +110,7 @@ template <int FAM, int K, int V>
 __device__ __forceinline__ void issue_window(const FlushParams& p, long long u, unsigned char* base,
                                              const FlushLayout& L, uint64_t* bar, unsigned extra) {
     const int h = int(u % p.H);
-    const int r = p.do_sketch ? p.off[h + 1] - p.off[h] : 0;
+    const int r = p.do_sketch && !head_dense(p.dense, h) ? p.off[h + 1] - p.off[h] : 0;   // basis rows
     mbar_expect_tx(bar, window_bytes<FAM, K, V>(p, r) + extra);
     const long long ring_row = u * p.W;
     const int nr = p.n_ring, n4r = (nr + 3) & ~3;
@@ -583,7 +583,8 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_kernel(const __g
         }
 
         // 2. Per-head preparation: keys, decays, coefficients, extended basis.
-        const int r_h = p.do_sketch ? p.off[h + 1] - p.off[h] : 0;
+        // dense-fallback heads keep no sketch here: dense_copy_kernel writes their state copy
+        const int r_h = p.do_sketch && !head_dense(p.dense, h) ? p.off[h + 1] - p.off[h] : 0;
         const int next = r_h + p.has_token;                           // columns of [Omega_h | q]
         const int nch = (next + 3) / 4;
         prepare_head<FAM, K, V>(p, h, n, r_h, rpad, sl, L, smem, tgate, tbeta, t);
@@ -848,6 +849,60 @@ cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int r
 }
 
 bool flush_map_fits(int dk, int dv, int r) { return map_fits(dk, dv, r); }
+
+namespace {
+
+// The dense-fallback heads of a launch (project page and paper App. D:
+// such heads read a BF16 copy of their state at non-flush steps).
+struct DenseList {
+    int n;
+    int16_t head[SS_MAX_HEADS];
+};
+
+// After a flush has written the state: copy each dense head's state into its
+// sketch rows, row k = S[k][:], in the sketch dtype.  Block (i, b) copies
+// head dl.head[i] of sequence b; in a mixed step only flushing sequences.
+template <int K, int V>
+__global__ void __launch_bounds__(256) dense_copy_kernel(const __grid_constant__ FlushParams p,
+                                                         const __grid_constant__ DenseList dl) {
+    const int h = dl.head[blockIdx.x];
+    const long long b = blockIdx.y;
+    if (p.fill_in != nullptr && p.fill_in[b] != p.W - 1) return;
+    const float4* src = reinterpret_cast<const float4*>(p.state + (b * p.H + h) * (long long)(K * V));
+    const long long row0 = b * p.R + p.off[h];
+    for (int i = threadIdx.x; i < K * V / 4; i += blockDim.x) {
+        const float4 a = src[i];
+        const int k = (4 * i) / V, v = (4 * i) % V;
+        const long long o = (row0 + k) * V + v;
+        if (p.sketch_bf16)
+            *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.sketch) + o) =
+                make_uint2(uint32_t(f2bf(a.x)) | (uint32_t(f2bf(a.y)) << 16),
+                           uint32_t(f2bf(a.z)) | (uint32_t(f2bf(a.w)) << 16));
+        else
+            *reinterpret_cast<float4*>(static_cast<float*>(p.sketch) + o) = a;
+    }
+}
+
+template <int K, int V>
+cudaError_t dense_copy_t(const FlushParams& p, const DenseList& dl, cudaStream_t stream) {
+    dense_copy_kernel<K, V><<<dim3(unsigned(dl.n), unsigned(p.B)), dim3(256), 0, stream>>>(p, dl);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Launch dense_copy_kernel for the dense heads of p.dense (none: nothing).
+cudaError_t launch_dense_copy(int dk, int dv, const FlushParams& p, cudaStream_t stream) {
+    DenseList dl;
+    dl.n = 0;
+    for (int h = 0; h < p.H; ++h)
+        if (head_dense(p.dense, h)) dl.head[dl.n++] = int16_t(h);
+    if (dl.n == 0 || !p.do_sketch) return cudaSuccess;
+    if (dk == 128 && dv == 128) return dense_copy_t<128, 128>(p, dl, stream);
+    if (dk == 128 && dv == 64) return dense_copy_t<128, 64>(p, dl, stream);
+    if (dk == 64 && dv == 128) return dense_copy_t<64, 128>(p, dl, stream);
+    return dense_copy_t<64, 64>(p, dl, stream);
+}
 
 // rpad = rows of [Omega | q] rounded up to 4 (the CUDA-core kernel's read-out
 // passes); smap: the flush builds the state-dependent map (CUDA-core kernel).

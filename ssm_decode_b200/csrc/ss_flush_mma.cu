@@ -79,7 +79,7 @@ template <int K, int V>
 __device__ __forceinline__ void mma_issue_window(const FlushParams& p, long long u, unsigned char* smem,
                                                  const MmaLayout& L, uint64_t* bar, unsigned extra) {
     const int h = int(u % p.H);
-    const int r = p.do_sketch ? p.off[h + 1] - p.off[h] : 0;
+    const int r = p.do_sketch && !head_dense(p.dense, h) ? p.off[h + 1] - p.off[h] : 0;   // basis rows
     mbar_expect_tx(bar, mma_window_bytes<K, V>(p, r) + extra);
     const int nr = p.n_ring, n4r = (nr + 3) & ~3;
     if (nr > 0) {
@@ -262,7 +262,8 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
         }
 
         // 2. Per-head preparation.
-        const int r_h = p.do_sketch ? p.off[h + 1] - p.off[h] : 0;
+        // dense-fallback heads keep no sketch here: dense_copy_kernel writes their state copy
+        const int r_h = p.do_sketch && !head_dense(p.dense, h) ? p.off[h + 1] - p.off[h] : 0;
         const int ne = r_h + p.has_token;                             // columns of [Omega_h | q]
         mma_prepare<K, V>(p, h, n, r_h, e16, smem, L, tgate, t);
         __syncthreads();                                              // (B)

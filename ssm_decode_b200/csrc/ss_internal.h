@@ -41,6 +41,10 @@ struct FlushParams {
     // for every head it sketches, as [B][R][dk] in the sketch dtype.
     void* cmap;
     float ridge;
+    // Dense-fallback heads (bit h): the sketch rows of head h hold a copy of
+    // its state, row k = S[k][:], in the sketch dtype, written by the flush
+    // instead of S^T Omega; no basis rows are read for them.
+    uint32_t dense[SS_MAX_HEADS / 32];
     int off[SS_MAX_HEADS + 1];
 };
 
@@ -75,8 +79,15 @@ struct StepParams {
     // SS_COEF_STATE: per-unit maps [B][R][dk] in the sketch dtype, staged with
     // each unit instead of the shared `coef` (decode only).
     const void* cmap;
+    // Dense-fallback heads (bit h): the read is S0^T q~ from the state copy in
+    // the sketch rows, streamed from HBM; no map, nothing staged for it.
+    // dense_any: some head is dense (the unit buffer then holds q~, dk floats).
+    uint32_t dense[SS_MAX_HEADS / 32];
+    int dense_any;
     int off[SS_MAX_HEADS + 1];
 };
+
+__host__ __device__ inline bool head_dense(const uint32_t* mask, int h) { return (mask[h >> 5] >> (h & 31)) & 1u; }
 
 // Launchers return the launch's cudaError_t (cudaSuccess when queued).
 // `rmax` is the largest per-head rank taking part in the launch.
@@ -84,6 +95,8 @@ cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int r
                          cudaStream_t stream);
 // Mamba-2 flush on the tensor cores (any dk, dv in {64, 128}).
 cudaError_t launch_flush_mma(int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream);
+// After a flush with a sketch: the dense-fallback heads' state copies.
+cudaError_t launch_dense_copy(int dk, int dv, const FlushParams& p, cudaStream_t stream);
 int flush_mma_smem_bytes(int dk, int dv, int n, int e16);
 cudaError_t launch_decode(int family, int dk, int dv, const StepParams& p, int rmax,
                           cudaStream_t stream);

@@ -404,6 +404,13 @@ constexpr int DEC_WARPS = 4;              // warps per decode CTA
 // per unit, which 32 lanes (one unit per warp, more warps per SM) hide best.
 __host__ __device__ constexpr int dec_gl(int fam) { return fam == MAMBA2 ? 16 : 32; }
 
+// A unit's sketch (and own map) rows; with dense-fallback heads in the plan
+// at least dk floats, which hold q~ for a dense head's read.
+__host__ __device__ inline int dec_ubytes(int K, int V, int rmax, int esz, bool smap, bool dense_any) {
+    const int ub = rmax * (V + (smap ? K : 0)) * esz;
+    return dense_any && ub < K * 4 ? K * 4 : ub;
+}
+
 __host__ __device__ inline int dec_stage_bytes(int fam, int K, int V, int P, int ubytes) {
     return 16 + (32 / dec_gl(fam)) * unit_smem(fam, K, V, P, ubytes).total;   // mbarrier + the warp's units
 }
@@ -544,13 +551,16 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
     const int ngroups = (p.B + UPW - 1) / UPW;
     const int gstride = gridDim.x * wpc;
     const int g0 = blockIdx.x * wpc + warp;
-    const int off = p.off[h], r = p.off[h + 1] - off;
+    // A dense-fallback head (its sketch rows hold a copy of the state) stages
+    // no sketch or map rows: its read streams the copy from HBM.
+    const bool dense = head_dense(p.dense, h);
+    const int off = p.off[h], r = dense ? 0 : p.off[h + 1] - off;
     const int P = p.p;
     // With the state-dependent map each unit stages its own C rows (r x dk,
     // sketch dtype) after its sketch rows; otherwise the CTA stages the
     // head's shared fp32 C once.
     const bool smap = p.cmap != nullptr;
-    const UnitSmem L = unit_smem(FAM, K, V, P, rmax * (V + (smap ? K : 0)) * ESZ);
+    const UnitSmem L = unit_smem(FAM, K, V, P, dec_ubytes(K, V, rmax, ESZ, smap, p.dense_any));
     const int cbytes = smap ? 0 : align16(rmax * K * 4);
     const float* csm = reinterpret_cast<const float*>(smem);
     uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + cbytes);
@@ -612,7 +622,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         if (!ok) break;
         phases ^= 1u << s;
         pending &= ~(1u << s);
-        const unsigned char* sh = wbase + s * stage_bytes + 16 + g * L.total;
+        unsigned char* sh = wbase + s * stage_bytes + 16 + g * L.total;
         const uint16_t* kraw = reinterpret_cast<const uint16_t*>(sh + L.kraw);
         const uint16_t* vraw = reinterpret_cast<const uint16_t*>(sh + L.vraw);
         const float* graw = reinterpret_cast<const float*>(sh + L.graw);
@@ -845,6 +855,23 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
 
         // 3. Coefficients c = C q~ and the sketched read o = U c + term,
         //    4 rows of C at a time.
+        if (dense) {
+            // Dense fallback: o += S0^T q~ from the state copy (row k = S0[k][:]);
+            // q~ goes through the unit's buffer so every lane sees all of it.
+            float* xs = reinterpret_cast<float*>(sh + L.ush);
+            store_row_f32<K, G>(xs, x, l);
+            __syncwarp();
+            if (active) {
+                const char* rows = static_cast<const char*>(p.sketch) + (b * (long long)p.R + off) * (V * ESZ);
+                for (int k0 = 0; k0 < K; k0 += 8) {
+                    float ui[8][EV];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) row_any<V, G, UB16>(rows + (k0 + q) * V * ESZ, l, ui[q]);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) axpy<EV>(xs[k0 + q], ui[q], ob);
+                }
+            }
+        }
         const unsigned char* us = sh + L.ush;
         const unsigned char* cmu = us + r * V * ESZ;          // this unit's map rows (smap)
         auto crow = [&](int i, float (&ci)[EK]) {
@@ -981,8 +1008,8 @@ __global__ void __launch_bounds__(128) replay_kernel(const __grid_constant__ Ste
 // ---------------------------------------------------------------------------
 // One warp's staging buffer; with the state-dependent map (`smap`) each unit
 // also stages its own map rows.
-int decode_stage(int fam, int K, int V, int P, int rmax, int esz, bool smap) {
-    return dec_stage_bytes(fam, K, V, P, rmax * (V + (smap ? K : 0)) * esz);
+int decode_stage(int fam, int K, int V, int P, int rmax, int esz, bool smap, bool dense_any) {
+    return dec_stage_bytes(fam, K, V, P, dec_ubytes(K, V, rmax, esz, smap, dense_any));
 }
 
 // The CTA-wide part: the head's shared C (fixed map only) and its mbarrier.
@@ -992,7 +1019,7 @@ template <int FAM, int K, int V, bool UB16, bool MIXED>
 cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
     constexpr int esz = UB16 ? 2 : 4, upw = 32 / dec_gl(FAM);
     const bool smap = p.cmap != nullptr;
-    const int stage = decode_stage(FAM, K, V, p.p, rmax, esz, smap);
+    const int stage = decode_stage(FAM, K, V, p.p, rmax, esz, smap, p.dense_any != 0);
     const int cpart = decode_cpart(K, rmax, smap);
     if (cpart + stage > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
     int wpc = DEC_WARPS;
@@ -1043,8 +1070,8 @@ cudaError_t launch_replay(int family, int dk, int dv, const StepParams& p, cudaS
     SS_DISPATCH(replay_t, p, stream);
 }
 
-int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz, bool smap) {
-    return decode_cpart(dk, rmax, smap) + decode_stage(family, dk, dv, P, rmax, esz, smap);
+int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz, bool smap, bool dense_any) {
+    return decode_cpart(dk, rmax, smap) + decode_stage(family, dk, dv, P, rmax, esz, smap, dense_any);
 }
 
 }  // namespace ss

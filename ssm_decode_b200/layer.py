@@ -36,9 +36,10 @@ class DecodeLayer:
     """Plan plus caller-owned device buffers for one linear-attention layer."""
 
     def __init__(self, family, batch, heads, dk, dv, window, ranks, sketch_dtype=B.SS_F32,
-                 device="cuda", coef_mode=B.SS_COEF_FIXED, coef_ridge=0.0):
+                 device="cuda", coef_mode=B.SS_COEF_FIXED, coef_ridge=0.0, dense_heads=None):
         import torch
-        self.plan = B.Plan(family, batch, heads, dk, dv, window, ranks, sketch_dtype, coef_mode, coef_ridge)
+        self.plan = B.Plan(family, batch, heads, dk, dv, window, ranks, sketch_dtype, coef_mode, coef_ridge,
+                           dense_heads)
         self.family, self.batch, self.heads, self.dk, self.dv, self.window = family, batch, heads, dk, dv, window
         self.device = device
         sz = B.ss_buffer_sizes(self.plan)

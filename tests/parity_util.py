@@ -59,7 +59,7 @@ class Pair:
     compare sampled sequences); the GPU always runs the whole batch.
     """
 
-    def __init__(self, wl, st=None, sketch_dtype=B.SS_F32, sel=None, state_map=False, rho=0.0):
+    def __init__(self, wl, st=None, sketch_dtype=B.SS_F32, sel=None, state_map=False, rho=0.0, dense=None):
         import torch
         self.wl = wl
         self.st = st if st is not None else synth.static_inputs(wl)
@@ -68,11 +68,12 @@ class Pair:
         self.layer = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, wl.window,
                                  self.st.ranks, sketch_dtype,
                                  coef_mode=B.SS_COEF_STATE if state_map else B.SS_COEF_FIXED,
-                                 coef_ridge=rho)
+                                 coef_ridge=rho, dense_heads=dense)
         self.layer.load(self.st.state, self.st.basis, self.st.coef, self.st.A)
         self.sess = orc.Session(wl.family, self.st.state[self.sel], wl.window, self.st.A,
                                 self.st.basis, self.st.coef, self.st.offsets,
-                                sketch_bf16=sketch_dtype == B.SS_BF16, state_map=state_map, rho=rho)
+                                sketch_bf16=sketch_dtype == B.SS_BF16, state_map=state_map, rho=rho,
+                                dense=dense)
         self.bf16 = sketch_dtype == B.SS_BF16
         self.ring_k = np.zeros((wl.batch, wl.heads, wl.window, wl.dk), np.uint16)
         self.ring_v = np.zeros((wl.batch, wl.heads, wl.window, wl.dv), np.uint16)
@@ -125,13 +126,14 @@ class Pair:
         g = to_np(self.layer.coef_state)[self.sel]
         if self.bf16:
             Ug = self.gpu_sketch_heads()
-            ref = np.concatenate([orc.round_bf16(orc.coefficient_map(Ug[h], self.sess.S[:, h], self.sess.rho))
+            ref = np.concatenate([np.zeros((len(self.sel), self.wl.dk, self.wl.dk)) if self.sess.dense[h] else
+                                  orc.round_bf16(orc.coefficient_map(Ug[h], self.sess.S[:, h], self.sess.rho))
                                   for h in range(self.wl.heads)], axis=1)
         else:
             ref = self.sess.packed_map()
         offs = self.st.offsets
         for h in range(self.wl.heads):
-            if offs[h + 1] == offs[h]:
+            if offs[h + 1] == offs[h] or self.sess.dense[h]:     # a dense head has no map
                 continue
             gh, rh = g[:, offs[h]:offs[h + 1]], ref[:, offs[h]:offs[h + 1]]
             if self.bf16:
@@ -199,7 +201,10 @@ class Pair:
                 offs = self.st.offsets
                 ref = np.empty_like(o_hat)
                 for h in range(self.wl.heads):
-                    c = np.einsum("brk,bk->br", Cg[:, offs[h]:offs[h + 1]], self.sess.last_q_tilde[:, h])
+                    if self.sess.dense[h]:                               # the identity map
+                        c = self.sess.last_q_tilde[:, h]
+                    else:
+                        c = np.einsum("brk,bk->br", Cg[:, offs[h]:offs[h + 1]], self.sess.last_q_tilde[:, h])
                     ref[:, h] = np.einsum("bvr,br->bv", Ug[h], c) + self.sess.last_o_buf[:, h]
                 err = vec_relerr(g, ref)
                 self.worst["sketched"] = max(self.worst["sketched"], err)

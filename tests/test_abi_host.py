@@ -174,6 +174,28 @@ def test_state_map_config_sizes_and_traffic(L):
         B.Plan(B.SS_MAMBA2, 1, 1, K, V, 16, [min(K, V) // 2], B.SS_BF16, B.SS_COEF_STATE)
 
 
+def test_dense_heads_config_and_traffic(L):
+    """Dense-fallback heads: rank dk, their state copy in the sketch rows."""
+    with pytest.raises(B.SSError) as e:
+        B.Plan(B.SS_GDN, 2, 3, 128, 64, 8, [5, 64, 7], B.SS_BF16, dense_heads=[0, 1, 0])
+    assert e.value.status == B.SS_ERR_INVALID_ARG and "dense head 1" in B.ss_last_error_string()
+    d = B.Plan(B.SS_GDN, 2, 3, 128, 64, 8, [5, 128, 7], B.SS_BF16, dense_heads=[0, 1, 0])
+    s = B.Plan(B.SS_GDN, 2, 3, 128, 64, 8, [5, 128, 7], B.SS_BF16)
+    assert B.ss_buffer_sizes(d)["sketch"] == 2 * 140 * 64 * 2
+    dd, ds = B.ss_traffic_bytes(d, B.SS_OP_DECODE, 3), B.ss_traffic_bytes(s, B.SS_OP_DECODE, 3)
+    # the dense head's 128 basis/coef rows are not read
+    assert ds["read_bytes"] - dd["read_bytes"] == 128 * 128 * 4
+    fd, fs = B.ss_traffic_bytes(d, B.SS_OP_FLUSH), B.ss_traffic_bytes(s, B.SS_OP_FLUSH)
+    # the copy re-reads each sequence's dense state once; no basis rows for it
+    assert fd["read_bytes"] - fs["read_bytes"] == 2 * 128 * 64 * 4 - 128 * 128 * 4
+    # paper metric: the dense head reads a bf16 state copy, dk x dv, per non-flush step
+    assert dd["paper_read_bytes"] == 2 * (12 * (128 + 64) * 2 + 12 * 8 * 2 + 128 * 64 * 2)
+    # a dense head does not raise the sketched heads' staging (rank 128 would not fit here)
+    B.Plan(B.SS_KDA, 1, 2, 128, 128, 32, [128, 16], B.SS_F32, dense_heads=[1, 0])
+    with pytest.raises(B.SSError):
+        B.Plan(B.SS_KDA, 1, 2, 128, 128, 32, [128, 16], B.SS_F32)
+
+
 @pytest.mark.skipif(not _no_gpu(), reason="fake-pointer validation tests run on CPU hosts only")
 def test_state_map_needs_its_buffer(L):
     p = B.Plan(B.SS_KDA, 2, 2, 64, 64, 4, [2, 3], B.SS_F32, B.SS_COEF_STATE, 0.0)
