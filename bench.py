@@ -343,32 +343,65 @@ def run_ours(args, rank, world):
     for lay in layers:
         lay.prime()
 
-    # end to end through the C ABI: pinned host inputs in, outputs back, every call
+    # end to end through the C ABI: pinned host inputs in, outputs back, every
+    # call.  Copies are pipelined the way a serving loop would run them: the
+    # inputs of later launches are copied in on one stream and finished
+    # outputs read back on another while the kernels run; NB device buffers
+    # rotate, each copy waiting (CUDA events) for the last use of its buffer.
     keys = ("q", "k", "v", "gate") + (() if wl.family == synth.MAMBA2 else ("beta",))
     pin = [{k: torch.from_numpy(np.ascontiguousarray(x[k].view(np.int16) if x[k].dtype == np.uint16 else x[k]))
             .pin_memory() for k in keys} for x in host_inputs]
     host_out = torch.empty((W, NL) + tuple(layers[0].out.shape), dtype=torch.float32).pin_memory()
     h2d = NL * sum(t.numel() * t.element_size() for x in pin for t in x.values())
     d2h = host_out.numel() * host_out.element_size()
+    NB = 2 * NL
+    from ssm_decode_b200.layer import Token
+    dev_tok = [Token({k: torch.empty_like(v) for k, v in toks[0].items()}) for _ in range(NB)]
+    dev_out = [torch.empty_like(layers[0].out) for _ in range(NB)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    used = [None] * NB      # event: the kernel that last read dev_tok[i] / wrote dev_out[i] is done
+    drained = [None] * NB   # event: dev_out[i] has been copied back
     e2e_times = []
     for k in range(args.warmup + args.steps):
         a, b = ev(), ev()
         torch.cuda.synchronize()
         a.record(stream)
+        s_in.wait_event(a)
+        s_out.wait_event(a)
+        n = 0
         for p in range(W):
             for l, lay in enumerate(layers):
-                tok = toks[(p + l) % W]
-                for key, t in pin[(p + l) % W].items():
-                    tok[key].copy_(t, non_blocking=True)
-                lay.step(tok)
-                host_out[p, l].copy_(lay.out, non_blocking=True)
+                i = n % NB
+                with torch.cuda.stream(s_in):
+                    if used[i] is not None:
+                        s_in.wait_event(used[i])
+                    for key, t in pin[(p + l) % W].items():
+                        dev_tok[i][key].copy_(t, non_blocking=True)
+                    ready = torch.cuda.Event()
+                    ready.record(s_in)
+                stream.wait_event(ready)
+                if drained[i] is not None:
+                    stream.wait_event(drained[i])
+                lay.step(dev_tok[i], out=dev_out[i])
+                used[i] = torch.cuda.Event()
+                used[i].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(used[i])
+                    host_out[p, l].copy_(dev_out[i], non_blocking=True)
+                    drained[i] = torch.cuda.Event()
+                    drained[i].record(s_out)
+                n += 1
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
         b.record(stream)
         torch.cuda.synchronize()
         if k >= args.warmup:
             e2e_times.append(a.elapsed_time(b))
     e2e_ms = reduce_max(sum(e2e_times), dev)
     e2e = {"value": weak_scaling_value(units * W * NL * args.steps, world, e2e_ms / 1e3),
-           "unit": "seq*heads/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "unit": "seq*heads/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "copies": "pinned host buffers; input copies and output read-backs pipelined on two "
+                     "copy streams against the kernels, all inside the timed region"}
 
     result = {
         "metric": "decode steps/sec (seq*heads/s), flush + sketched decode",
