@@ -262,8 +262,12 @@ ss_status ss_replay_step(ss_plan* plan, const ss_buffers* bufs, const ss_step_io
  * 0..W-1 sets SS_DEVICE_BAD_FILL in bufs->status; that sequence's outputs,
  * ring, state and fill_out entry are left as they were.  Needs the plan at
  * phase 0 with a valid sketch (ss_prime), bufs->state, sketch, basis, coef
- * (and A for Mamba-2); the plan's phase is not used and stays 0.  Two
- * kernels on `stream`; the fills are read on the device only. */
+ * (and A for Mamba-2); the plan's phase is not used and stays 0.  The
+ * decode runs on `stream`; the flush runs beside it on a stream the plan
+ * owns (created on first use), forked from `stream` after its earlier work
+ * and joined back to it with events, so work queued on `stream` afterwards
+ * sees both (this also holds under stream capture).  The fills are read on
+ * the device only. */
 ss_status ss_step_mixed(ss_plan* plan, const ss_buffers* bufs, const ss_step_io* io,
                         const int32_t* fill_in, int32_t* fill_out, ss_stream stream);
 
