@@ -179,13 +179,15 @@ typedef struct {
     /* State-access traffic as the paper counts it (paper App. D, Table 4 as
      * summarised on the paperlayer page): fp32 state reads and writes plus
      * bf16 sketch + coefficient-map reads of G (dk + dv) elements per head at
-     * non-flush steps (plus G W bf16 projected erase vectors for GDN/KDA).
+     * non-flush steps (plus G W bf16 projected erase vectors for GDN/KDA); a
+     * dense-fallback head reads a bf16 dk x dv state copy instead.
      * Ring-buffer traffic and sketch/map writes are excluded, as there. */
     double paper_read_bytes;
     double paper_write_bytes;
-    /* Every byte this library's kernel for the call must move (inputs,
-     * ring slots, state, sketch, basis/map once per head, outputs).  This is
-     * the numerator of the HBM roofline. */
+    /* Every byte this library's kernels for the call must move (inputs,
+     * ring slots, state, sketch, basis/map once per head or per sequence,
+     * outputs, and the extra state read that writes dense heads' copies).
+     * This is the numerator of the HBM roofline. */
     double read_bytes;
     double write_bytes;
 } ss_traffic;
