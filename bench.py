@@ -141,10 +141,13 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 def kernel_source_sha():
-    """Hash of the CUDA sources, to tell whether ncu counters are still current."""
+    """Hash of the device-code sources (every CUDA source but the host-only
+    API file), to tell whether ncu counters are still current."""
     d = os.path.join(ROOT, "ssm_decode_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(d)):
+        if f == "ss_api.cu":
+            continue
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]

@@ -421,11 +421,21 @@ ss_status ss_step_mixed(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
     CHECK(check_io(pl, io));
     CHECK(check_status(b));
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (pl->side == nullptr) {
-        cudaError_t e = cudaStreamCreateWithFlags(&pl->side, cudaStreamNonBlocking);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pl->fork, cudaEventDisableTiming);
-        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pl->join, cudaEventDisableTiming);
-        if (e != cudaSuccess) return fail(SS_ERR_CUDA, "mixed step: side stream: %s", cudaGetErrorString(e));
+    if (pl->side == nullptr) {                 // all three or none
+        cudaStream_t side = nullptr;
+        cudaEvent_t fork = nullptr, join = nullptr;
+        cudaError_t e = cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            if (join) cudaEventDestroy(join);
+            if (fork) cudaEventDestroy(fork);
+            if (side) cudaStreamDestroy(side);
+            return fail(SS_ERR_CUDA, "mixed step: side stream: %s", cudaGetErrorString(e));
+        }
+        pl->side = side;
+        pl->fork = fork;
+        pl->join = join;
     }
     const int stall = take_stall(pl);
     const int W = pl->cfg.window;
