@@ -210,6 +210,68 @@ def sketch_vs_exact(layers, toks, W, torch):
     return res
 
 
+def other_modes(args, wl, st, layers, toks, W, units, dev, stream, torch, B, DecodeLayer):
+    """Outside the timed region: the same workload with sequences at mixed
+    window positions (ss_step_mixed) and with the state-dependent map, each
+    timed with CUDA events over a few steps.  Errors are reported, not raised."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    out = {}
+    try:                                   # mixed positions: fills spread evenly over 0..W-1
+        fills = [torch.arange(wl.batch, dtype=torch.int32, device=dev) % W for _ in layers]
+        nxt = [torch.empty_like(f) for f in fills]
+        ts = []
+        for k in range(3):
+            a, b = ev(), ev()
+            a.record(stream)
+            for p in range(W):
+                for l, lay in enumerate(layers):
+                    lay.step_mixed(toks[(p + l) % W], fills[l], nxt[l])
+                    fills[l], nxt[l] = nxt[l], fills[l]
+            b.record(stream)
+            torch.cuda.synchronize()
+            if k:
+                ts.append(a.elapsed_time(b))
+        ms = min(ts) / (W * len(layers))
+        out["mixed"] = {"what": "ss_step_mixed, fills spread evenly over the window, every layer",
+                        "us_per_step": ms * 1e3, "value": units / (ms / 1e3), "unit": "seq*heads/s",
+                        "status": int(sum(int(l.status[0].item()) for l in layers))}
+    except Exception as e:                 # noqa: BLE001 - reported in the line
+        out["mixed"] = {"error": repr(e)[:200]}
+    try:                                   # the state-dependent coefficient map (rho 0.01)
+        import numpy as np  # noqa: F401
+        skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
+        sl = []
+        for _ in range(2):
+            lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev,
+                              coef_mode=B.SS_COEF_STATE, coef_ridge=0.01)
+            lay.state.copy_(layers[0].state)
+            lay.basis.copy_(layers[0].basis)
+            lay.A.copy_(layers[0].A)
+            lay.prime()
+            sl.append(lay)
+        ts = []
+        for k in range(3):
+            a, b = ev(), ev()
+            a.record(stream)
+            for p in range(W):
+                for l, lay in enumerate(sl):
+                    lay.step(toks[(p + l) % W])
+            b.record(stream)
+            torch.cuda.synchronize()
+            if k:
+                ts.append(a.elapsed_time(b))
+        ms = min(ts) / len(sl)
+        approx = sketch_vs_exact(sl, toks, W, torch)
+        out["state_map"] = {"what": "the same window with the state-dependent map (rho 0.01) built by every flush",
+                            "ms_per_window": ms, "value": units * W / (ms / 1e3), "unit": "seq*heads/s",
+                            "approx_mean": approx["mean"], "approx_aggregate": approx["aggregate"]}
+        del sl
+        torch.cuda.empty_cache()
+    except Exception as e:                 # noqa: BLE001
+        out["state_map"] = {"error": repr(e)[:200]}
+    return out
+
+
 def run_ours(args, rank, world):
     import torch
     from ssm_decode_b200 import binding as B
@@ -406,6 +468,9 @@ def run_ours(args, rank, world):
            "copies": "pinned host buffers; input copies and output read-backs pipelined on two "
                      "copy streams against the kernels, all inside the timed region"}
 
+    modes = other_modes(args, wl, st, layers, toks, W, units, dev, stream, torch, B, DecodeLayer) \
+        if rank == 0 else None
+
     result = {
         "metric": "decode steps/sec (seq*heads/s), flush + sketched decode",
         "value": value, "unit": "seq*heads/s", "n_gpus": world, "steps": args.steps,
@@ -419,7 +484,7 @@ def run_ours(args, rank, world):
                    "l2": f"inputs larger than L2: {NL} layers rotated, back-to-back launches",
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline, "kernels": kernels, "baselines": baselines, "e2e": e2e,
-        "gpu_launches": launches, "clocks": clk.summary(), "approx": approx,
+        "gpu_launches": launches, "clocks": clk.summary(), "approx": approx, "modes": modes,
     }
     return result
 
