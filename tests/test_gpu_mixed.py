@@ -84,7 +84,7 @@ def _check_step(layer, sess, inp, fill, wl):
             assert err <= TOL, f"seq {b} at fill {fill[b]}: sketched output relerr {err:.3e}"
 
 
-@pytest.mark.parametrize("window", [2, 5, 16])
+@pytest.mark.parametrize("window", [1, 2, 5, 16])
 @pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
 def test_mixed_positions_match_per_sequence_oracle(cuda_ok, family, window):
     """Every starting position 0..W-1 is present (ragged: the batch is not a
