@@ -176,6 +176,32 @@ __device__ __forceinline__ long long fq_next(const FlushParams& p, FlushQueue* q
     return u;
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl may start
+// while the previous kernel in the stream is still finishing; it runs only
+// set-up that touches no global memory (shared memory, mbarriers) before
+// griddep_wait(), which returns once the previous kernel has completed and
+// its writes are visible, so the data order is the plain stream order.
+// griddep_launch_next() then lets the next such kernel start its set-up.
+// Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 __device__ __forceinline__ void report_timeout(int32_t* status) {
     if (status != nullptr) atomicOr(status, SS_DEVICE_TIMEOUT);
 }

@@ -215,6 +215,8 @@ __global__ void __launch_bounds__(2 * V, V == 64 ? 3 : 2) flush_mma_kernel(const
         if (MIXED) fq_init(fq);
     }
     __syncthreads();
+    griddep_wait();                                   // the previous kernel's writes are visible
+    griddep_launch_next();
     if constexpr (MIXED) {
         if (warp == 0) fq_next(p, fq, units);
         __syncthreads();
@@ -423,8 +425,7 @@ cudaError_t flush_mma_launch(const FlushParams& p, int rmax, cudaStream_t stream
     const long long units = (long long)p.B * p.H;
     const long long cap = (long long)per_sm * sm_count();
     const long long grid = units < cap ? units : cap;
-    kern<<<dim3(unsigned(grid)), dim3(MS<K, V>::T), bytes, stream>>>(p, map, e16);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(unsigned(grid)), dim3(MS<K, V>::T), bytes, stream, p, map, e16);
 }
 
 // A mixed step (fill_in set) runs its own instance: the unit selection would

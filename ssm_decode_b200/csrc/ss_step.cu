@@ -566,7 +566,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
     uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + cbytes);
     unsigned char* wbase = smem + cbytes + 16 + warp * ns * stage_bytes;
     const bool stall = p.stall && blockIdx.x == 0 && blockIdx.y == 0 && warp == 0;
-    const float A = FAM == MAMBA2 ? p.A[h] : 0.f;
 
     auto bar = [&](int s) { return reinterpret_cast<uint64_t*>(wbase + s * stage_bytes); };
     unsigned pending = 0;      // bit s: stage s has copies in flight
@@ -594,6 +593,9 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         for (int s = 0; s < ns; ++s) mbar_init(bar(s), UPW);
     fence_mbar_init();
     __syncthreads();                                        // the only block barrier
+    griddep_wait();                                         // the previous kernel's writes are visible
+    griddep_launch_next();
+    const float A = FAM == MAMBA2 ? p.A[h] : 0.f;
     if (threadIdx.x == 0) {
         mbar_expect_tx(cbar, smap ? 0 : r * K * 4);
         if (!smap && r > 0) bulk_g2s(smem, p.coef + (long long)off * K, r * K * 4, cbar);
@@ -1031,8 +1033,7 @@ cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const long long groups = (p.B + upw - 1) / upw;
     const long long nb = (groups + wpc - 1) / wpc;          // one group per warp
-    kern<<<dim3(unsigned(nb), unsigned(p.H)), dim3(wpc * 32), bytes, stream>>>(p, rmax, 1, stage);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(unsigned(nb), unsigned(p.H)), dim3(wpc * 32), bytes, stream, p, rmax, 1, stage);
 }
 
 template <int FAM, int K, int V>
