@@ -143,3 +143,53 @@ def test_allocation_favours_sensitive_high_error_heads():
 def test_budget_below_cheapest_is_refused():
     with pytest.raises(ValueError):
         cal.allocate(np.ones((2, 2)), np.ones((2, 2)), 1.0)
+
+
+def test_calibration_feeds_the_library():
+    """Bases and ranks calibrated on a synthetic model are valid library input:
+    the plan accepts the ranks and dense flags, its buffers hold the packed
+    basis and map rows, and the oracle's sketched read with the calibrated
+    basis and map has the error the calibration predicted."""
+    from oracle import sketchssm_oracle as orc
+    from ssm_decode_b200 import binding as B
+    from ssm_decode_b200 import build
+    build.build()
+    wl = synth.Workload("calpipe", synth.GDN, 24, 6, 64, 64, 16, 0, 8, 11)
+    st = synth.static_inputs(wl)
+    q = np.stack([synth.bf16_bits_to_f32(synth.step_inputs(wl, st, t)["q"]) for t in range(20)])   # [T, B, H, K]
+    bases, errors = [], []
+    for h in range(wl.heads):
+        hb = cal.fit_head_basis(st.state[:, h], q[:, :, h].reshape(-1, wl.dk))
+        bases.append(hb)
+        errors.append([cal.reconstruction_error(hb, st.state[:, h], q[:, :, h].reshape(-1, wl.dk), r)
+                       for r in range(17)])
+    sens = np.random.default_rng(12).uniform(0.5, 2.0, wl.heads)
+    alloc = cal.allocate_ranks(np.array(errors), sens, wl.dk, wl.dv, wl.window, mean_rank=8)
+    dense = alloc.ranks == cal.DENSE
+    ranks = np.where(dense, wl.dk, alloc.ranks).astype(np.int32)
+    basis = np.concatenate([np.eye(wl.dk) if dense[h] else bases[h].omega[:, :ranks[h]].T
+                            for h in range(wl.heads)]).astype(np.float32)
+    coef = np.concatenate([np.eye(wl.dk) if dense[h] else bases[h].coef[:ranks[h]]
+                           for h in range(wl.heads)]).astype(np.float32)
+    plan = B.Plan(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, wl.window, ranks, B.SS_BF16,
+                  dense_heads=dense.astype(np.uint8))
+    sizes = B.ss_buffer_sizes(plan)
+    assert sizes["total_rank"] == ranks.sum() == len(basis) == len(coef)
+    assert sizes["basis"] == basis.nbytes and sizes["coef"] == coef.nbytes
+    # the oracle reads with the calibrated basis and map: error as predicted
+    offs = np.concatenate([[0], np.cumsum(ranks)])
+    sess = orc.Session(wl.family, st.state, wl.window, None, basis, coef, offs, dense=dense)
+    sess.prime()
+    qt = q[0]                                           # no buffered updates: q~ = q
+    for h in range(wl.heads):
+        if dense[h]:
+            continue
+        o = np.einsum("bkv,bk->bv", st.state[:, h], qt[:, h])
+        o_hat = orc.sketched_output(sess.U[h], sess.C[h], qt[:, h], 0.0)
+        got = np.mean(np.sum((o - o_hat) ** 2, axis=-1))
+        hb = bases[h]
+        # the same error from the calibration side, on these states and queries
+        proj = hb.omega[:, :ranks[h]] @ hb.coef[:ranks[h]]
+        d = qt[:, h] - qt[:, h] @ proj.T
+        want = np.mean(np.einsum("bk,bkv,bjv,bj->b", d, st.state[:, h], st.state[:, h], d))
+        assert abs(got - want) <= 1e-6 * max(want, 1e-12) + 1e-9
