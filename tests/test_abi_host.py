@@ -264,3 +264,28 @@ def test_all_bytes_model(L):
 def test_status_strings(L):
     assert B.ss_status_string(B.SS_ERR_SCHEDULE) == "SS_ERR_SCHEDULE"
     assert B.ss_status_string(99) == "unknown ss_status"
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="fake-pointer validation tests run on CPU hosts only")
+def test_mixed_step_host_checks(L):
+    """ss_step_mixed refuses bad fills and schedules before launching anything."""
+    p = B.Plan(B.SS_GDN, 4, 2, 64, 64, 4, [2, 3])
+    st = ctypes.c_void_p(0)
+    bufs, io = _fake_bufs(), _fake_io()
+    fin, fout = ctypes.c_void_p(0x700000), ctypes.c_void_p(0x710000)
+
+    def rc(fi, fo, b=bufs):
+        return L.ss_step_mixed(p.handle, ctypes.byref(b), ctypes.byref(io), fi, fo, st)
+
+    assert rc(fin, fout) == B.SS_ERR_SCHEDULE                  # no sketch yet (ss_prime first)
+    B.ss_set_phase(p, 2, True)
+    assert rc(fin, fout) == B.SS_ERR_SCHEDULE                  # the plan must sit at phase 0
+    B.ss_set_phase(p, 0, True)
+    assert rc(None, fout) == B.SS_ERR_INVALID_ARG
+    assert rc(fin, None) == B.SS_ERR_INVALID_ARG
+    assert rc(ctypes.c_void_p(0x700002), fout) == B.SS_ERR_ALIGNMENT
+    assert rc(fin, fin) == B.SS_ERR_INVALID_ARG                 # fill_out may not alias fill_in
+    assert "alias" in B.ss_last_error_string()
+    for name in ("sketch", "basis", "coef", "state"):
+        assert rc(fin, fout, _fake_bufs(null=name)) == B.SS_ERR_INVALID_ARG, name
+    assert B.ss_get_phase(p) == (0, True) and B.ss_launch_count() == 0
