@@ -120,8 +120,8 @@ typedef struct {
     int32_t coef_mode;       /* ss_coef_mode; 0 (zero-initialised) = SS_COEF_FIXED */
     float coef_ridge;        /* rho >= 0 of SS_COEF_STATE (ignored otherwise) */
     const uint8_t* dense_heads; /* host [heads] or NULL; copied.  Nonzero: a dense-fallback head
-                              * (paper App. D: it "reads a BF16 state copy" at non-flush
-                              * steps).  Its rank must be dk; its dk sketch rows hold the
+                              * (paper App. D: at non-flush steps it reads a BF16 copy of its
+                              * state).  Its rank must be dk; its dk sketch rows hold the
                               * copy, row k = S[k][:] in the sketch dtype, written by every
                               * flush with a sketch; its non-flush read is S0^T q~ + (buffered
                               * term), exact up to the copy's rounding.  Its basis, coef and

@@ -42,12 +42,12 @@ Readings of points the pages leave open:
 * P4 the coefficient map is either a fixed per-head matrix C (the workloads
   use C = P^T) or the state-dependent map of the project page ("Per window ·
   Flush: Sketch & coefficient map", C = (U^T U)^+ U^T S0^T; paper §A.2.1),
-  refreshed with the sketch at every flush.  The pages call the map "exact
-  regularized" without giving the regulariser; this oracle takes a ridge
+  refreshed with the sketch at every flush.  The pages compare against an
+  exact map with a regulariser whose value they do not give; this oracle takes a ridge
   relative to the Gram matrix's mean diagonal, lambda = rho * tr(U^T U) / r,
   so that rho = 0 is the pseudoinverse form for a full-column-rank U.  With a
   bf16 sketch the map is built from the stored (rounded) U and is itself
-  stored rounded to bf16 ("reads the BF16 sketch and coefficient map", §D).
+  stored rounded to bf16 (App. D has non-flush steps read both in BF16).
 * P7 a bf16 sketch is the fp64 sketch rounded once to bf16 (nearest, ties
   to even).
 
@@ -248,7 +248,7 @@ class Session:
             coef = np.asarray(coef, dtype=np.float64)
             self.P = [basis[self.offsets[h]:self.offsets[h + 1]].T for h in range(self.H)]
             self.C = [coef[self.offsets[h]:self.offsets[h + 1]] for h in range(self.H)]
-        # Dense-fallback heads (paper App. D: they "read a BF16 state copy"):
+        # Dense-fallback heads (paper App. D: they read a BF16 copy of their state):
         # the sketch of P = I is that copy (u_k = S0^T e_k = row k of S0), and
         # the read is S0^T q~ through the identity map.
         self.dense = np.zeros(self.H, bool) if dense is None else np.asarray(dense, bool)

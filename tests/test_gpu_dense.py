@@ -1,5 +1,5 @@
-"""GPU parity of dense-fallback heads (paper App. D: such heads "read a BF16
-state copy" at non-flush steps instead of a sketch).
+"""GPU parity of dense-fallback heads (paper App. D: at non-flush steps such
+heads read a BF16 copy of their state instead of a sketch).
 
 A dense head has rank dk; every flush with a sketch writes its state into its
 sketch rows (row k = S[k][:], in the sketch dtype) and its non-flush read is
