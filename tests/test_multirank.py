@@ -54,3 +54,21 @@ def test_single_process_defaults():
     import bench
     assert bench.reduce_max(3.25) == 3.25
     assert bench.weak_scaling_value(10.0, 1, 2.0) == 5.0
+
+
+def test_reference_arm_under_two_ranks():
+    """bench.py --impl reference launched as two ranks: rank 0 alone runs the
+    oracle on the host and prints one line; the other rank exits 0 silently."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"]
+    res = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["value"] > 0 and rec["e2e"]["h2d_bytes_per_step"] == 0
