@@ -48,6 +48,10 @@ Readings of points the pages leave open:
   so that rho = 0 is the pseudoinverse form for a full-column-rank U.  With a
   bf16 sketch the map is built from the stored (rounded) U and is itself
   stored rounded to bf16 (App. D has non-flush steps read both in BF16).
+  The pages' cheaper variant (§A.2.2: the state metric approximated as low
+  rank plus diagonal with P = 4 pivots) is read as keeping the n_piv output
+  columns of S with the most energy exactly and the rest as a diagonal
+  (coefficient_map_lrd); no kernel builds it yet.
 * P7 a bf16 sketch is the fp64 sketch rounded once to bf16 (nearest, ties
   to even).
 
@@ -185,6 +189,43 @@ def sketched_output(U, C, q_tilde, o_buf):
     C is [r, K] (fixed, shared by the batch) or [..., r, K] (state-dependent)."""
     c = np.einsum("...rk,...k->...r", C, q_tilde)
     return np.einsum("...vr,...r->...v", U, c) + o_buf
+
+
+def coefficient_map_lrd(S, P, n_piv=4, rho=0.0):
+    """The cheaper map of paper §A.2.2 under this reading: the state metric
+    H = S S^T (the exact map is C = (P^T H P)^-1 P^T H, since U = S^T P) is
+    replaced by H^ = L L^T + D, where L holds the n_piv output columns of S
+    with the largest energy ||S[:, v]||^2 (their correlations kept exactly)
+    and D = diag of the remaining columns' contribution (their coordinate-wise
+    energy).  C = (P^T H^ P + lambda I)^-1 P^T H^, lambda = rho tr(P^T H^ P) / r.
+    S [..., K, V], basis P [K, r] -> C [..., r, K].  Oracle only so far (no
+    kernel builds it yet)."""
+    S = np.asarray(S, dtype=np.float64)
+    P = np.asarray(P, dtype=np.float64)
+    K, V = S.shape[-2], S.shape[-1]
+    r = P.shape[-1]
+    if r == 0:
+        return np.zeros(S.shape[:-2] + (0, K))
+    energy = np.einsum("...kv,...kv->...v", S, S)                      # ||S[:, v]||^2
+    order = np.argsort(-energy, axis=-1, kind="stable")
+    piv = order[..., :n_piv]
+    rest = order[..., n_piv:]
+    L = np.take_along_axis(S, piv[..., None, :], axis=-1)               # [..., K, n_piv]
+    Sr = np.take_along_axis(S, rest[..., None, :], axis=-1)
+    d = np.einsum("...kv,...kv->...k", Sr, Sr)                          # diag of the rest
+    H = np.einsum("...kp,...jp->...kj", L, L) + d[..., :, None] * np.eye(K)
+    Z = np.einsum("kr,...kj->...rj", P, H)                              # P^T H^
+    G = np.einsum("...rj,js->...rs", Z, P)                              # P^T H^ P
+    lam = rho * np.trace(G, axis1=-2, axis2=-1) / r
+    A = G + lam[..., None, None] * np.eye(r)
+    C = np.zeros(Z.shape)
+    for idx in np.ndindex(A.shape[:-2]):
+        try:
+            np.linalg.cholesky(A[idx])
+        except np.linalg.LinAlgError:
+            continue
+        C[idx] = np.linalg.solve(A[idx], Z[idx])
+    return C
 
 
 def coefficient_map(U, S, rho=0.0):

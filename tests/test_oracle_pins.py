@@ -401,6 +401,42 @@ def test_coefficient_map_of_zero_state_is_zero():
     assert not orc.coefficient_map(orc.sketch(S, P), S, 0.5).any()
 
 
+def test_lrd_map_with_every_column_kept_is_the_exact_map():
+    """n_piv = V keeps every output column: H^ = H and the map is the exact one."""
+    S, P, U, q = _map_case(7, K=10, V=6, r=4)
+    for rho in (0.0, 0.2):
+        assert relerr(orc.coefficient_map_lrd(S, P, n_piv=6, rho=rho), orc.coefficient_map(U, S, rho)) < 1e-10
+
+
+def test_lrd_map_of_isotropic_energy_is_the_fixed_map():
+    """No pivots and equal coordinate-wise energy (H^ = cI): with an orthonormal
+    basis the map is P^T, the fixed map."""
+    K, V, r = 8, 16, 3
+    rng = np.random.default_rng(8)
+    Q = np.linalg.qr(rng.standard_normal((V, V)))[0][:K]        # orthonormal rows: S S^T = I
+    S = np.stack([2.0 * Q, 0.5 * Q])
+    P = np.linalg.qr(rng.standard_normal((K, K)))[0][:, :r]
+    C = orc.coefficient_map_lrd(S, P, n_piv=0)
+    assert relerr(C, np.broadcast_to(P.T, C.shape)) < 1e-10
+
+
+def test_lrd_map_matches_a_direct_construction():
+    """Against H^ built column by column from its definition (pivots by energy,
+    diagonal of the rest) and a least-squares solve in the H^ metric."""
+    S, P, U, q = _map_case(9, n=2, K=7, V=9, r=3)
+    C = orc.coefficient_map_lrd(S, P, n_piv=2)
+    for i in range(len(S)):
+        e = [float(S[i][:, v] @ S[i][:, v]) for v in range(S.shape[2])]
+        piv = sorted(range(len(e)), key=lambda v: -e[v])[:2]
+        H = sum(np.outer(S[i][:, v], S[i][:, v]) for v in piv)
+        H = H + np.diag(sum(S[i][:, v] ** 2 for v in range(len(e)) if v not in piv))
+        # c minimises (q - P c)^T H (q - P c): weighted least squares via a square root of H
+        w, Qh = np.linalg.eigh(H)
+        Hh = Qh @ np.diag(np.sqrt(np.maximum(w, 0))) @ Qh.T
+        c_ls = np.linalg.lstsq(Hh @ P, Hh @ q[i], rcond=None)[0]
+        assert relerr(C[i] @ q[i], c_ls) < 1e-8
+
+
 @pytest.mark.parametrize("family", FAMS)
 def test_session_state_map_identity_basis_reads_exactly(family):
     """Session with the state map and P = I (r = K <= V): every sketched read
@@ -460,6 +496,29 @@ def _run_map_pins():
 
 
 ORIG_MAP = orc.coefficient_map
+ORIG_LRD = orc.coefficient_map_lrd
+
+
+def _mut_lrd_no_diagonal(S, P, n_piv=4, rho=0.0):
+    # keeps only the pivot columns: the remaining coordinate-wise energy is dropped
+    e = np.einsum("...kv,...kv->...v", S, S)
+    keep = np.argsort(-e, axis=-1, kind="stable")[..., :n_piv]
+    mask = np.zeros(e.shape, bool)
+    np.put_along_axis(mask, keep, True, axis=-1)
+    return ORIG_LRD(S * mask[..., None, :], P, n_piv, rho)
+
+
+def test_planted_lrd_mistake_is_caught(monkeypatch):
+    def run():
+        try:
+            test_lrd_map_of_isotropic_energy_is_the_fixed_map()
+            test_lrd_map_matches_a_direct_construction()
+        except AssertionError:
+            return False
+        return True
+    assert run()
+    monkeypatch.setattr(orc, "coefficient_map_lrd", _mut_lrd_no_diagonal)
+    assert not run(), "dropping the diagonal went unnoticed"
 
 
 def _mut_map_no_ridge(U, S, rho=0.0):
