@@ -268,8 +268,9 @@ ss_status ss_replay_step(ss_plan* plan, const ss_buffers* bufs, const ss_step_io
  * decode runs on `stream`; the flush runs beside it on a stream the plan
  * owns (created on first use), forked from `stream` after its earlier work
  * and joined back to it with events, so work queued on `stream` afterwards
- * sees both (this also holds under stream capture).  The fills are read on
- * the device only. */
+ * sees both (this also holds under stream capture).  If a launch fails
+ * after the fork, the side stream is still joined back before the error
+ * (SS_ERR_CUDA) is returned.  The fills are read on the device only. */
 ss_status ss_step_mixed(ss_plan* plan, const ss_buffers* bufs, const ss_step_io* io,
                         const int32_t* fill_in, int32_t* fill_out, ss_stream stream);
 

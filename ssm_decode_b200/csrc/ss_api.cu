@@ -447,6 +447,10 @@ ss_status ss_step_mixed(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
     cudaError_t e = cudaEventRecord(pl->fork, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(pl->side, pl->fork, 0);
     if (e != cudaSuccess) return fail(SS_ERR_CUDA, "mixed step: fork: %s", cudaGetErrorString(e));
+    // Once forked, the side stream is joined back whatever happens below, so a
+    // failed launch never leaves a flush running unordered with the caller's
+    // later work; the first failure is the status returned.
+    ss_status s = SS_OK;
     {
         ss::FlushParams f = flush_params(pl, b, io);   // sequences with fill == W-1: the flush
         f.n_ring = W - 1;
@@ -454,20 +458,21 @@ ss_status ss_step_mixed(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
         f.do_sketch = 1;
         f.fill_in = fill_in;
         f.fill_out = fill_out;
-        CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, f, pl->rmax, pl->side),
-                       "mixed flush"));
-        CHECK(dense_copies(pl, f, pl->side));
+        s = launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, f, pl->rmax, pl->side),
+                     "mixed flush");
+        if (s == SS_OK) s = dense_copies(pl, f, pl->side);
     }
-    if (W > 1) {                              // sequences with fill < W-1: a non-flush step
+    if (s == SS_OK && W > 1) {                // sequences with fill < W-1: a non-flush step
         ss::StepParams p = step_params(pl, b, io);
         p.p = W - 2;                          // staging is sized for the longest window
         p.fill_in = fill_in;
         p.fill_out = fill_out;
         p.stall = stall;
-        CHECK(launched(ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax, st), "mixed decode"));
+        s = launched(ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax, st), "mixed decode");
     }
     e = cudaEventRecord(pl->join, pl->side);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, pl->join, 0);
+    if (s != SS_OK) return s;
     if (e != cudaSuccess) return fail(SS_ERR_CUDA, "mixed step: join: %s", cudaGetErrorString(e));
     return ok();
 }
