@@ -27,9 +27,13 @@
  *   - Pointers marked "device" must be device (or managed) addresses aligned
  *     to 16 bytes; a misaligned pointer returns SS_ERR_ALIGNMENT.
  *   - Launches are asynchronous on `stream` (NULL = the legacy default
- *     stream).  A call that returns an error launches nothing and leaves the
- *     plan unchanged.  Errors raised later by the device surface on the
- *     caller's next CUDA synchronisation.
+ *     stream).  A call rejected by its checks (any status but SS_ERR_CUDA)
+ *     launches nothing and leaves the plan unchanged.  SS_ERR_CUDA means a
+ *     kernel launch failed: kernels the call queued before it stay queued and
+ *     the plan accounts for them (a flush whose dense-head copies failed
+ *     leaves the plan at phase 0 with no valid sketch, so ss_prime comes
+ *     next).  Errors raised later by the device surface on the caller's next
+ *     CUDA synchronisation.
  *   - No call throws, exits or aborts; every call returns an ss_status.
  *     ss_last_error_string() describes the last failure on this thread.
  *   - bf16 tensors are passed as their uint16_t bit patterns.

@@ -360,8 +360,12 @@ ss_status ss_flush(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_st
     p.stall = take_stall(pl);
     CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
                                     reinterpret_cast<cudaStream_t>(stream)), "flush"));
-    CHECK(dense_copies(pl, p, reinterpret_cast<cudaStream_t>(stream)));
+    // The flush is queued: the window is applied whatever happens next.  If the
+    // dense heads' copies fail to launch, the plan is left at phase 0 without a
+    // valid sketch, so the next read asks for ss_prime instead of using it.
     pl->phase = 0;
+    pl->sketch_valid = 0;
+    CHECK(dense_copies(pl, p, reinterpret_cast<cudaStream_t>(stream)));
     pl->sketch_valid = sk;
     return ok();
 }
