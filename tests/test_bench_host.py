@@ -66,3 +66,20 @@ def test_kernel_source_sha_ignores_the_host_api_file(tmp_path, monkeypatch):
     assert bench.kernel_source_sha() == a
     (csrc / "k.cu").write_text("kernel changed")
     assert bench.kernel_source_sha() != a
+
+
+def test_cpu_baseline_all_cores_leg_and_its_fallback():
+    """The oracle baseline: a 1-thread figure, then single-threaded spawned
+    processes whose rates add up; a parallel leg that fails or runs out of
+    time leaves the 1-thread figure and says why."""
+    import argparse
+    a = argparse.Namespace(workload="mamba2_b4")
+    r = bench.cpu_baseline(a, one_s=0.3, each_s=0.3, max_workers=2)
+    assert r["kind"] == "oracle" and r["one_thread"]["value"] > 0
+    if bench.host_cores() > 1:
+        assert r["cores"] == 2 and "parallel_error" not in r
+        assert r["value"] > r["one_thread"]["value"]
+    f = bench.cpu_baseline(a, one_s=0.3, each_s=30.0, max_workers=2, timeout_s=0.5)
+    if bench.host_cores() > 1:
+        assert f["cores"] == 1 and f["value"] == f["one_thread"]["value"]
+        assert f["parallel_error"].startswith("TimeoutError")
