@@ -272,6 +272,95 @@ def other_modes(args, wl, st, layers, toks, W, units, dev, stream, torch, B, Dec
     return out
 
 
+NOMINAL_HBM_GBS = 8000.0        # B200 HBM3e data-sheet figure (context beside the measured copy peak)
+
+
+def kernel_stats(plan, B, W, dec_ms, n_dec, fl_ms, n_fl, flush_name, peak, wl_name, coef="fixed"):
+    """Per-kernel mean durations and HBM fractions: algorithmic bytes from the
+    library's traffic model (mean over the window's decode positions for the
+    decode) over the mean launch duration."""
+    dec_bytes = [B.ss_traffic_bytes(plan, B.SS_OP_DECODE, p) for p in range(W - 1)]
+    dec_b = sum(t["read_bytes"] + t["write_bytes"] for t in dec_bytes) / max(W - 1, 1)
+    fl = B.ss_traffic_bytes(plan, B.SS_OP_FLUSH)
+    fl_b = fl["read_bytes"] + fl["write_bytes"]
+    kernel_ms = dec_ms + fl_ms
+    kernels = {}
+    for name, ms, count, nbytes in (("decode_kernel", dec_ms, n_dec, dec_b), (flush_name, fl_ms, n_fl, fl_b)):
+        if not count:
+            continue
+        avg_s = ms / count / 1e3
+        ach = nbytes / avg_s / 1e9
+        rec = kernel_traffic_record(name, wl_name, coef)
+        kernels[name] = {"launches": count, "avg_us": avg_s * 1e6, "bytes_per_launch": nbytes,
+                         "achieved_gbs": ach, "frac": ach / peak, "frac_nominal": ach / NOMINAL_HBM_GBS,
+                         "share": ms / kernel_ms,
+                         "traffic": rec["dram_bytes_per_launch"] if rec else None,
+                         "timing": "events at window boundaries and around the flush group"}
+    return kernels
+
+
+def flush_kernel_name(family, smap, synth):
+    """The kernel that runs a family's flush (see launch_flush in the library)."""
+    if family == synth.MAMBA2 and not smap:
+        return "flush_mma_kernel"
+    return "flush_kernel"
+
+
+def other_families(args, dev, stream, torch, B, synth, DecodeLayer, peak, names=("gdn_b256", "kda_b256")):
+    """Outside the timed region (rank 0): the GDN and KDA target workloads'
+    decode and flush, timed like the headline workload (layers rotated so the
+    inputs exceed L2, back-to-back launches, events at window boundaries), so
+    one bench line carries every family's kernel fractions."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    out = {}
+    for name in names:
+        try:
+            wl = synth.WORKLOADS[name]
+            W, NL = wl.window, args.layers
+            st = synth.static_inputs(wl)
+            skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
+            layers = []
+            for _ in range(NL):
+                lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev)
+                lay.load(st.state, st.basis, st.coef, st.A)
+                layers.append(lay)
+            toks = [layers[0].token(synth.step_inputs(wl, st, t)) for t in range(W)]
+            for lay in layers:
+                lay.prime()
+
+            def window(marks=None):
+                if marks:
+                    marks[0].record(stream)
+                for p in range(W):
+                    if marks and p == W - 1:
+                        marks[1].record(stream)
+                    for l, lay in enumerate(layers):
+                        lay.step(toks[(p + l) % W])
+                if marks:
+                    marks[2].record(stream)
+
+            for _ in range(3):
+                window()
+            nwin = max(3, min(args.steps, 10))
+            marks = [(ev(), ev(), ev()) for _ in range(nwin)]
+            for m in marks:
+                window(m)
+            torch.cuda.synchronize()
+            dec_ms = sum(m[0].elapsed_time(m[1]) for m in marks)
+            fl_ms = sum(m[1].elapsed_time(m[2]) for m in marks)
+            tot_ms = sum(m[0].elapsed_time(m[2]) for m in marks)
+            kern = kernel_stats(layers[0].plan, B, W, dec_ms, nwin * NL * (W - 1), fl_ms, nwin * NL,
+                                flush_kernel_name(wl.family, False, synth), peak, wl.name)
+            out[name] = {"value": wl.units * W * NL * nwin / (tot_ms / 1e3), "unit": "seq*heads/s",
+                         "windows": nwin, "layers": NL, "kernels": kern,
+                         "status": int(sum(int(l.status[0].item()) for l in layers))}
+            del layers, toks
+            torch.cuda.empty_cache()
+        except Exception as e:             # noqa: BLE001 - reported in the line
+            out[name] = {"error": repr(e)[:200]}
+    return out
+
+
 def run_ours(args, rank, world):
     import torch
     from ssm_decode_b200 import binding as B
@@ -360,24 +449,8 @@ def run_ours(args, rank, world):
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
     plan = layers[0].plan
-    dec_bytes = [B.ss_traffic_bytes(plan, B.SS_OP_DECODE, p) for p in range(W - 1)]
-    dec_b = sum(t["read_bytes"] + t["write_bytes"] for t in dec_bytes) / max(W - 1, 1)
-    fl = B.ss_traffic_bytes(plan, B.SS_OP_FLUSH)
-    fl_b = fl["read_bytes"] + fl["write_bytes"]
-    kernel_ms = dec_ms + fl_ms
-    kernels = {}
-    # Mamba-2's flush runs on the tensor cores unless it also builds the state-dependent map
-    flush_name = "flush_mma_kernel" if wl.family == synth.MAMBA2 and not smap else "flush_kernel"
-    for name, ms, count, nbytes in (("decode_kernel", dec_ms, n_dec, dec_b), (flush_name, fl_ms, n_fl, fl_b)):
-        if not count:
-            continue
-        avg_s = ms / count / 1e3
-        ach = nbytes / avg_s / 1e9
-        rec = kernel_traffic_record(name, wl.name, args.coef)
-        kernels[name] = {"launches": count, "avg_us": avg_s * 1e6, "bytes_per_launch": nbytes,
-                         "achieved_gbs": ach, "frac": ach / peak, "share": ms / kernel_ms,
-                         "traffic": rec["dram_bytes_per_launch"] if rec else None,
-                         "timing": "events at window boundaries and around the flush group"}
+    flush_name = flush_kernel_name(wl.family, smap, synth)
+    kernels = kernel_stats(plan, B, W, dec_ms, n_dec, fl_ms, n_fl, flush_name, peak, wl.name, args.coef)
     if W > 1:
         kernels["decode_kernel"]["by_phase_us"] = [
             round(sum(per_launch[p][l][0].elapsed_time(per_launch[p][l][1]) for l in range(NL)) / NL * 1e3, 2)
@@ -387,7 +460,9 @@ def run_ours(args, rank, world):
     d = kernels[dom]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(d["achieved_gbs"], 1), "peak": peak,
                 "unit": "GB/s", "frac": round(d["frac"], 4), "traffic": d["traffic"],
-                "peak_source": f"{peak_kind} hbm_gbs (burst copy; kernels timed inside the step)"}
+                "peak_source": f"{peak_kind} hbm_gbs (burst copy; kernels timed inside the step)",
+                "frac_nominal": round(d["achieved_gbs"] / NOMINAL_HBM_GBS, 4),
+                "nominal_peak": NOMINAL_HBM_GBS}
 
     # baselines in the same library: Standard (exact step) and ReplaySSM
     baselines = {}
@@ -470,6 +545,11 @@ def run_ours(args, rank, world):
 
     modes = other_modes(args, wl, st, layers, toks, W, units, dev, stream, torch, B, DecodeLayer) \
         if rank == 0 else None
+    del layers, toks, dev_tok, dev_out
+    torch.cuda.empty_cache()
+    families = None
+    if rank == 0 and args.workload == "mamba2_b320" and not args.batch and not args.no_families:
+        families = other_families(args, dev, stream, torch, B, synth, DecodeLayer, peak)
 
     result = {
         "metric": "decode steps/sec (seq*heads/s), flush + sketched decode",
@@ -485,6 +565,7 @@ def run_ours(args, rank, world):
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline, "kernels": kernels, "baselines": baselines, "e2e": e2e,
         "gpu_launches": launches, "clocks": clk.summary(), "approx": approx, "modes": modes,
+        "families": families,
     }
     return result
 
@@ -696,6 +777,8 @@ def main():
                     help="override the workload's batch (smaller cases for profiler captures)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-families", action="store_true",
+                    help="skip the GDN / KDA kernel timings that follow the default Mamba-2 line")
     ap.add_argument("--coef", default="fixed", choices=["fixed", "state"],
                     help="coefficient map: the fixed C = P^T of the workloads, or the state-dependent "
                          "least-squares map rebuilt by every flush")

@@ -294,6 +294,16 @@ uint64_t ss_launch_count(void);
  * after that call.  Used to test the timeout path without a device fault. */
 ss_status ss_debug_stall_next_copy(ss_plan* plan, int32_t stall);
 
+/* Testing hook for the host-side launch-failure paths.  With n > 0, the
+ * n-th kernel launch that this plan's calls make from now on (counting
+ * every launch of every call: a flush with dense heads makes two, a mixed
+ * step two or three) is not made: the call behaves as if the CUDA runtime
+ * had refused it (SS_ERR_CUDA, "injected launch failure").  Launches queued
+ * before it stay queued and the plan accounts for them, as for a real
+ * failure.  The hook clears itself when it fires; n = 0 disarms it.  No
+ * device code is involved, so the path is tested without a GPU fault. */
+ss_status ss_debug_fail_launch(ss_plan* plan, int32_t n);
+
 const char* ss_status_string(ss_status status);
 const char* ss_last_error_string(void);
 

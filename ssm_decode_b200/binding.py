@@ -88,6 +88,7 @@ def lib():
             "ss_traffic_bytes": ([P, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ss_traffic)], S),
             "ss_launch_count": ([], ctypes.c_uint64),
             "ss_debug_stall_next_copy": ([P, ctypes.c_int32], S),
+            "ss_debug_fail_launch": ([P, ctypes.c_int32], S),
             "ss_status_string": ([S], ctypes.c_char_p),
             "ss_last_error_string": ([], ctypes.c_char_p),
         }
@@ -260,6 +261,11 @@ def ss_launch_count():
 
 def ss_debug_stall_next_copy(plan, stall=True):
     _check(lib().ss_debug_stall_next_copy(plan.handle, int(bool(stall))))
+
+
+def ss_debug_fail_launch(plan, n):
+    """Testing hook: the n-th launch of this plan's next calls is refused on the host."""
+    _check(lib().ss_debug_fail_launch(plan.handle, int(n)))
 
 
 def ss_status_string(s):

@@ -30,6 +30,7 @@ struct ss_plan {
     int32_t phase;
     int32_t sketch_valid;
     int32_t stall_next;
+    int32_t fail_launch;      // testing hook: the launch (1-based, counted from arming) to refuse
 };
 
 namespace {
@@ -161,12 +162,21 @@ ss_status launched(cudaError_t e, const char* what) {
     return SS_OK;
 }
 
+// Make one launch through the testing hook: when the plan's armed counter
+// reaches this launch, the launch is not made and an error stands for it.
+template <typename F>
+ss_status launch_via(ss_plan* pl, const char* what, F&& fn) {
+    if (pl->fail_launch > 0 && --pl->fail_launch == 0)
+        return fail(SS_ERR_CUDA, "%s launch failed: injected launch failure", what);
+    return launched(fn(), what);
+}
+
 int esize(const ss_plan* pl) { return pl->cfg.sketch_dtype == SS_BF16 ? 2 : 4; }
 
 // After a flush that sketches: the dense-fallback heads' state copies.
-ss_status dense_copies(const ss_plan* pl, const ss::FlushParams& p, cudaStream_t st) {
+ss_status dense_copies(ss_plan* pl, const ss::FlushParams& p, cudaStream_t st) {
     if (pl->n_dense == 0 || !p.do_sketch) return SS_OK;
-    return launched(ss::launch_dense_copy(pl->cfg.dk, pl->cfg.dv, p, st), "dense copy");
+    return launch_via(pl, "dense copy", [&] { return ss::launch_dense_copy(pl->cfg.dk, pl->cfg.dv, p, st); });
 }
 
 }  // namespace
@@ -311,8 +321,10 @@ ss_status ss_prime(ss_plan* pl, const ss_buffers* b, ss_stream stream) {
     ss::FlushParams p = flush_params(pl, b, nullptr);
     p.n_ring = 0; p.has_token = 0; p.do_sketch = 1;
     p.stall = take_stall(pl);
-    CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
-                                    reinterpret_cast<cudaStream_t>(stream)), "prime"));
+    CHECK(launch_via(pl, "prime", [&] {
+        return ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
+                                reinterpret_cast<cudaStream_t>(stream));
+    }));
     CHECK(dense_copies(pl, p, reinterpret_cast<cudaStream_t>(stream)));
     pl->sketch_valid = 1;
     return ok();
@@ -333,8 +345,10 @@ ss_status ss_decode_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io,
     CHECK(check_status(b));
     ss::StepParams p = step_params(pl, b, io);
     p.stall = take_stall(pl);
-    CHECK(launched(ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
-                                     reinterpret_cast<cudaStream_t>(stream)), "decode"));
+    CHECK(launch_via(pl, "decode", [&] {
+        return ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
+                                 reinterpret_cast<cudaStream_t>(stream));
+    }));
     pl->phase += 1;
     return ok();
 }
@@ -358,8 +372,10 @@ ss_status ss_flush(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, ss_st
     p.has_token = io != nullptr;
     p.do_sketch = sk;
     p.stall = take_stall(pl);
-    CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
-                                    reinterpret_cast<cudaStream_t>(stream)), "flush"));
+    CHECK(launch_via(pl, "flush", [&] {
+        return ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax,
+                                reinterpret_cast<cudaStream_t>(stream));
+    }));
     // The flush is queued: the window is applied whatever happens next.  If the
     // dense heads' copies fail to launch, the plan is left at phase 0 without a
     // valid sketch, so the next read asks for ss_prime instead of using it.
@@ -381,8 +397,10 @@ ss_status ss_exact_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
     ss::FlushParams p = flush_params(pl, b, io);
     p.n_ring = 0; p.has_token = 1; p.do_sketch = 0;
     p.stall = take_stall(pl);
-    CHECK(launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, 0,
-                                    reinterpret_cast<cudaStream_t>(stream)), "exact"));
+    CHECK(launch_via(pl, "exact", [&] {
+        return ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, 0,
+                                reinterpret_cast<cudaStream_t>(stream));
+    }));
     pl->sketch_valid = 0;
     return ok();
 }
@@ -397,8 +415,10 @@ ss_status ss_replay_step(ss_plan* pl, const ss_buffers* b, const ss_step_io* io,
     CHECK(check_status(b));
     ss::StepParams p = step_params(pl, b, io);
     p.stall = take_stall(pl);
-    CHECK(launched(ss::launch_replay(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p,
-                                     reinterpret_cast<cudaStream_t>(stream)), "replay"));
+    CHECK(launch_via(pl, "replay", [&] {
+        return ss::launch_replay(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p,
+                                 reinterpret_cast<cudaStream_t>(stream));
+    }));
     pl->phase += 1;
     return ok();
 }
@@ -462,8 +482,9 @@ ss_status ss_step_mixed(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
         f.do_sketch = 1;
         f.fill_in = fill_in;
         f.fill_out = fill_out;
-        s = launched(ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, f, pl->rmax, pl->side),
-                     "mixed flush");
+        s = launch_via(pl, "mixed flush", [&] {
+            return ss::launch_flush(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, f, pl->rmax, pl->side);
+        });
         if (s == SS_OK) s = dense_copies(pl, f, pl->side);
     }
     if (s == SS_OK && W > 1) {                // sequences with fill < W-1: a non-flush step
@@ -472,7 +493,9 @@ ss_status ss_step_mixed(ss_plan* pl, const ss_buffers* b, const ss_step_io* io, 
         p.fill_in = fill_in;
         p.fill_out = fill_out;
         p.stall = stall;
-        s = launched(ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax, st), "mixed decode");
+        s = launch_via(pl, "mixed decode", [&] {
+            return ss::launch_decode(pl->cfg.family, pl->cfg.dk, pl->cfg.dv, p, pl->rmax, st);
+        });
     }
     e = cudaEventRecord(pl->join, pl->side);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, pl->join, 0);
@@ -561,6 +584,13 @@ uint64_t ss_launch_count(void) { return g_launches.load(std::memory_order_relaxe
 ss_status ss_debug_stall_next_copy(ss_plan* pl, int32_t stall) {
     if (pl == nullptr) return fail(SS_ERR_INVALID_ARG, "plan is NULL");
     pl->stall_next = stall ? 1 : 0;
+    return ok();
+}
+
+ss_status ss_debug_fail_launch(ss_plan* pl, int32_t n) {
+    if (pl == nullptr) return fail(SS_ERR_INVALID_ARG, "plan is NULL");
+    if (n < 0) return fail(SS_ERR_INVALID_ARG, "n = %d < 0", n);
+    pl->fail_launch = n;
     return ok();
 }
 

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "ss_internal.h"
 
@@ -148,11 +149,14 @@ __device__ __forceinline__ long long fq_next(const FlushParams& p, FlushQueue* q
         int n = 0;
         while (pos < units && n <= FQ_CAP - 32) {
             const long long c = pos + (long long)lane * gridDim.x;
-            const bool hit = c < units && p.fill_in[c / p.H] == p.W - 1;
+            const int f = c < units ? p.fill_in[c / p.H] : 0;
+            const bool hit = c < units && f == p.W - 1;
             const unsigned m = __ballot_sync(0xffffffffu, hit);
             if (hit) {
                 q->unit[n + __popc(m & ((1u << lane) - 1u))] = int(c);
                 if (c % p.H == 0) p.fill_out[c / p.H] = 0;   // the sequence's new fill, once per sequence
+            } else if (c < units && (f < 0 || f > p.W - 1) && c % p.H == 0 && p.status != nullptr) {
+                atomicOr(p.status, SS_DEVICE_BAD_FILL);      // neither flushed nor decoded: reported once
             }
             n += __popc(m);
             pos += 32LL * gridDim.x;
@@ -272,12 +276,23 @@ cudaError_t cached_regs(F kern, KernelCache& kc, int* regs) {
     return cudaSuccess;
 }
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes`.  The
+// check, the attribute call and the cache update run under one lock, so two
+// host threads asking for different sizes cannot leave the attribute below
+// the cached value.
+inline std::mutex& smem_attr_mutex() {
+    static std::mutex mu;
+    return mu;
+}
+
 template <typename F>
 cudaError_t ensure_smem(F kern, KernelCache& kc, int bytes) {
     const int d = cur_device();
+    if (bytes <= kc.smem[d].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(smem_attr_mutex());
     if (bytes <= kc.smem[d].load(std::memory_order_relaxed)) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) kc.smem[d].store(bytes, std::memory_order_relaxed);
+    if (e == cudaSuccess) kc.smem[d].store(bytes, std::memory_order_release);
     return e;
 }
 

@@ -333,40 +333,6 @@ __device__ __forceinline__ void sweep_seq(const StepParams& p, int h, int l, con
     }
 }
 
-// c = C q~ for nr <= NR rows of C (shared memory), reduce-scattered; then
-// o += sum_i c_i u_i, the sketch rows read through `U(i, u)`.
-template <int NR, int K, int V, int LPU, typename LoadU>
-__device__ __forceinline__ void readout(const float* csm, int nr, int l, int gbase, const float (&x)[K / LPU],
-                                        float (&o)[V / LPU], LoadU U) {
-    constexpr int EK = K / LPU, EV = V / LPU;
-    using SC = Scatter<NR, LPU>;
-    float v[NR];
-#pragma unroll
-    for (int i = 0; i < NR; ++i) {
-        float acc = 0.f;
-        if (i < nr) {
-            float cr[EK];
-            ld_f32<EK>(csm + i * K + l * EK, cr);
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int e = 0; e < EK; e += 2) { a0 = fmaf(cr[e], x[e], a0); a1 = fmaf(cr[e + 1], x[e + 1], a1); }
-            acc = a0 + a1;
-        }
-        v[i] = acc;
-    }
-    group_reduce_scatter<NR, LPU>(v, l);
-#pragma unroll
-    for (int i = 0; i < NR; ++i) {
-        const float ci = __shfl_sync(FULL, v[SC::slot(i)], gbase + SC::holder(i));
-        if (i < nr) {
-            float u[EV];
-            U(i, u);
-#pragma unroll
-            for (int e = 0; e < EV; ++e) o[e] = fmaf(ci, u[e], o[e]);
-        }
-    }
-}
-
 template <int FAM, int K, int V, int LPU>
 __device__ __forceinline__ void window_read(const StepParams& p, int h, int l, int gbase, const unsigned char* sh,
                                             const UnitSmem& L, const Tok<K, V, LPU>& tk, float (&x)[K / LPU],

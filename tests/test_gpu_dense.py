@@ -89,3 +89,36 @@ def test_dense_heads_full_size_sampled(cuda_ok):
     st.coef = st.basis.copy()
     p = Pair(wl, st=st, sketch_dtype=B.SS_BF16, sel=[0, 128, 255], dense=dense)
     run(p, wl.window + 1)
+
+
+def test_flush_with_failed_dense_copy_needs_prime(cuda_ok):
+    """The flush is queued but the dense heads' copy launch is refused (the
+    host-side testing hook stands in for the runtime's refusal): the call
+    returns SS_ERR_CUDA, the window has been applied exactly once, and the
+    plan sits at phase 0 with no valid sketch, so reads are refused until
+    ss_prime rebuilds the sketch and the copies."""
+    import torch
+    wl, st, dense = case("gdn", 128, 64, window=4, seed=2600)
+    p = Pair(wl, st=st, dense=dense)
+    p.prime()
+    for t in range(wl.window - 1):
+        p.step(synth.step_inputs(wl, st, t))
+    inp = synth.step_inputs(wl, st, wl.window - 1)
+    tok = p.layer.token(inp)
+    B.ss_debug_fail_launch(p.layer.plan, 2)            # launch 1: the flush; launch 2: the copies
+    with pytest.raises(B.SSError) as err:
+        p.layer.flush(tok)
+    assert "injected" in str(err.value)
+    assert B.ss_get_phase(p.layer.plan) == (0, 0)
+    torch.cuda.synchronize()
+    o = p.sess.flush(inp)                               # the oracle's flush of the same window
+    p.check_state()
+    from tests.parity_util import vec_relerr
+    assert vec_relerr(p.out(), o) <= TOL
+    with pytest.raises(B.SSError):                      # no sketch: a read is a schedule error
+        p.layer.decode(p.layer.token(synth.step_inputs(wl, st, wl.window)))
+    p.layer.prime()                                     # the hook has fired: this runs
+    p.sess.prime()
+    p.check_sketch()
+    for t in range(wl.window, wl.window + 3):
+        p.step(synth.step_inputs(wl, st, t))

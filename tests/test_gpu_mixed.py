@@ -135,13 +135,15 @@ def test_mixed_uniform_equals_scheduled_steps(cuda_ok, family):
     assert torch.equal(a.ring_k, b_layer.ring_k)
 
 
-def test_mixed_bad_fill_sets_status_and_skips(cuda_ok):
+@pytest.mark.parametrize("W", [1, 4])
+def test_mixed_bad_fill_sets_status_and_skips(cuda_ok, W):
     """Fill counts outside 0..W-1 are refused on the device: the status word
     gets SS_DEVICE_BAD_FILL and those sequences are left untouched; the
-    others step normally."""
+    others step normally.  At W = 1 no decode kernel runs, so the flush's
+    unit queue is the one that reports the bad fills."""
     import torch
-    W, batch = 4, 5
-    fills = np.array([0, 1, 2, 3, 0], np.int32)
+    batch = 5
+    fills = np.array([0, 1, 2, 3, 0], np.int32) % W
     wl, st, layer, sess = _setup("gdn", W, batch, fills, seed=1300)
     bad = fills.copy()
     bad[1], bad[4] = W, -1
@@ -180,3 +182,51 @@ def test_mixed_host_checks(cuda_ok):
     layer.decode(tok)                                   # plan phase 1
     with pytest.raises(B.SSError):
         layer.step_mixed(tok, f, g)
+
+
+@pytest.mark.parametrize("fail_at", [1, 2])
+def test_mixed_launch_failure_still_joins(cuda_ok, fail_at):
+    """A mixed step whose flush (fail_at 1) or decode (fail_at 2) launch is
+    refused on the host: SS_ERR_CUDA comes back, the side stream has been
+    joined to the caller's stream, and whatever was queued ran to the
+    oracle's values; the next mixed step on the same plan runs normally."""
+    import torch
+    W, batch = 4, 4
+    fills = np.array([3, 1, 3, 0], np.int32)
+    wl, st, layer, sess = _setup("kda", W, batch, fills, seed=1500)
+    fin = torch.from_numpy(fills).cuda()
+    fout = torch.full_like(fin, -7)
+    layer.out.fill_(12.5)
+    inp = synth.step_inputs(wl, st, 0)
+    B.ss_debug_fail_launch(layer.plan, fail_at)
+    with pytest.raises(B.SSError) as err:
+        layer.step_mixed(layer.token(inp), fin, fout)
+    assert "injected" in str(err.value)
+    marker = torch.zeros(1, device="cuda")
+    marker.add_(1.0)                                    # queued after the join on the caller's stream
+    torch.cuda.synchronize()
+    assert marker.item() == 1.0
+    g = to_np(layer.out)
+    flushing = [b for b in range(batch) if fills[b] == W - 1]
+    decoding = [b for b in range(batch) if fills[b] != W - 1]
+    if fail_at == 1:                                    # nothing ran
+        assert (g == 12.5).all()
+        assert (to_np(fout) == -7).all()
+        return
+    for b in flushing:                                  # the flush ran; the decode did not
+        o = sess[b].flush(_one(inp, b))
+        assert vec_relerr(g[b:b + 1], o) <= TOL
+        assert head_relerr(to_np(layer.state)[b:b + 1], sess[b].S) <= TOL
+        assert int(fout[b].item()) == 0
+    for b in decoding:
+        assert (g[b] == 12.5).all()
+    # the plan is still usable: the decoding sequences step now, the flushed ones start a window
+    nf = torch.from_numpy(np.where(fills == W - 1, 0, fills)).cuda().to(torch.int32)
+    nout = torch.empty_like(nf)
+    inp2 = synth.step_inputs(wl, st, 1)
+    layer.step_mixed(layer.token(inp2), nf, nout)
+    torch.cuda.synchronize()
+    g2 = to_np(layer.out)
+    for b in range(batch):
+        o, _ = sess[b].decode(_one(inp2, b))
+        assert vec_relerr(g2[b:b + 1], o) <= TOL

@@ -72,16 +72,23 @@ def test_ragged_ranks_with_zero_and_one(cuda_ok, family):
 
 
 @pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
-def test_standard_exact_step(cuda_ok, family):
-    wl = small(FAM[family], 128, 64, seed=600)
+@pytest.mark.parametrize("dk,dv", [(128, 128), (128, 64), (64, 128), (64, 64)])
+def test_standard_exact_step(cuda_ok, family, dk, dv):
+    """The Standard baseline (paper App. D): every step reads and writes the
+    full state; output and state against the oracle's recurrence."""
+    wl = small(FAM[family], dk, dv, seed=600 + dk + dv)
     p = Pair(wl)
     for t in range(6):
         p.exact_step(synth.step_inputs(wl, p.st, t))
 
 
 @pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
-def test_replay_window(cuda_ok, family):
-    wl = small(FAM[family], 128, 128, window=8, seed=700)
+@pytest.mark.parametrize("dk,dv", [(128, 128), (128, 64), (64, 128), (64, 64)])
+def test_replay_window(cuda_ok, family, dk, dv):
+    """The ReplaySSM baseline (GitHub page "Overview"; paper App. D): exact
+    windowed reads of S0 and a flush without a sketch, over two windows and
+    a part of a third."""
+    wl = small(FAM[family], dk, dv, window=8, seed=700 + dk + dv)
     p = Pair(wl)
     for t in range(19):
         p.replay_step(synth.step_inputs(wl, p.st, t))
@@ -214,13 +221,17 @@ def test_full_size_sampled(cuda_ok, name, sketch):
     dt = B.SS_F32 if sketch == "f32" else B.SS_BF16
     p = Pair(wl, sketch_dtype=dt, sel=sel)
     p.prime()
-    for t in range(wl.window + 2):
+    # two full windows and two steps of a third: the second window's decodes
+    # read a sketch written by a full-size flush, and the second flush's state
+    # and sketch are compared again
+    for t in range(2 * wl.window + 2):
         p.step(synth.step_inputs(wl, p.st, t), ring=False)
     # properties that hold at any size: all outputs finite, ring slots hold the inputs
     g = to_np(p.layer.out)
     assert np.isfinite(g).all()
-    inp = synth.step_inputs(wl, p.st, wl.window + 1)
+    inp = synth.step_inputs(wl, p.st, 2 * wl.window + 1)
     assert np.array_equal(to_np(p.layer.ring_k)[:, :, 1], inp["k"])
+    assert p.worst["state"] <= TOL and p.worst["out"] <= TOL
 
 
 @pytest.mark.parametrize("batch,window,mean_rank", [(1, 4, 4), (32, 32, 16), (1024, 8, 8)])
