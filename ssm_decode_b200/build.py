@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsketchssm.so")
-SOURCES = ["ss_api.cu", "ss_flush.cu", "ss_flush_mma.cu", "ss_step.cu"]
+SOURCES = ["ss_api.cu", "ss_flush.cu", "ss_flush_mma.cu", "ss_flush_tc.cu", "ss_step.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

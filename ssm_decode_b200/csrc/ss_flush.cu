@@ -841,11 +841,13 @@ cudaError_t flush_t(const FlushParams& p, int rmax, cudaStream_t stream) {
 
 }  // namespace
 
-// Mamba-2 runs on the tensor-core kernel (ss_flush_mma.cu); GDN and KDA, and
-// every family when the flush also builds the state-dependent coefficient
-// map, on the CUDA-core kernel above.
+// Mamba-2 runs on the warp-MMA kernel (ss_flush_mma.cu); GDN and KDA with
+// dv = 128 and up to 16 updates on the tcgen05 kernel (ss_flush_tc.cu); the
+// other shapes, mixed-phase steps and every family when the flush also builds
+// the state-dependent coefficient map, on the CUDA-core kernel above.
 cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream) {
     if (family == MAMBA2 && !(p.cmap && p.do_sketch)) return launch_flush_mma(dk, dv, p, rmax, stream);
+    if (flush_tc_eligible(family, dk, dv, p, rmax)) return launch_flush_tc(family, dk, p, rmax, stream);
     SS_DISPATCH(flush_t, p, rmax, stream);
 }
 

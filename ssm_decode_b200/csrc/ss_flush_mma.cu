@@ -458,8 +458,8 @@ EncodeTiled tensor_map_encoder() {
 // Tensor map of the state viewed as (B*H*dk) rows of dv floats, boxes of
 // dk rows x 32 floats, 128-byte swizzle.  The last few encodings are cached
 // (the state buffer of a layer does not move between calls).
-cudaError_t state_tensor_map(const float* state, long long rows, int K, int V, CUtensorMap* out) {
-    struct Entry { int dev; const float* ptr; long long rows; int K, V; CUtensorMap map; };
+cudaError_t state_tensor_map(const float* state, long long rows, int K, int V, CUtensorMap* out, bool atom32) {
+    struct Entry { int dev; const float* ptr; long long rows; int K, V; bool atom32; CUtensorMap map; };
     static Entry cache[8];
     static int next = 0, used = 0;
     static std::mutex mu;
@@ -468,7 +468,10 @@ cudaError_t state_tensor_map(const float* state, long long rows, int K, int V, C
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i) {
         const Entry& e = cache[i];
-        if (e.dev == dev && e.ptr == state && e.rows == rows && e.K == K && e.V == V) { *out = e.map; return cudaSuccess; }
+        if (e.dev == dev && e.ptr == state && e.rows == rows && e.K == K && e.V == V && e.atom32 == atom32) {
+            *out = e.map;
+            return cudaSuccess;
+        }
     }
     EncodeTiled enc = tensor_map_encoder();
     if (enc == nullptr) return cudaErrorNotSupported;
@@ -478,10 +481,11 @@ cudaError_t state_tensor_map(const float* state, long long rows, int K, int V, C
     const cuuint32_t estr[2] = {1, 1};
     CUtensorMap m;
     const CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(state), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    cache[next] = Entry{dev, state, rows, K, V, m};
+    cache[next] = Entry{dev, state, rows, K, V, atom32, m};
     next = (next + 1) % 8;
     if (used < 8) ++used;
     *out = m;

@@ -95,6 +95,11 @@ cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int r
                          cudaStream_t stream);
 // Mamba-2 flush on the tensor cores (any dk, dv in {64, 128}).
 cudaError_t launch_flush_mma(int dk, int dv, const FlushParams& p, int rmax, cudaStream_t stream);
+// GDN / KDA flush on the fifth-generation tensor cores (dv = 128, dk in
+// {64, 128}, at most 16 updates and 32 read-out columns, uniform batch, fixed
+// coefficient map); flush_tc_eligible tells whether a launch qualifies.
+bool flush_tc_eligible(int family, int dk, int dv, const FlushParams& p, int rmax);
+cudaError_t launch_flush_tc(int family, int dk, const FlushParams& p, int rmax, cudaStream_t stream);
 // After a flush with a sketch: the dense-fallback heads' state copies.
 cudaError_t launch_dense_copy(int dk, int dv, const FlushParams& p, cudaStream_t stream);
 int flush_mma_smem_bytes(int dk, int dv, int n, int e16);

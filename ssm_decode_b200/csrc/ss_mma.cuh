@@ -51,8 +51,10 @@ __device__ __forceinline__ int tile_off(int row, int col) {
 }
 
 // Tensor map of the state viewed as (B*H*dk) rows of dv floats, boxes of
-// dk rows x 32 floats, 128-byte swizzle (host; cached per buffer).
-cudaError_t state_tensor_map(const float* state, long long rows, int K, int V, CUtensorMap* out);
+// dk rows x 32 floats, 128-byte swizzle of 16-byte chunks, or of 32-byte
+// chunks with atom32 (host; cached per buffer and swizzle).
+cudaError_t state_tensor_map(const float* state, long long rows, int K, int V, CUtensorMap* out,
+                             bool atom32 = false);
 
 // Issue (one thread) the dv/32 swizzled boxes of head u's state tile.
 template <int K, int V>
