@@ -15,53 +15,52 @@
 //     w_t = b_t (v_t - A(t,-1) y_t - sum_{j<t} A(t,j) (k_t . k_j) w_j).
 // KDA (S_t = (I - b_t k_t k_t^T) Diag(a_t) S_{t-1} + b_t k_t v_t^T) is the same
 // with per-channel products G(t,j) = a_{j+1} ⊙ ... ⊙ a_t: y_t = S_0^T (G(t,-1) ⊙ k_t),
-// pair weights sum_c k_t[c] k_j[c] G(t,j)[c] and S_W = Diag(G(n-1,-1)) S_0 +
-// sum_j (G(n-1,j) ⊙ k_j) w_j^T.  Every decay factor is a product of decays in
-// [0, 1]: nothing overflows and the window needs no renormalisation.
+// pair weights sum_c k_t[c] k_j[c] G(t,j)[c] = (G(t,-1) ⊙ k_t) . (k_j / G(j,-1))
+// and S_W = Diag(G(n-1,-1)) S_0 + sum_j (G(n-1,j) ⊙ k_j) w_j^T.  Every decay
+// factor is a product of decays in [0, 1]: nothing overflows and the window
+// needs no renormalisation (KDA heads whose products fall below 2^-100 take
+// their pair weights channel by channel instead of through k_j / G(j,-1)).
 //
 // Read-out without a second pass over the state.  With S_W = Diag(g) S_0 +
 // sum_j k^_j w~_j^T (g = A(n-1,-1) for GDN, G(n-1,-1) per channel for KDA; k^_j
 // the update keys, w~_j = w_j scaled by A(n-1,j) for GDN), for any probe x (a
 // basis vector omega_e or the query q):
-//     S_W^T x = S_0^T (g ⊙ x) + sum_j w~_j (k^_j . x).
-// One tensor-core pass over S_0 yields Y and S_0^T (g ⊙ x); the small products
-// k^_j . x run on the CUDA cores meanwhile and are added by a few more MMAs
-// (A = W~^T, already in TMEM for the update) onto the pass's output.
+//     S_W^T x = S_0^T (g ⊙ x) + sum_j w~_j (k^_j . x),
+// and for KDA k^_j . x = (k_j / G(j,-1)) . (g ⊙ x).
 //
-// Tensor-core products per head (tf32 operands, fp32 accumulators in TMEM,
-// M = dv = 128 on the TMEM lanes; lane v is state column v):
-//     D   = S_0^T [Y's keys | g ⊙ probes | their lo halves | (KDA) keys' lo]
-//                                                        N <= 96, K = dk
-//     D  += W~^T (K^ X^T) on the probe columns           N = 16 or 32, K = 16
-//     C  += W~^T K^   (C = Diag(g) S_0 before)           N = dk,  K = 16
-// An instruction costs about as much at N = 16 as at N = 128 (it is bound by
-// reading its 128 x 8 slice of A), so products sharing an A are packed along
-// N.  fp32 accuracy from tf32 operands: each fp32 operand is split x = hi + lo,
+// Tensor-core products per head (tf32 operands, fp32 accumulators in TMEM):
+//     Gm = [keys | probes] K'^T     M = 128 rows of the pass's B buffer, N = 16
+//          (GDN K' = the keys; KDA K' = k_j / G(j,-1), hi and lo: N = 32) --
+//          the pair weights and k^_j . x, for the recursion and the read-out
+//     D  = S_0^T [keys | probes | their lo halves]   M = dv, N <= 96, K = dk
+//     Dc = W~^T (K^ X^T)                              M = dv, N = 16 or 32, K = 16
+//     C += W~^T K^   (C = Diag(g) S_0 before)         M = dv, N = dk, K = 16
+// D, Dc and C have lane v = state column v; C ends as S_W^T.  An instruction
+// costs about as much at N = 16 as at N = 128 (it is bound by reading its
+// 128 x 8 slice of A), so products that share an A operand are packed along N.
+// fp32 accuracy from tf32 operands: each fp32 operand is split x = hi + lo,
 // hi = x with the low 13 mantissa bits cleared (the tensor core takes a tf32
 // operand from fp32 by this truncation, so a raw fp32 value serves as its own
 // hi half), lo = x - hi exactly; products are hi*hi + hi*lo + lo*hi, or
 // hi*b + lo*b when b is exact in tf32 (bf16 keys and queries).  Both halves of
-// S_0 live in TMEM (A operands); the B operands in 128-byte-swizzled shared
-// memory (K-major: 16-byte atoms; MN-major: 32-byte atoms, the only layout the
-// tensor core takes for MN-major tf32).
+// S_0 live in TMEM (A operands); B operands in 128-byte-swizzled shared memory
+// (K-major: 16-byte atoms; MN-major: 32-byte atoms, the only layout the tensor
+// core takes for MN-major tf32).
 //
-// The update accumulates onto C = Diag(g) S_0 (written by the workers from
-// S_0's TMEM copy), so C ends as S_W^T itself.
-//
-// Work split.  Persistent CTAs, one per SM, of 8 worker warps and a control
-// warp; CTA c walks heads c, c + grid, ...  Worker (v, half) owns state column
-// v and half of the dk rows; lane 0 of the control warp issues every bulk copy
-// and MMA, so no worker stalls while the tensor core drains its queue.  The
-// state tile arrives by bulk tensor copies; once it is split into TMEM (early
-// in the head) the tile buffer takes the next head's copy, which has the rest
-// of the head to arrive.  A head's S_W leaves by coalesced stores from
-// registers while the next head's pass runs on the tensor core, so the
-// workers' wait for the stores to drain overlaps the pass.  The window
-// (keys, values, decays, query, basis rows) arrives by bulk copies.  MMA
-// groups complete on mbarriers.  Every wait is bounded: when one runs out the
-// kernel sets SS_DEVICE_TIMEOUT in the caller's status word, waits (bounded)
-// for its own copies and MMAs in flight, releases its tensor memory and
-// returns.
+// Work split.  Persistent CTAs, one per SM, of 8 worker warps, an issuing warp
+// and a moving warp; CTA c walks heads c, c + grid, ...  Worker (v, half) owns
+// state column v and half of the dk rows.  Lane 0 of the issuing warp issues
+// the window copies and every MMA.  Lane 0 of the moving warp moves data in
+// and out with bulk copies, paced by mbarriers only (it takes part in no
+// barrier of the others): a head's tile is split into TMEM early in the head;
+// its buffer then stages the previous head's S_W (read from C), which the
+// mover stores before it loads the next head's tile into the same buffer; the
+// read-out is staged in shared memory and stored the same way.  No worker or
+// issuer waits for the tensor core's queue or for stores to drain.  MMA
+// groups complete on mbarriers.  Every wait on an mbarrier is bounded: when one runs
+// out the kernel sets SS_DEVICE_TIMEOUT in the caller's status word, waits
+// (bounded) for its own copies and MMAs in flight, releases its tensor memory
+// and returns.
 #include "ss_mma.cuh"
 #include "ss_tc.cuh"
 
@@ -70,15 +69,14 @@ namespace {
 
 constexpr int TV = 128;            // dv: state columns = TMEM lanes
 constexpr int NWK = 256;           // worker threads: two per state column
-constexpr int TT = NWK + 32;       // and the control warp
+constexpr int TT = NWK + 64;       // the issuing warp and the moving warp
 constexpr int NJ = 16;             // update slots per head (n <= 16)
 // Tensor-memory columns (all 512 allocated; one CTA per SM).
-constexpr uint32_t T_HI = 0;       // S_0 (its raw fp32 value, the hi half): dk columns
+constexpr uint32_t T_HI = 0;       // S_0 (its raw fp32 value, the hi half): dk columns; later Dc
 constexpr uint32_t T_LO = 128;     // lo half of S_0: dk columns
-constexpr uint32_t T_C = 256;      // the update's accumulator C: dk columns
+constexpr uint32_t T_C = 256;      // Diag(g) S_0 plus the update, i.e. S_W^T: dk columns
 constexpr uint32_t T_D = 384;      // the pass over S_0: up to 96 columns
-constexpr uint32_t T_WH = 480;     // hi half of W~^T: 16 columns
-constexpr uint32_t T_WL = 496;     // lo half of W~^T: 16 columns
+constexpr uint32_t T_W = 480;      // Gm (16 or 32 columns), then W~^T: hi 16, lo 16 columns
 constexpr uint32_t T_COLS = 512;
 // KDA heads whose running decay products fall below this take the pair
 // weights channel by channel instead of through k_j / G(j,-1).
@@ -100,10 +98,22 @@ __device__ __forceinline__ bool wsync_or(bool x) {
     return r != 0;
 }
 
-// Rows of the pass's B operand (K-major, 16-byte-atom swizzle, dk columns):
+// Barrier of the workers and the issuing warp (named barrier 2), returning
+// whether any of them passed `x` true.
+__device__ __forceinline__ bool csync_or(bool x) {
+    unsigned r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 2, 288, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"(unsigned(x))
+        : "memory");
+    return r != 0;
+}
+
+// Rows of the pass's B buffer (K-major, 16-byte-atom swizzle, dk columns):
 //   [0, 16)              Y's keys (KDA: hi half of G(t,-1) ⊙ k_t)
-//   [16, 16 + E)         g ⊙ probe e, hi halves: omega_e for e < r_h, q at
-//                        e = r_h (with a token), then zeros
+//   [16, 16 + E)         probe e, hi halves (GDN: x_e; KDA: g ⊙ x_e): omega_e
+//                        for e < r_h, q at e = r_h (with a token), then zeros
 //   [16 + E, 16 + 2E)    lo halves of the same rows
 //   [16 + 2E, 32 + 2E)   KDA only: lo half of Y's keys
 // E = 16 or 32 (read-out columns rounded up).  The pass with S_0's hi half
@@ -112,24 +122,22 @@ __host__ __device__ constexpr int pass_rows(int fam, int E) { return 16 + 2 * E 
 
 // Per-CTA shared-memory layout (byte offsets from a 1024-byte-aligned base).
 struct TcLayout {
-    int tile, bp, ku, ku2, kxh, kxl, kq, kp, xp, kraw, vraw, graw, braw, sg, sb, tq, tab, bars, total;
+    int tile, bp, ku, ku2, kq, kxh, kxl, part, ust, kraw, vraw, graw, braw, sg, sb, tq, tab, bars, total;
 };
 
-// Rows of the row-major buffers are padded by 16 bytes, so the rows that a
-// warp reads together start in different banks.
 __host__ __device__ inline TcLayout tc_layout(int fam, int K, int E) {
     const bool kda = fam == KDA;
     TcLayout L;
     int o = 0;
-    L.tile = o; o += K * TV * 4;                    // state tile (32-byte-atom swizzle)
-    L.bp = o;   o += pass_rows(fam, E) * K * 4;     // the pass's B operand
+    L.tile = o; o += K * TV * 4;                    // the state tile (32-byte-atom swizzle), then S_W
+    L.bp = o;   o += pass_rows(fam, E) * K * 4;     // the pass's B buffer
     L.ku = o;   o += NJ * K * 4;                    // update keys, MN-major (KDA: hi half)
     L.ku2 = o;  o += kda ? NJ * K * 4 : 0;          // KDA: their lo half
+    L.kq = o;   o += kda ? 2 * NJ * K * 4 : 0;      // KDA: k_j / G(j,-1), K-major, hi rows then lo rows
     L.kxh = o;  o += E * 128;                       // k^_j . x_e, K-major [e][j] (j < 32), hi half
     L.kxl = o;  o += E * 128;                       // and lo half
-    L.kq = o;   o += kda ? NJ * (K + 4) * 4 : 0;    // KDA: k_j / G(j,-1), rows padded by 16 bytes
-    L.kp = o;   o += kda ? NJ * (K + 4) * 4 : 0;    // KDA: update keys, rows padded
-    L.xp = o;   o += E * (K + 4) * 4;               // the probes unscaled, rows padded
+    L.part = o; o += (2 * NJ + 2 * E) * NJ * 4;     // pieces of the pair weights and of k^ . x
+    L.ust = o;  o += E * TV * 4 + TV * 4;           // the read-out staged: sketch rows, then o
     L.kraw = o; o += NJ * K * 2;
     L.vraw = o; o += NJ * TV * 2;
     L.graw = o; o += kda ? NJ * K * 4 : 0;
@@ -138,7 +146,7 @@ __host__ __device__ inline TcLayout tc_layout(int fam, int K, int E) {
     L.sb = o;   o += NJ * 4;
     L.tq = o;   o += align16(K * 2);
     L.tab = o;  o += (NJ * NJ + 6 * NJ + K) * 4;
-    L.bars = o; o += 64;
+    L.bars = o; o += 128;
     L.total = o + 1024;                             // room to align the base to 1024 bytes
     return L;
 }
@@ -203,16 +211,28 @@ __device__ __forceinline__ void tc_issue_window(const FlushParams& p, long long 
     if (r > 0) bulk_g2s(sm + L.braw, p.basis + (long long)p.off[u % p.H] * K, r * K * 4, bar);
 }
 
-// Four consecutive channels c .. c+3 (c % 4 == 0) of row `row` of a K-major
-// operand buffer with `rows` rows (16-byte-atom swizzle).
-__device__ __forceinline__ float4 ld_row4(const unsigned char* buf, int rows, int row, int c) {
-    return *reinterpret_cast<const float4*>(buf + tc::sw128_off(rows, row, c));
+// Bulk tensor store of one box of the state (32 columns x dk rows) from
+// shared memory (bulk async-group of the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
 }
-__device__ __forceinline__ float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// shared -> global (bulk async-group).
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, unsigned bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(smem_u32(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// The committed stores have finished reading shared memory / are complete.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
-__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
-    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
-}
+__device__ __forceinline__ float4 hi4(float4 x) { return make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w)); }
 
 template <int FAM, int K>
 __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__ FlushParams p,
@@ -220,22 +240,30 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     extern __shared__ __align__(16) unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const bool ctl = warp == NWK / 32;                                // the control warp
-    const bool issuer = ctl && lane == 0;
+    const bool ctl = warp == NWK / 32;                                // the issuing warp
+    const bool mov = warp == NWK / 32 + 1;                            // the moving warp
+    const bool issuer = ctl && lane == 0;                             // window copies and MMAs
+    const bool mover = mov && lane == 0;                              // bulk copies in and out
     const int v = t & (TV - 1);                                       // a worker's state column
     const int hk = (t >> 7) & 1;                                      // which half of the dk rows
     constexpr int KH = K / 2;
     const TcLayout L = tc_layout(FAM, K, E);
-    const int NB = pass_rows(FAM, E);                                 // rows of the pass's B operand
+    const int NB = pass_rows(FAM, E);                                 // rows of the pass's B buffer
+    const int NG = FAM == KDA ? 32 : 16;                              // columns of Gm
     const long long units = (long long)p.B * p.H;
     const int n = p.n_ring + p.has_token;
-    constexpr int KP = K + 4;                                         // padded row of the row-major buffers
-    uint64_t* tbar = reinterpret_cast<uint64_t*>(sm + L.bars);       // the tile
-    uint64_t* wbar = tbar + 1;                                       // the window
-    uint64_t* pbar = tbar + 2;                                       // MMA groups: the pass,
-    uint64_t* cbar = tbar + 3;                                       //   the read-out's correction,
-    uint64_t* ubar = tbar + 4;                                       //   the update
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tbar + 5);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
+    uint64_t* tbar = bars + 0;                                       // the tile
+    uint64_t* wbar = bars + 1;                                       // the window
+    uint64_t* gbar = bars + 2;                                       // MMA groups: Gm,
+    uint64_t* pbar = bars + 3;                                       //   the pass,
+    uint64_t* cbar = bars + 4;                                       //   the read-out's correction,
+    uint64_t* ubar = bars + 5;                                       //   the update
+    uint64_t* sbar = bars + 6;                                       // tile read, S_W staged (256 arrivals)
+    uint64_t* rbar = bars + 7;                                       // read-out staged (256 arrivals)
+    uint64_t* xbar = bars + 8;                                       // read-out staging free again (mover)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+    volatile int* slow_flag = reinterpret_cast<volatile int*>(bars + 10);
     const bool stall = p.stall && blockIdx.x == 0;
     Tab tab(sm + L.tab);
     unsigned char* const tile = sm + L.tile;
@@ -247,12 +275,16 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     const float* sg = reinterpret_cast<const float*>(sm + L.sg);
     const float* sb = reinterpret_cast<const float*>(sm + L.sb);
     const uint16_t* tq = reinterpret_cast<const uint16_t*>(sm + L.tq);
-    float* kq = reinterpret_cast<float*>(sm + L.kq);                 // KDA [NJ][KP]
-    float* kp = reinterpret_cast<float*>(sm + L.kp);                 // KDA [NJ][KP]
-    float* xp = reinterpret_cast<float*>(sm + L.xp);                 // [E][KP]
+    float* const pa = reinterpret_cast<float*>(sm + L.part);          // [NJ][NJ] from the keys' hi rows
+    float* const pb = pa + NJ * NJ;                                   // [NJ][NJ] KDA: from the keys' lo rows
+    float* const xa = pb + NJ * NJ;                                   // [E][NJ] from the probes' hi rows
+    float* const xb = xa + E * NJ;                                    // [E][NJ] from the probes' lo rows
 
     if (t == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(tbar + i, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+        mbar_init(sbar, NWK);
+        mbar_init(rbar, NWK);
+        mbar_init(xbar, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -267,31 +299,107 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     griddep_wait();                                                   // the previous kernel's writes are visible
     griddep_launch_next();
 
-    // in-flight copies and MMA groups: the issuer's (bit 0 tile, bit 1 window,
-    // bits 2, 3, 4: the pass, correction and update groups) and worker 0's
-    // (bit 1: a window it issued itself)
+    // Copies and MMA groups in flight, for the bounded waits before an early
+    // exit: the issuer's bit 1 (window) and bits 2..5 (the Gm, pass, correction
+    // and update groups); worker 0's bit 1 (a window it issued itself).  The
+    // mover keeps its own.
     unsigned pending = 0;
-    unsigned tph = 0, wph = 0, pph = 0, cph = 0, uph = 0;
-    long long u_prev = -1;                                            // the head whose S_W is still in C
+    unsigned tph = 0, wph = 0, gph = 0, pph = 0, cph = 0, uph = 0, sph = 0, rph = 0, xph = 0;
     long long u = blockIdx.x;
+    long long u_prev = -1;                                            // the head whose S_W is in C
     const long long stride = gridDim.x;
     if (issuer && u < units) {
-        issue_state_tile<K, TV>(&tmap, u, tile, tbar);
         tc_issue_window<FAM, K>(p, u, sm, L, wbar, stall ? 16u : 0u);
-        pending = 3u;
+        pending |= 2u;
     }
     const uint32_t s_bp = smem_u32(bp), s_ku = smem_u32(sm + L.ku), s_ku2 = smem_u32(sm + L.ku2);
-    const uint32_t s_kxh = smem_u32(sm + L.kxh), s_kxl = smem_u32(sm + L.kxl);
+    const uint32_t s_kq = smem_u32(sm + L.kq), s_kxh = smem_u32(sm + L.kxh), s_kxl = smem_u32(sm + L.kxl);
+
+    // Workers: S_W of head u_prev (in C) into the tile buffer for the mover
+    // (after the update of that head has completed); arrive on sbar when done.
+    auto stage_sw = [&]() -> bool {
+        const bool f = wsync_or(!mbar_wait(ubar, uph));
+        tc::fence_after();
+        if (f) return true;
+        unsigned char* colb = tile + (v >> 5) * (K * 128) + ((lane & 7) << 2);
+#pragma unroll 1
+        for (int k0 = 0; k0 < KH; k0 += 32) {
+            const int kb = hk * KH + k0;
+            uint32_t cr[2][16];
+            tc::ld16(tmem + lane_q + T_C + kb, cr[0]);
+            tc::ld16(tmem + lane_q + T_C + kb + 16, cr[1]);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int kk = kb + i;
+                *reinterpret_cast<uint32_t*>(colb + kk * 128 + (((lane >> 3) ^ (kk & 3)) << 5)) = cr[i >> 4][i & 15];
+            }
+        }
+        tc::fence_proxy_async();
+        mbar_arrive(sbar);
+        return false;
+    };
 
     bool ok = true;
+    if (mov) {
+        // ---- the moving warp: tiles in, S_W and read-outs out ------------------------------------
+        if (mover) {
+            long long up = -1;
+            bool tile_out = false;                                      // a tile copy in flight
+            if (u < units) {
+                issue_state_tile<K, TV>(&tmap, u, tile, tbar);
+                tile_out = true;
+            }
+            const size_t esz = p.sketch_bf16 ? 2 : 4;
+            for (; u < units; u += stride) {
+                // the workers have read this head's tile (and staged S_W of head up)
+                if (!mbar_wait(sbar, sph)) { ok = false; break; }
+                sph ^= 1u;
+                tph ^= 1u;
+                tile_out = false;
+                if (n > 0 && up >= 0) {
+#pragma unroll
+                    for (int bx = 0; bx < TV / 32; ++bx) tma_store_2d(&tmap, 32 * bx, int(up * K), tile + bx * K * 128);
+                    bulk_commit();
+                }
+                bulk_wait_read0();
+                if (u + stride < units) {
+                    issue_state_tile<K, TV>(&tmap, u + stride, tile, tbar);
+                    tile_out = true;
+                }
+                // this head's read-out, staged by the workers
+                if (!mbar_wait(rbar, rph)) { ok = false; break; }
+                rph ^= 1u;
+                const int r_h = tc_basis_rows(p, u);
+                if (r_h > 0) {
+                    const long long row0 = (u / p.H) * p.R + p.off[u % p.H];
+                    bulk_s2g(static_cast<unsigned char*>(p.sketch) + row0 * TV * esz, sm + L.ust, unsigned(r_h * TV * esz));
+                }
+                if (p.has_token) bulk_s2g(p.out + u * TV, sm + L.ust + E * TV * 4, TV * 4);
+                bulk_commit();
+                bulk_wait_read0();
+                mbar_arrive(xbar);
+                if (n > 0) up = u;
+            }
+            if (ok && n > 0 && up >= 0) {                               // the last head's S_W
+                if (mbar_wait(sbar, sph)) {
+#pragma unroll
+                    for (int bx = 0; bx < TV / 32; ++bx) tma_store_2d(&tmap, 32 * bx, int(up * K), tile + bx * K * 128);
+                    bulk_commit();
+                }
+            }
+            if (tile_out) mbar_wait(tbar, tph);                         // own copies: one more bounded wait
+            bulk_wait0();                                               // every store complete
+        }
+        u = units;                                                      // the loop below is not the mover's
+    }
     for (; u < units; u += stride) {
-        const int h = int(u % p.H);
-        const long long b = u / p.H;
         const int r_h = tc_basis_rows(p, u);
         const int ne = r_h + p.has_token;                              // read-out columns [Omega_h | q]
+        const bool more = u + stride < units;
         bool fail = false, slow = false;
-
         float vv[NJ];                                                   // the values of this column
+
         if (!ctl) {
             bool w_ok = mbar_wait(tbar, tph);
             w_ok = mbar_wait(wbar, wph) && w_ok;
@@ -299,7 +407,7 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             if (t == 0 && !fail) pending &= ~2u;
         }
         if (!ctl && !fail) {
-            // ---- phase 1a: S_0 into TMEM, keys, scalars -----------------------------------------
+            // ---- phase 1a: S_0 into TMEM, values, keys, scalars -----------------------------------
             {
                 // S_0's raw value (the hi half) and its lo half, this thread's column
                 // and half of the rows; the tile is in the 32-byte-atom swizzle, and
@@ -344,9 +452,10 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     *reinterpret_cast<float4*>(sm + L.ku + tc::sw32b_off(NJ, j, c)) = v4;
                 }
             } else if (t < K) {
-                // thread c: prefix products G(t,-1)[c] (Y's keys, k_j / G(j,-1) for the
-                // pair weights), suffix products G(n-1,j)[c] (the update's keys)
+                // thread c: prefix products G(t,-1)[c] (Y's keys, and k_j / G(j,-1) as Gm's
+                // B operand), suffix products G(n-1,j)[c] (the update's keys)
                 const int c = t;
+                unsigned char* kq = sm + L.kq;
                 float gam = 1.f;
                 for (int j = 0; j < NJ; ++j) {
                     float x = 0.f, xq = 0.f;
@@ -357,10 +466,11 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                         tiny |= !(gam >= KDA_GMIN);
                         xq = kv * __frcp_rn(gam);
                     }
-                    const float hi = tf32_hi(x);
+                    const float hi = tf32_hi(x), hq = tf32_hi(xq);
                     *reinterpret_cast<float*>(bp + tc::sw128_off(NB, j, c)) = hi;
                     *reinterpret_cast<float*>(bp + tc::sw128_off(NB, 16 + 2 * E + j, c)) = x - hi;
-                    kq[j * KP + c] = xq;
+                    *reinterpret_cast<float*>(kq + tc::sw128_off(2 * NJ, j, c)) = hq;
+                    *reinterpret_cast<float*>(kq + tc::sw128_off(2 * NJ, NJ + j, c)) = xq - hq;
                 }
                 tab.gw[c] = gam;
                 float suf = 1.f;
@@ -374,16 +484,10 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     const uint32_t o = tc::sw32b_off(NJ, j, c);
                     *reinterpret_cast<float*>(sm + L.ku + o) = hi;
                     *reinterpret_cast<float*>(sm + L.ku2 + o) = x - hi;
-                    kp[j * KP + c] = x;
                 }
             }
-            slow = wsync_or(tiny) && FAM == KDA;                        // the tables above are written
-            // ---- phase 1b: probes, unscaled (for k^ . x) and scaled by g (for the pass) -----------
-            float g1 = 1.f;
-            if (FAM == GDN) {
-#pragma unroll
-                for (int i = 0; i < NJ; ++i) g1 *= i < n ? tab.al[i] : 1.f;
-            }
+            slow = wsync_or(tiny) && FAM == KDA;                        // tab.gw is written
+            // ---- phase 1b: the probes (KDA: scaled by G(n-1,-1)), hi and lo halves ----------------
             for (int idx = t; idx < E * (K / 4); idx += NWK) {
                 const int e = idx / (K / 4), c = (idx % (K / 4)) * 4;
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -393,10 +497,8 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     const uint2 w = *reinterpret_cast<const uint2*>(tq + c);
                     x = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
                 }
-                *reinterpret_cast<float4*>(xp + e * KP + c) = x;
                 if (FAM == KDA) x = mul4(x, *reinterpret_cast<const float4*>(tab.gw + c));
-                else x = make_float4(g1 * x.x, g1 * x.y, g1 * x.z, g1 * x.w);
-                const float4 hi = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+                const float4 hi = hi4(x);
                 *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, 16 + e, c)) = hi;
                 *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, 16 + E + e, c)) =
                     make_float4(x.x - hi.x, x.y - hi.y, x.z - hi.z, x.w - hi.w);
@@ -405,27 +507,34 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             tc::fence_proxy_async();
         }
         tc::fence_before();
-        // (1) operands written, tile read; KDA's slow flag is worker 0's to pass on
-        if (t == 0) reinterpret_cast<volatile int*>(tmem_slot)[1] = slow ? 1 : 0;
-        if (__syncthreads_or(fail)) { ok = false; break; }
+        if (t == 0) *slow_flag = slow ? 1 : 0;
+        if (csync_or(fail)) { ok = false; break; }                      // (1) operands written, tile read
         tph ^= 1u;
         wph ^= 1u;
-        slow = FAM == KDA && reinterpret_cast<volatile int*>(tmem_slot)[1] != 0;
+        slow = FAM == KDA && *slow_flag != 0;
 
         if (ctl) {
             if (issuer) {
                 tc::fence_after();
-                pending &= ~3u;
-                // the tile buffer is free: the next head's tile; the window buffers
-                // too, unless KDA's slow pair weights still read the raw keys and decays
-                if (u + stride < units) {
-                    issue_state_tile<K, TV>(&tmap, u + stride, tile, tbar);
-                    pending |= 1u;
-                    if (!slow) {
-                        tc_issue_window<FAM, K>(p, u + stride, sm, L, wbar, 0u);
-                        pending |= 2u;
+                pending &= ~2u;
+                if (more && !slow) {                                    // the window buffers are free
+                    tc_issue_window<FAM, K>(p, u + stride, sm, L, wbar, 0u);
+                    pending |= 2u;
+                }
+                // Gm = [keys | probes] K'^T: the pass buffer's rows against the keys
+                if (!slow && n > 0) {
+                    const uint32_t id_g = tc::idesc_tf32(128, NG, 0, 0);
+                    const uint32_t s_b = FAM == KDA ? s_kq : s_bp;
+                    const int brows = FAM == KDA ? 2 * NJ : NB;
+#pragma unroll 1
+                    for (int q = 0; q < K / 8; ++q) {
+                        const uint32_t ko = (q & 3) * 32;
+                        const uint64_t a = tc::sdesc(s_bp + (q >> 2) * (NB * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
+                        const uint64_t bk = tc::sdesc(s_b + (q >> 2) * (brows * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
+                        tc::mma_ss(tmem + T_W, a, bk, id_g, q > 0);
                     }
                 }
+                tc::commit(gbar);
                 // D = S_0^T [keys | probes]: the hi half against every row, the lo half against the first 16 + E
                 const uint32_t id_hi = tc::idesc_tf32(TV, NB, 0, 0), id_lo = tc::idesc_tf32(TV, 16 + E, 0, 0);
 #pragma unroll 1
@@ -435,133 +544,28 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     tc::mma_ts(tmem + T_D, tmem + T_LO + 8 * q, bd, id_lo, 1);
                 }
                 tc::commit(pbar);
-                pending |= 4u;
+                pending |= 4u | 8u;
             }
             __syncwarp();
         } else {
-            // ---- phase 2 (beside the pass): pair sums, k^_j . x_e, the recursion's tables -----------
-            {
-                // pair sums for j < t, two threads per pair (half the channels each)
-                const int pair = t >> 1, part = t & 1;
-                int tt = 1, rem = pair;
-                while (rem >= tt && tt < NJ) { rem -= tt; ++tt; }
-                const int j = rem;
-                const bool act = pair < n * (n - 1) / 2 && !slow;
-                float acc = 0.f;
-                if (act) {
-#pragma unroll 4
-                    for (int c = part * KH; c < (part + 1) * KH; c += 4) {
-                        if (FAM == KDA) {
-                            const float4 x = add4(ld_row4(bp, NB, tt, c), ld_row4(bp, NB, 16 + 2 * E + tt, c));
-                            acc = dot4(x, *reinterpret_cast<const float4*>(kq + j * KP + c), acc);
-                        } else {
-                            acc = dot4(ld_row4(bp, NB, tt, c), ld_row4(bp, NB, j, c), acc);
-                        }
-                    }
-                }
-                acc += __shfl_xor_sync(FULL, acc, 1);
-                if (act && part == 0) tab.P[tt * NJ + j] = acc;        // times b_t below
-            }
-            if (FAM == KDA && slow) {
-                // channel by channel, with the ratio G(t,j)[c] as a running product:
-                // thread (j = t / 16, group cg = t % 16) over dk / 16 channels
-                const int j = t >> 4, cg = t & 15;
-                constexpr int CPG = K / 16;
-                float acc[NJ];
-#pragma unroll
-                for (int q = 0; q < NJ; ++q) acc[q] = 0.f;
-                if (j < n) {
-                    for (int ci = 0; ci < CPG; ++ci) {
-                        const int c = cg * CPG + ci;
-                        const float kj = bf2f(kraw[j * K + c]);
-                        float r = 1.f;
-#pragma unroll
-                        for (int q = 1; q < NJ; ++q) {
-                            if (q > j && q < n) {
-                                r *= graw[q * K + c];
-                                acc[q] = fmaf(kj * bf2f(kraw[q * K + c]), r, acc[q]);
-                            }
-                        }
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < NJ; ++q) {
-                    float x = acc[q];
-                    x += __shfl_xor_sync(FULL, x, 1);
-                    x += __shfl_xor_sync(FULL, x, 2);
-                    x += __shfl_xor_sync(FULL, x, 4);
-                    x += __shfl_xor_sync(FULL, x, 8);
-                    acc[q] = x;
-                }
-                if (cg == 0 && j < n) {
-#pragma unroll
-                    for (int q = 0; q < NJ; ++q)
-                        if (q > j && q < n) tab.P[q * NJ + j] = acc[q];
-                }
-            }
-            // k^_j . x_e (unscaled probes): thread (j = t / 16, e = t % 16, and e + 16),
-            // split into hi and lo halves as the B operand of the correction MMAs
-            {
-                const int j = t >> 4, e0 = t & 15;
-                const float* krow = FAM == KDA ? kp + j * KP : nullptr;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int e = e0 + 16 * half;
-                    if (e >= E) break;
-                    float acc0 = 0.f, acc1 = 0.f;
-                    if (j < n && e < ne) {
-                        const float* xrow = xp + e * KP;
-#pragma unroll 4
-                        for (int c = 0; c < K; c += 8) {
-                            float4 k0, k1;
-                            if (FAM == KDA) {
-                                k0 = *reinterpret_cast<const float4*>(krow + c);
-                                k1 = *reinterpret_cast<const float4*>(krow + c + 4);
-                            } else {
-                                k0 = ld_row4(bp, NB, j, c);
-                                k1 = ld_row4(bp, NB, j, c + 4);
-                            }
-                            acc0 = dot4(k0, *reinterpret_cast<const float4*>(xrow + c), acc0);
-                            acc1 = dot4(k1, *reinterpret_cast<const float4*>(xrow + c + 4), acc1);
-                        }
-                    }
-                    const float x = acc0 + acc1;
-                    const float hi = tf32_hi(x);
-                    *reinterpret_cast<float*>(sm + L.kxh + tc::sw128_off(E, e, j)) = hi;
-                    *reinterpret_cast<float*>(sm + L.kxl + tc::sw128_off(E, e, j)) = x - hi;
-                }
-            }
-            tc::fence_proxy_async();
+            // ---- phase 2 (beside Gm and the pass) ----------------------------------------------
             if (n > 0) {
-                // the previous head's S_W (in C) to global memory, then C = Diag(g) S_0
-                // for this head; this thread's column and half of the rows
-                if (u_prev >= 0) {
-                    fail = wsync_or(!mbar_wait(ubar, uph));
-                    tc::fence_after();
-                }
+                // the previous head's S_W (in C) to the tile buffer, then C = Diag(g) S_0
+                if (u_prev >= 0) fail = stage_sw();
+                else mbar_arrive(sbar);                                 // the tile is read
                 if (!fail) {
                     float g1 = 1.f;
                     if (FAM == GDN) {
 #pragma unroll
                         for (int i = 0; i < NJ; ++i) g1 *= i < n ? tab.al[i] : 1.f;
                     }
-                    float* dst = p.state + u_prev * (long long)(K * TV) + v;
 #pragma unroll 1
                     for (int k0 = 0; k0 < KH; k0 += 32) {
                         const int kb = hk * KH + k0;
-                        uint32_t cr[2][16], sh[2][16];
-                        if (u_prev >= 0) {
-                            tc::ld16(tmem + lane_q + T_C + kb, cr[0]);
-                            tc::ld16(tmem + lane_q + T_C + kb + 16, cr[1]);
-                        }
+                        uint32_t sh[2][16];
                         tc::ld16(tmem + lane_q + T_HI + kb, sh[0]);
                         tc::ld16(tmem + lane_q + T_HI + kb + 16, sh[1]);
                         tc::wait_ld();
-                        if (u_prev >= 0) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                __stcs(dst + (long long)(kb + i) * TV, __uint_as_float(cr[i >> 4][i & 15]));
-                        }
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
                             const float dec = FAM == KDA ? tab.gw[kb + i] : g1;
@@ -572,19 +576,106 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     }
                     tc::wait_st();
                 }
+                // Gm's pieces to shared memory: row r of the pass buffer is TMEM lane r,
+                // read by the workers of the first half (one lane quarter per warp)
+                if (!fail) fail = wsync_or(!mbar_wait(gbar, gph));
+                tc::fence_after();
+                if (!fail && !slow && hk == 0) {
+                    const int r = v;                                    // TMEM lane = B-buffer row
+                    uint32_t g0[16], g1r[16];
+                    tc::ld16(tmem + lane_q + T_W, g0);
+                    if (FAM == KDA) tc::ld16(tmem + lane_q + T_W + 16, g1r);
+                    tc::wait_ld();
+                    float* dst = nullptr;
+                    bool both = FAM == KDA;                             // add the K' lo columns
+                    if (r < 16) dst = pa + r * NJ;
+                    else if (r < 16 + E) dst = xa + (r - 16) * NJ;
+                    else if (r < 16 + 2 * E) { dst = xb + (r - 16 - E) * NJ; both = false; }
+                    else if (FAM == KDA && r < 32 + 2 * E) { dst = pb + (r - 16 - 2 * E) * NJ; both = false; }
+                    if (dst != nullptr) {
+#pragma unroll
+                        for (int j = 0; j < NJ; ++j)
+                            dst[j] = __uint_as_float(g0[j]) + (both ? __uint_as_float(g1r[j]) : 0.f);
+                    }
+                }
+                if (FAM == KDA && slow && !fail) {
+                    // channel by channel: pair weights with the ratio G(t,j)[c] as a
+                    // running product (thread (j = t / 16, group cg = t % 16)), and
+                    // k^_j . x_e from the update keys and the unscaled probes
+                    const int j = t >> 4, cg = t & 15;
+                    constexpr int CPG = K / 16;
+                    float acc[NJ];
+#pragma unroll
+                    for (int q = 0; q < NJ; ++q) acc[q] = 0.f;
+                    if (j < n) {
+                        for (int ci = 0; ci < CPG; ++ci) {
+                            const int c = cg * CPG + ci;
+                            const float kj = bf2f(kraw[j * K + c]);
+                            float r = 1.f;
+#pragma unroll
+                            for (int q = 1; q < NJ; ++q) {
+                                if (q > j && q < n) {
+                                    r *= graw[q * K + c];
+                                    acc[q] = fmaf(kj * bf2f(kraw[q * K + c]), r, acc[q]);
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < NJ; ++q) {
+                        float x = acc[q];
+                        x += __shfl_xor_sync(FULL, x, 1);
+                        x += __shfl_xor_sync(FULL, x, 2);
+                        x += __shfl_xor_sync(FULL, x, 4);
+                        x += __shfl_xor_sync(FULL, x, 8);
+                        acc[q] = x;
+                    }
+                    if (cg == 0) {
+#pragma unroll
+                        for (int q = 0; q < NJ; ++q) {
+                            pa[q * NJ + j] = acc[q];
+                            pb[q * NJ + j] = 0.f;
+                        }
+                    }
+                    for (int idx = t; idx < E * NJ; idx += NWK) {
+                        const int e = idx / NJ, jj = idx % NJ;
+                        float s = 0.f;
+                        if (jj < n && e < ne) {
+                            for (int c = 0; c < K; ++c) {
+                                const uint32_t o = tc::sw32b_off(NJ, jj, c);
+                                const float kk = *reinterpret_cast<const float*>(sm + L.ku + o) +
+                                                 *reinterpret_cast<const float*>(sm + L.ku2 + o);
+                                const float x = e < r_h ? braw[e * K + c] : bf2f(tq[c]);
+                                s = fmaf(kk, x, s);
+                            }
+                        }
+                        xa[idx] = s;
+                        xb[idx] = 0.f;
+                    }
+                }
             }
-            wsync();                                                    // (2) raw pair sums
-            if (t == 0 && slow && u + stride < units) {                 // KDA slow path: the window now
+            if (n == 0) mbar_arrive(sbar);                              // the tile is read
+            wsync();                                                    // (2) Gm's pieces
+            if (t == 0 && slow && more) {                               // KDA slow path: the window now
                 tc_issue_window<FAM, K>(p, u + stride, sm, L, wbar, 0u);
                 pending |= 2u;
             }
+            // k^_j . x_e as the correction's B operand (K-major [e][j]), hi and lo
+            for (int idx = t; idx < E * NJ; idx += NWK) {
+                const int e = idx / NJ, j = idx % NJ;
+                const float x = (j < n && e < ne) ? xa[idx] + xb[idx] : 0.f;
+                const float hi = tf32_hi(x);
+                *reinterpret_cast<float*>(sm + L.kxh + tc::sw128_off(E, e, j)) = hi;
+                *reinterpret_cast<float*>(sm + L.kxl + tc::sw128_off(E, e, j)) = x - hi;
+            }
+            tc::fence_proxy_async();
             if (t < NJ) {
                 const int tt = t;
                 float al[NJ], pr[NJ];
 #pragma unroll
                 for (int i = 0; i < NJ; ++i) {
                     al[i] = tab.al[i];
-                    pr[i] = tab.P[tt * NJ + i];
+                    pr[i] = pa[tt * NJ + i] + (FAM == KDA ? pb[tt * NJ + i] : 0.f);
                 }
                 const float cbt = tab.cb[tt];
                 if (FAM == GDN) {
@@ -609,11 +700,8 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     tab.cy[tt] = tt < n ? cbt : 0.f;
                     tab.g[tt] = tt < n ? 1.f : 0.f;
                 }
-                if (tt < n) {
 #pragma unroll
-                    for (int j = 0; j < NJ - 1; ++j)
-                        if (j < tt) tab.P[tt * NJ + j] = pr[j];
-                }
+                for (int j = 0; j < NJ; ++j) tab.P[tt * NJ + j] = (j < tt && tt < n) ? pr[j] : 0.f;
             }
             wsync();                                                    // (3) tables
 
@@ -651,29 +739,30 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     wh[j] = __float_as_uint(hi);
                     wl[j] = __float_as_uint(x - hi);
                 }
-                tc::st16(tmem + lane_q + T_WH, wh);
-                tc::st16(tmem + lane_q + T_WL, wl);
+                tc::st16(tmem + lane_q + T_W, wh);
+                tc::st16(tmem + lane_q + T_W + 16, wl);
                 tc::wait_st();
             }
         }
         tc::fence_before();
-        if (__syncthreads_or(fail)) { ok = false; break; }              // (4) W~ and k^.x ready
+        if (csync_or(fail)) { ok = false; break; }                      // (4) W~ and k^.x ready
+        gph ^= 1u;
         pph ^= 1u;
         if (n > 0 && u_prev >= 0) uph ^= 1u;
         if (issuer) {
-            pending &= ~(4u | 16u);
+            pending &= ~(4u | 8u | 32u);
             tc::fence_after();
-            // the probes' correction D[:, 16 ..] += W~^T (K^ X^T), then C += W~^T K^;
-            // each group completes on its own mbarrier (committed even when empty)
+            // Dc = W~^T (K^ X^T) into the first E columns of the (now free) S_0
+            // region, then C += W~^T K^; each group completes on its own mbarrier
             const int nq = (n + 7) / 8;
             if (n > 0 && ne > 0) {
                 const uint32_t id_x = tc::idesc_tf32(TV, E, 0, 0);
                 for (int q = 0; q < nq; ++q) {
                     const uint64_t xh = tc::sdesc(s_kxh + q * 32, 16, 1024, tc::LAYOUT_SW128);
                     const uint64_t xl = tc::sdesc(s_kxl + q * 32, 16, 1024, tc::LAYOUT_SW128);
-                    tc::mma_ts(tmem + T_D + 16, tmem + T_WH + 8 * q, xh, id_x, 1);
-                    tc::mma_ts(tmem + T_D + 16, tmem + T_WH + 8 * q, xl, id_x, 1);
-                    tc::mma_ts(tmem + T_D + 16, tmem + T_WL + 8 * q, xh, id_x, 1);
+                    tc::mma_ts(tmem + T_HI, tmem + T_W + 8 * q, xh, id_x, q > 0);
+                    tc::mma_ts(tmem + T_HI, tmem + T_W + 8 * q, xl, id_x, 1);
+                    tc::mma_ts(tmem + T_HI, tmem + T_W + 16 + 8 * q, xh, id_x, 1);
                 }
             }
             tc::commit(cbar);
@@ -681,80 +770,76 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                 const uint32_t id_u = tc::idesc_tf32(TV, K, 0, 1);
                 for (int q = 0; q < nq; ++q) {
                     const uint64_t bh = tc::sdesc(s_ku + q * 1024, NJ * 128, 512, tc::LAYOUT_SW128_32B);
-                    tc::mma_ts(tmem + T_C, tmem + T_WH + 8 * q, bh, id_u, 1);
-                    tc::mma_ts(tmem + T_C, tmem + T_WL + 8 * q, bh, id_u, 1);
+                    tc::mma_ts(tmem + T_C, tmem + T_W + 8 * q, bh, id_u, 1);
+                    tc::mma_ts(tmem + T_C, tmem + T_W + 16 + 8 * q, bh, id_u, 1);
                     if (FAM == KDA)
-                        tc::mma_ts(tmem + T_C, tmem + T_WH + 8 * q,
+                        tc::mma_ts(tmem + T_C, tmem + T_W + 8 * q,
                                    tc::sdesc(s_ku2 + q * 1024, NJ * 128, 512, tc::LAYOUT_SW128_32B), id_u, 1);
                 }
                 tc::commit(ubar);
-                pending |= 16u;
+                pending |= 32u;
             }
-            pending |= 8u;
+            pending |= 16u;
         }
         if (!ctl) {
             fail = wsync_or(!mbar_wait(cbar, cph));
             tc::fence_after();
-            // ---- read-out: S_W^T x_e = (D_hi + D_lo)[e]; this thread's half of the columns -----
+            // the staging buffer is free once the mover has stored the previous read-out
+            if (!fail && u != (long long)blockIdx.x) fail = wsync_or(!mbar_wait(xbar, xph));
+            // ---- read-out: S_W^T x_e = g (D_hi + D_lo)[e] + Dc[e]; this thread's half of the columns
             const int e0 = 16 * hk;
             if (!fail && e0 < ne) {
-                uint32_t dh[16], dl[16];
+                float g1 = 1.f;
+                if (FAM == GDN) {
+#pragma unroll
+                    for (int i = 0; i < NJ; ++i) g1 *= i < n ? tab.al[i] : 1.f;
+                }
+                uint32_t dh[16], dl[16], dc[16];
                 tc::ld16(tmem + lane_q + T_D + 16 + e0, dh);
                 tc::ld16(tmem + lane_q + T_D + 16 + E + e0, dl);
+                if (n > 0) tc::ld16(tmem + lane_q + T_HI + e0, dc);
                 tc::wait_ld();
-                const long long row0 = b * p.R + p.off[h];
+                unsigned char* ust = sm + L.ust;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int e = e0 + i;
                     if (e < ne) {
-                        const float x = __uint_as_float(dh[i]) + __uint_as_float(dl[i]);
+                        float x = g1 * (__uint_as_float(dh[i]) + __uint_as_float(dl[i]));
+                        if (n > 0) x += __uint_as_float(dc[i]);
                         if (e < r_h) {
-                            const long long o = (row0 + e) * TV + v;
-                            if (p.sketch_bf16) static_cast<uint16_t*>(p.sketch)[o] = f2bf(x);
-                            else static_cast<float*>(p.sketch)[o] = x;
+                            if (p.sketch_bf16) reinterpret_cast<uint16_t*>(ust)[e * TV + v] = f2bf(x);
+                            else reinterpret_cast<float*>(ust)[e * TV + v] = x;
                         } else {
-                            p.out[u * TV + v] = x;
+                            reinterpret_cast<float*>(ust + E * TV * 4)[v] = x;
                         }
                     }
                 }
             }
+            tc::fence_proxy_async();
+            if (!fail) mbar_arrive(rbar);
         }
         cph ^= 1u;
         tc::fence_before();
-        if (__syncthreads_or(fail)) { ok = false; break; }              // (5) TMEM, tables and buffers read
-        if (issuer) pending &= ~8u;
+        if (csync_or(fail)) { ok = false; break; }                      // (5) TMEM, tables and buffers read
+        if (u != (long long)blockIdx.x) xph ^= 1u;
+        if (issuer) pending &= ~16u;
         if (n > 0) u_prev = u;
     }
-    // the last head's S_W
-    if (ok && n > 0 && u_prev >= 0) {
+    // the last head's S_W: staged by the workers, stored by the mover
+    if (!mov && ok && n > 0 && u_prev >= 0) {
         bool f = false;
-        if (!ctl) {
-            f = wsync_or(!mbar_wait(ubar, uph));
-            tc::fence_after();
-            if (!f) {
-                float* dst = p.state + u_prev * (long long)(K * TV) + v;
-#pragma unroll 1
-                for (int k0 = 0; k0 < KH; k0 += 16) {
-                    const int kb = hk * KH + k0;
-                    uint32_t cr[16];
-                    tc::ld16(tmem + lane_q + T_C + kb, cr);
-                    tc::wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) __stcs(dst + (long long)(kb + i) * TV, __uint_as_float(cr[i]));
-                }
-            }
-        }
-        if (__syncthreads_or(f)) ok = false;
-        else if (issuer) pending &= ~16u;
+        if (!ctl) f = stage_sw();
+        if (csync_or(f)) ok = false;
+        else if (issuer) pending &= ~32u;
     }
     if (!ok && (issuer || t == 0)) {
         // a bounded wait ran out: report it, then wait (bounded) for this
         // thread's copies and MMAs still in flight before the memory is released
         if (issuer) report_timeout(p.status);
-        if (pending & 4u) mbar_wait(pbar, pph);
-        if (pending & 8u) mbar_wait(cbar, cph);
-        if (pending & 16u) mbar_wait(ubar, uph);
-        if (pending & 1u) mbar_wait(tbar, tph);
+        if (pending & 4u) mbar_wait(gbar, gph);
+        if (pending & 8u) mbar_wait(pbar, pph);
+        if (pending & 16u) mbar_wait(cbar, cph);
+        if (pending & 32u) mbar_wait(ubar, uph);
         if (pending & 2u) mbar_wait(wbar, wph);
     }
     tc::fence_before();
