@@ -122,7 +122,7 @@ __host__ __device__ constexpr int pass_rows(int fam, int E) { return 16 + 2 * E 
 
 // Per-CTA shared-memory layout (byte offsets from a 1024-byte-aligned base).
 struct TcLayout {
-    int tile, bp, ku, ku2, kq, kxh, kxl, part, ust, kraw, vraw, graw, braw, sg, sb, tq, tab, bars, total;
+    int tile, bp, ku[2], ku2[2], kq, kxh, kxl, part, ust, kraw, vraw, graw, braw, sg, sb, tq, tab, bars, total;
 };
 
 __host__ __device__ inline TcLayout tc_layout(int fam, int K, int E) {
@@ -131,8 +131,12 @@ __host__ __device__ inline TcLayout tc_layout(int fam, int K, int E) {
     int o = 0;
     L.tile = o; o += K * TV * 4;                    // the state tile (32-byte-atom swizzle), then S_W
     L.bp = o;   o += pass_rows(fam, E) * K * 4;     // the pass's B buffer
-    L.ku = o;   o += NJ * K * 4;                    // update keys, MN-major (KDA: hi half)
-    L.ku2 = o;  o += kda ? NJ * K * 4 : 0;          // KDA: their lo half
+    for (int i = 0; i < 2; ++i) {                   // update keys, MN-major (KDA: hi half), by head parity
+        L.ku[i] = o; o += NJ * K * 4;
+    }
+    for (int i = 0; i < 2; ++i) {                   // KDA: their lo half
+        L.ku2[i] = o; o += kda ? NJ * K * 4 : 0;
+    }
     L.kq = o;   o += kda ? 2 * NJ * K * 4 : 0;      // KDA: k_j / G(j,-1), K-major, hi rows then lo rows
     L.kxh = o;  o += E * 128;                       // k^_j . x_e, K-major [e][j] (j < 32), hi half
     L.kxl = o;  o += E * 128;                       // and lo half
@@ -155,7 +159,8 @@ __host__ __device__ inline TcLayout tc_layout(int fam, int K, int E) {
 // cy[t] (weight of y_t), cb[t] = b_t, g[j] (GDN: A(n-1, j); KDA: 1), al[t] (GDN
 // decays), gw[k] (KDA: G(n-1,-1)[k]).
 struct Tab {
-    float *P, *cy, *cb, *g, *al, *gw;
+    float *P, *cy, *cb, *g, *al, *tok, *gw;
+    int* hr;
     __device__ explicit Tab(unsigned char* base) {
         float* f = reinterpret_cast<float*>(base);
         P = f;
@@ -163,14 +168,19 @@ struct Tab {
         cb = cy + NJ;
         g = cb + NJ;
         al = g + NJ;
+        tok = al + NJ;                                              // the next head's token b_t, a_t
+        hr = reinterpret_cast<int*>(tok + 2);                       // basis rows of the head, by parity
         gw = al + 2 * NJ;
     }
 };
 
-// Basis rows of unit u's head that its flush reads.
+// Basis rows of unit u's head that its flush reads, and the first of them.
 __device__ __forceinline__ int tc_basis_rows(const FlushParams& p, long long u) {
     const int h = int(u % p.H);
     return p.do_sketch && !head_dense(p.dense, h) ? p.off[h + 1] - p.off[h] : 0;
+}
+__device__ __forceinline__ int2 tc_head_rows(const FlushParams& p, long long u) {
+    return make_int2(tc_basis_rows(p, u), p.off[u % p.H]);
 }
 
 // Bytes of one head's window copies.
@@ -186,12 +196,16 @@ __device__ __forceinline__ unsigned tc_window_bytes(const FlushParams& p, int r)
     return b;
 }
 
-// One thread: the bulk copies of head u's window.  `extra` bytes more than the
-// copies deliver are expected (testing hook: the wait then runs out).
+// One thread: the bulk copies of head u's window, whose basis rows hr =
+// {count, first row} are given; the count is also written to *r_out for the
+// threads that wait on `bar`.  `extra` bytes more than the copies deliver are
+// expected (testing hook: the wait then runs out).
 template <int FAM, int K>
 __device__ __forceinline__ void tc_issue_window(const FlushParams& p, long long u, unsigned char* sm,
-                                                const TcLayout& L, uint64_t* bar, unsigned extra) {
-    const int r = tc_basis_rows(p, u);
+                                                const TcLayout& L, uint64_t* bar, unsigned extra, int2 hr,
+                                                int* r_out) {
+    const int r = hr.x;
+    *r_out = r;
     mbar_expect_tx(bar, tc_window_bytes<FAM, K>(p, r) + extra);
     const long long row = u * p.W;
     const int nr = p.n_ring, n4r = (nr + 3) & ~3;
@@ -208,7 +222,7 @@ __device__ __forceinline__ void tc_issue_window(const FlushParams& p, long long 
         if (FAM == KDA) bulk_g2s(sm + L.graw + nr * K * 4, p.tok_gate + u * K, K * 4, bar);
         bulk_g2s(sm + L.tq, p.tok_q + u * K, K * 2, bar);
     }
-    if (r > 0) bulk_g2s(sm + L.braw, p.basis + (long long)p.off[u % p.H] * K, r * K * 4, bar);
+    if (r > 0) bulk_g2s(sm + L.braw, p.basis + (long long)hr.y * K, r * K * 4, bar);
 }
 
 // Bulk tensor store of one box of the state (32 columns x dk rows) from
@@ -233,6 +247,55 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
 __device__ __forceinline__ float4 hi4(float4 x) { return make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w)); }
+
+// KDA, phase 1x: thread (c, HALF) takes slots j of its half of the window.
+// Prefix products G(j,-1)[c] give Y's keys (hi and lo rows of the pass's B
+// buffer) and k_j / G(j,-1) (Gm's B operand, hi and lo); suffix products
+// G(n-1,j)[c] the update's keys (MN-major, hi and lo).  Every load is issued
+// before the products.  Returns whether a prefix product fell below KDA_GMIN.
+template <int K, int HALF>
+__device__ __forceinline__ bool kda_keys(int c, int n, int E, int NB, const uint16_t* kraw, const float* graw,
+                                         unsigned char* bp, unsigned char* kq, unsigned char* kub,
+                                         unsigned char* kub2, float* gw) {
+    constexpr int J0 = HALF * (NJ / 2);
+    float ga[NJ], kk[NJ / 2];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) ga[j] = j < n ? graw[j * K + c] : 1.f;
+#pragma unroll
+    for (int i = 0; i < NJ / 2; ++i) kk[i] = J0 + i < n ? bf2f(kraw[(J0 + i) * K + c]) : 0.f;
+    float gam = 1.f, suf = 1.f;
+#pragma unroll
+    for (int j = 0; j < J0; ++j) gam *= ga[j];
+#pragma unroll
+    for (int j = J0 + NJ / 2; j < NJ; ++j) suf *= ga[j];
+    bool tiny = false;
+#pragma unroll
+    for (int i = 0; i < NJ / 2; ++i) {
+        const int j = J0 + i;
+        gam *= ga[j];
+        const bool live = j < n;
+        const float x = live ? gam * kk[i] : 0.f;
+        const float xq = live ? __fdividef(kk[i], gam) : 0.f;
+        tiny |= live && !(gam >= KDA_GMIN);
+        const float hi = tf32_hi(x), hq = tf32_hi(xq);
+        *reinterpret_cast<float*>(bp + tc::sw128_off(NB, j, c)) = hi;
+        *reinterpret_cast<float*>(bp + tc::sw128_off(NB, 16 + 2 * E + j, c)) = x - hi;
+        *reinterpret_cast<float*>(kq + tc::sw128_off(2 * NJ, j, c)) = hq;
+        *reinterpret_cast<float*>(kq + tc::sw128_off(2 * NJ, NJ + j, c)) = xq - hq;
+    }
+    if (HALF == 1) gw[c] = gam;
+#pragma unroll
+    for (int i = NJ / 2 - 1; i >= 0; --i) {
+        const int j = J0 + i;
+        const float x = j < n ? suf * kk[i] : 0.f;
+        suf *= ga[j];
+        const float hi = tf32_hi(x);
+        const uint32_t o = tc::sw32b_off(NJ, j, c);
+        *reinterpret_cast<float*>(kub + o) = hi;
+        *reinterpret_cast<float*>(kub2 + o) = x - hi;
+    }
+    return tiny;
+}
 
 template <int FAM, int K>
 __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__ FlushParams p,
@@ -259,11 +322,12 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     uint64_t* pbar = bars + 3;                                       //   the pass,
     uint64_t* cbar = bars + 4;                                       //   the read-out's correction,
     uint64_t* ubar = bars + 5;                                       //   the update
-    uint64_t* sbar = bars + 6;                                       // tile read, S_W staged (256 arrivals)
+    uint64_t* sbar = bars + 6;                                       // tile read and S_W staged (256 arrivals)
     uint64_t* rbar = bars + 7;                                       // read-out staged (256 arrivals)
-    uint64_t* xbar = bars + 8;                                       // read-out staging free again (mover)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
-    volatile int* slow_flag = reinterpret_cast<volatile int*>(bars + 10);
+    uint64_t* ebar = bars + 10;                                      // the mover's stores have read the staging buffers
+    uint64_t* xbar = bars + 11;                                      // phase 1 has read the window buffers
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+    volatile int* slow_flag = reinterpret_cast<volatile int*>(bars + 9);
     const bool stall = p.stall && blockIdx.x == 0;
     Tab tab(sm + L.tab);
     unsigned char* const tile = sm + L.tile;
@@ -279,11 +343,13 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     float* const pb = pa + NJ * NJ;                                   // [NJ][NJ] KDA: from the keys' lo rows
     float* const xa = pb + NJ * NJ;                                   // [E][NJ] from the probes' hi rows
     float* const xb = xa + E * NJ;                                    // [E][NJ] from the probes' lo rows
+    const size_t esz = p.sketch_bf16 ? 2 : 4;
 
     if (t == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
         mbar_init(sbar, NWK);
         mbar_init(rbar, NWK);
+        mbar_init(ebar, 1);
         mbar_init(xbar, 1);
         fence_mbar_init();
     }
@@ -299,24 +365,18 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     griddep_wait();                                                   // the previous kernel's writes are visible
     griddep_launch_next();
 
-    // Copies and MMA groups in flight, for the bounded waits before an early
-    // exit: the issuer's bit 1 (window) and bits 2..5 (the Gm, pass, correction
-    // and update groups); worker 0's bit 1 (a window it issued itself).  The
-    // mover keeps its own.
+    // MMA groups in flight, for the issuer's bounded waits before an early
+    // exit: bits 2..5 (the Gm, pass, correction and update groups).  The
+    // mover keeps its own copies.
     unsigned pending = 0;
-    unsigned tph = 0, wph = 0, gph = 0, pph = 0, cph = 0, uph = 0, sph = 0, rph = 0, xph = 0;
+    unsigned tph = 0, wph = 0, gph = 0, pph = 0, cph = 0, uph = 0, sph = 0, rph = 0, eph = 0;
     long long u = blockIdx.x;
-    long long u_prev = -1;                                            // the head whose S_W is in C
     const long long stride = gridDim.x;
-    if (issuer && u < units) {
-        tc_issue_window<FAM, K>(p, u, sm, L, wbar, stall ? 16u : 0u);
-        pending |= 2u;
-    }
-    const uint32_t s_bp = smem_u32(bp), s_ku = smem_u32(sm + L.ku), s_ku2 = smem_u32(sm + L.ku2);
-    const uint32_t s_kq = smem_u32(sm + L.kq), s_kxh = smem_u32(sm + L.kxh), s_kxl = smem_u32(sm + L.kxl);
+    const uint32_t s_bp = smem_u32(bp), s_kq = smem_u32(sm + L.kq);
+    const uint32_t s_kxh = smem_u32(sm + L.kxh), s_kxl = smem_u32(sm + L.kxl);
 
-    // Workers: S_W of head u_prev (in C) into the tile buffer for the mover
-    // (after the update of that head has completed); arrive on sbar when done.
+    // Workers: S_W of head `up` (in C) into the tile buffer for the mover,
+    // once the update of that head has completed; arrive on sbar when done.
     auto stage_sw = [&]() -> bool {
         const bool f = wsync_or(!mbar_wait(ubar, uph));
         tc::fence_after();
@@ -339,20 +399,104 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
         mbar_arrive(sbar);
         return false;
     };
+    // Workers: the read-out of a head, once its correction has completed:
+    // S_W^T x_e = g (D_hi + D_lo)[e] + Dc[e], staged in shared memory for the
+    // mover; this thread's half of the columns.  Arrives on rbar.
+    auto readout = [&](int ne_p, int r_p, float g_p) -> bool {
+        // the correction is done, and the mover has read the previous read-out
+        // out of the staging buffer (one arrival per mover iteration)
+        const bool f = wsync_or(!mbar_wait(cbar, cph) || !mbar_wait(ebar, eph));
+        eph ^= 1u;
+        tc::fence_after();
+        if (f) return true;
+        const int e0 = 16 * hk;
+        if (e0 < ne_p) {
+            uint32_t dh[16], dl[16], dc[16];
+            tc::ld16(tmem + lane_q + T_D + 16 + e0, dh);
+            tc::ld16(tmem + lane_q + T_D + 16 + E + e0, dl);
+            if (n > 0) tc::ld16(tmem + lane_q + T_HI + e0, dc);
+            tc::wait_ld();
+            unsigned char* ust = sm + L.ust;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int e = e0 + i;
+                if (e < ne_p) {
+                    float x = g_p * (__uint_as_float(dh[i]) + __uint_as_float(dl[i]));
+                    if (n > 0) x += __uint_as_float(dc[i]);
+                    if (e < r_p) {
+                        if (p.sketch_bf16) reinterpret_cast<uint16_t*>(ust)[e * TV + v] = f2bf(x);
+                        else reinterpret_cast<float*>(ust)[e * TV + v] = x;
+                    } else {
+                        reinterpret_cast<float*>(ust + E * TV * 4)[v] = x;
+                    }
+                }
+            }
+        }
+        tc::fence_proxy_async();
+        mbar_arrive(rbar);
+        return false;
+    };
 
     bool ok = true;
     if (mov) {
-        // ---- the moving warp: tiles in, S_W and read-outs out ------------------------------------
+        // ---- the moving warp: windows and tiles in; read-outs and S_W out ----------------------------
+        // Per head k: once phase 1 of head k has read the window buffers, head
+        // k+1's window; the read-out of head k-1 (staged early in head k), then
+        // S_W of head k-1 (staged in the tile buffer once head k's tile is in
+        // TMEM); once both stores have read shared memory, head k+1's tile.  The
+        // scalars each copy needs (basis rows, token b_t and a_t) are fetched a
+        // head ahead into registers.
         if (mover) {
             long long up = -1;
             bool tile_out = false;                                      // a tile copy in flight
+            long long nwin = 0;                                         // windows issued
+            int2 h_prev = make_int2(0, 0), h_cur = make_int2(0, 0), h_next = make_int2(0, 0);
+            float tb_next = 0.f, tg_next = 1.f;
+            auto fetch = [&](long long uu) {
+                h_next = tc_head_rows(p, uu);
+                if (p.has_token) {
+                    tb_next = p.tok_beta[uu];
+                    if (FAM == GDN) tg_next = p.tok_gate[uu];
+                }
+            };
+            // the next head's window: its token scalars and basis rows go to
+            // shared memory before the copies (the window's barrier publishes them)
+            auto issue_window = [&](long long uu, long long j, unsigned extra) {
+                tab.tok[0] = tb_next;
+                tab.tok[1] = tg_next;
+                tc_issue_window<FAM, K>(p, uu, sm, L, wbar, extra, h_next, tab.hr + (j & 1));
+                ++nwin;
+            };
             if (u < units) {
                 issue_state_tile<K, TV>(&tmap, u, tile, tbar);
                 tile_out = true;
+                fetch(u);
+                issue_window(u, 0, stall ? 16u : 0u);
+                h_cur = h_next;
+                if (u + stride < units) fetch(u + stride);
             }
-            const size_t esz = p.sketch_bf16 ? 2 : 4;
-            for (; u < units; u += stride) {
-                // the workers have read this head's tile (and staged S_W of head up)
+            auto store_readout = [&](long long uu, int2 hr) {
+                if (hr.x > 0) {
+                    const long long row0 = (uu / p.H) * p.R + hr.y;
+                    bulk_s2g(static_cast<unsigned char*>(p.sketch) + row0 * TV * esz, sm + L.ust, unsigned(hr.x * TV * esz));
+                }
+                if (p.has_token) bulk_s2g(p.out + uu * TV, sm + L.ust + E * TV * 4, TV * 4);
+                bulk_commit();
+            };
+            unsigned xph = 0;
+            for (long long k = 0; u < units; u += stride, ++k) {
+                if (!mbar_wait(xbar, xph)) { ok = false; break; }       // the window buffers are free
+                xph ^= 1u;
+                const int2 h1 = h_next;                                 // head k+1's basis rows
+                if (u + stride < units) {
+                    issue_window(u + stride, k + 1, 0u);
+                    if (u + 2 * stride < units) fetch(u + 2 * stride);
+                }
+                if (up >= 0) {
+                    if (!mbar_wait(rbar, rph)) { ok = false; break; }
+                    rph ^= 1u;
+                    store_readout(up, h_prev);
+                }
                 if (!mbar_wait(sbar, sph)) { ok = false; break; }
                 sph ^= 1u;
                 tph ^= 1u;
@@ -363,52 +507,143 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     bulk_commit();
                 }
                 bulk_wait_read0();
+                mbar_arrive(ebar);                                      // the staging buffers are free
                 if (u + stride < units) {
                     issue_state_tile<K, TV>(&tmap, u + stride, tile, tbar);
                     tile_out = true;
                 }
-                // this head's read-out, staged by the workers
-                if (!mbar_wait(rbar, rph)) { ok = false; break; }
-                rph ^= 1u;
-                const int r_h = tc_basis_rows(p, u);
-                if (r_h > 0) {
-                    const long long row0 = (u / p.H) * p.R + p.off[u % p.H];
-                    bulk_s2g(static_cast<unsigned char*>(p.sketch) + row0 * TV * esz, sm + L.ust, unsigned(r_h * TV * esz));
-                }
-                if (p.has_token) bulk_s2g(p.out + u * TV, sm + L.ust + E * TV * 4, TV * 4);
-                bulk_commit();
-                bulk_wait_read0();
-                mbar_arrive(xbar);
-                if (n > 0) up = u;
+                up = u;
+                h_prev = h_cur;
+                h_cur = h1;
             }
-            if (ok && n > 0 && up >= 0) {                               // the last head's S_W
-                if (mbar_wait(sbar, sph)) {
+            if (ok && up >= 0) {                                        // the last head's read-out and S_W
+                if (mbar_wait(rbar, rph)) {
+                    store_readout(up, h_prev);
+                    if (n > 0 && mbar_wait(sbar, sph)) {
 #pragma unroll
-                    for (int bx = 0; bx < TV / 32; ++bx) tma_store_2d(&tmap, 32 * bx, int(up * K), tile + bx * K * 128);
-                    bulk_commit();
+                        for (int bx = 0; bx < TV / 32; ++bx) tma_store_2d(&tmap, 32 * bx, int(up * K), tile + bx * K * 128);
+                        bulk_commit();
+                    }
                 }
             }
-            if (tile_out) mbar_wait(tbar, tph);                         // own copies: one more bounded wait
+            // own copies: one more bounded wait each
+            if (tile_out) mbar_wait(tbar, tph);
+            if (nwin > 0) mbar_wait(wbar, unsigned((nwin - 1) & 1));
             bulk_wait0();                                               // every store complete
         }
         u = units;                                                      // the loop below is not the mover's
     }
-    for (; u < units; u += stride) {
-        const int r_h = tc_basis_rows(p, u);
-        const int ne = r_h + p.has_token;                              // read-out columns [Omega_h | q]
-        const bool more = u + stride < units;
+
+    // the previous head, whose read-out and S_W are finished during this one
+    long long u_prev = -1;
+    int ne_prev = 0, r_prev = 0;
+    float g_prev = 1.f;
+    for (int k = 0; u < units; u += stride, ++k) {
+        int r_h = 0, ne = 0;                                            // basis rows; read-out columns [Omega_h | q]
+        unsigned char* const kub = sm + L.ku[0] + (k & 1) * (NJ * K * 4);            // this head's update keys
+        unsigned char* const kub2 = sm + L.ku2[0] + (k & 1) * (FAM == KDA ? NJ * K * 4 : 0);
         bool fail = false, slow = false;
-        float vv[NJ];                                                   // the values of this column
+        uint32_t vv[NJ / 2];                                            // this column's values, bf16 pairs
+        float g1 = 1.f;                                                 // GDN: A(n-1,-1)
 
         if (!ctl) {
-            bool w_ok = mbar_wait(tbar, tph);
-            w_ok = mbar_wait(wbar, wph) && w_ok;
-            fail = wsync_or(!w_ok);                                     // the same verdict for every worker
-            if (t == 0 && !fail) pending &= ~2u;
+            fail = wsync_or(!mbar_wait(wbar, wph));                     // the same verdict for every worker
+            r_h = tab.hr[k & 1];                                        // written before the window was issued
         }
         if (!ctl && !fail) {
-            // ---- phase 1a: S_0 into TMEM, values, keys, scalars -----------------------------------
-            {
+            // ---- phase 1x: values, scalars, keys, probes (the window buffers) ----------------------
+#pragma unroll
+            for (int j = 0; j < NJ / 2; ++j) {
+                const uint32_t a = (hk == 0 && 2 * j < n) ? vraw[2 * j * TV + v] : 0u;
+                const uint32_t b = (hk == 0 && 2 * j + 1 < n) ? vraw[(2 * j + 1) * TV + v] : 0u;
+                vv[j] = a | (b << 16);
+            }
+            if (t < NJ) {                                               // b_t and the GDN decays
+                float a = 1.f, bt = 0.f;
+                if (t < n) {
+                    const bool tok = t >= p.n_ring;
+                    bt = tok ? tab.tok[0] : sb[t];
+                    if (FAM == GDN) a = tok ? tab.tok[1] : sg[t];
+                }
+                tab.al[t] = a;
+                tab.cb[t] = bt;
+            }
+            bool tiny = false;
+            if constexpr (FAM == GDN) {
+                for (int i = t; i < NJ * (K / 4); i += NWK) {
+                    const int j = i / (K / 4), c = (i % (K / 4)) * 4;
+                    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (j < n) {
+                        const uint2 w = *reinterpret_cast<const uint2*>(kraw + j * K + c);
+                        v4 = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
+                    }
+                    *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, j, c)) = v4;
+                    *reinterpret_cast<float4*>(kub + tc::sw32b_off(NJ, j, c)) = v4;
+                }
+            } else if (t < 2 * K) {
+                if (t < K) tiny = kda_keys<K, 0>(t, n, E, NB, kraw, graw, bp, sm + L.kq, kub, kub2, tab.gw);
+                else tiny = kda_keys<K, 1>(t - K, n, E, NB, kraw, graw, bp, sm + L.kq, kub, kub2, tab.gw);
+            }
+            slow = wsync_or(tiny) && FAM == KDA;                        // tab.gw is written
+            // the probes (KDA: scaled by G(n-1,-1)), hi and lo halves
+            for (int idx = t; idx < E * (K / 4); idx += NWK) {
+                const int e = idx / (K / 4), c = (idx % (K / 4)) * 4;
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (e < r_h) {
+                    x = *reinterpret_cast<const float4*>(braw + e * K + c);
+                } else if (e == r_h && p.has_token) {
+                    const uint2 w = *reinterpret_cast<const uint2*>(tq + c);
+                    x = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
+                }
+                if (FAM == KDA) x = mul4(x, *reinterpret_cast<const float4*>(tab.gw + c));
+                const float4 hi = hi4(x);
+                *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, 16 + e, c)) = hi;
+                *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, 16 + E + e, c)) =
+                    make_float4(x.x - hi.x, x.y - hi.y, x.z - hi.z, x.w - hi.w);
+            }
+            if (FAM == GDN) {
+#pragma unroll
+                for (int i = 0; i < NJ; ++i) g1 *= i < n ? tab.al[i] : 1.f;
+            }
+            tc::fence_proxy_async();
+        }
+        if (t == 0) *slow_flag = slow ? 1 : 0;
+        if (csync_or(fail)) { ok = false; break; }                      // (1) operands in shared memory
+        wph ^= 1u;
+        r_h = tab.hr[k & 1];
+        ne = r_h + p.has_token;
+        slow = FAM == KDA && *slow_flag != 0;
+
+        if (ctl) {
+            if (issuer) {
+                if (!slow) mbar_arrive(xbar);                           // the window buffers are free
+                // the previous head's MMAs have finished reading W~ and the B buffers
+                if (u_prev >= 0 && n > 0 && !mbar_wait(ubar, uph)) fail = true;
+                tc::fence_after();
+                // Gm = [keys | probes] K'^T: the pass buffer's rows against the keys
+                if (!fail && !slow && n > 0) {
+                    const uint32_t id_g = tc::idesc_tf32(128, NG, 0, 0);
+                    const uint32_t s_b = FAM == KDA ? s_kq : s_bp;
+                    const int brows = FAM == KDA ? 2 * NJ : NB;
+#pragma unroll 1
+                    for (int q = 0; q < K / 8; ++q) {
+                        const uint32_t ko = (q & 3) * 32;
+                        const uint64_t a = tc::sdesc(s_bp + (q >> 2) * (NB * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
+                        const uint64_t bk = tc::sdesc(s_b + (q >> 2) * (brows * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
+                        tc::mma_ss(tmem + T_W, a, bk, id_g, q > 0);
+                    }
+                }
+                tc::commit(gbar);
+                pending |= 4u;
+            }
+            __syncwarp();
+        } else {
+            // the previous head's read-out (its correction ran during phase 1x)
+            if (u_prev >= 0) fail = readout(ne_prev, r_prev, g_prev);
+            // the tile; the barrier also orders the TMEM Dc reads before S_0 lands there
+            fail = wsync_or(fail || !mbar_wait(tbar, tph));
+            // ---- phase 1y: S_0 into TMEM (beside Gm) ---------------------------------------------------
+            if (!fail) {
                 // S_0's raw value (the hi half) and its lo half, this thread's column
                 // and half of the rows; the tile is in the 32-byte-atom swizzle, and
                 // a warp reads one 128-byte row at a time, conflict-free
@@ -426,115 +661,18 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     tc::st16(tmem + lane_q + T_HI + hk * KH + k0, hi);
                     tc::st16(tmem + lane_q + T_LO + hk * KH + k0, lo);
                 }
+                tc::wait_st();
             }
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) vv[j] = (hk == 0 && j < n) ? bf2f(vraw[j * TV + v]) : 0.f;
-            if (t < NJ) {                                               // b_t and the GDN decays
-                float a = 1.f, bt = 0.f;
-                if (t < n) {
-                    const bool tok = t >= p.n_ring;
-                    bt = tok ? p.tok_beta[u] : sb[t];
-                    if (FAM == GDN) a = tok ? p.tok_gate[u] : sg[t];
-                }
-                tab.al[t] = a;
-                tab.cb[t] = bt;
-            }
-            bool tiny = false;
-            if constexpr (FAM == GDN) {
-                for (int i = t; i < NJ * (K / 4); i += NWK) {
-                    const int j = i / (K / 4), c = (i % (K / 4)) * 4;
-                    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (j < n) {
-                        const uint2 w = *reinterpret_cast<const uint2*>(kraw + j * K + c);
-                        v4 = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
-                    }
-                    *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, j, c)) = v4;
-                    *reinterpret_cast<float4*>(sm + L.ku + tc::sw32b_off(NJ, j, c)) = v4;
-                }
-            } else if (t < K) {
-                // thread c: prefix products G(t,-1)[c] (Y's keys, and k_j / G(j,-1) as Gm's
-                // B operand), suffix products G(n-1,j)[c] (the update's keys)
-                const int c = t;
-                unsigned char* kq = sm + L.kq;
-                float gam = 1.f;
-                for (int j = 0; j < NJ; ++j) {
-                    float x = 0.f, xq = 0.f;
-                    if (j < n) {
-                        gam *= graw[j * K + c];
-                        const float kv = bf2f(kraw[j * K + c]);
-                        x = gam * kv;
-                        tiny |= !(gam >= KDA_GMIN);
-                        xq = kv * __frcp_rn(gam);
-                    }
-                    const float hi = tf32_hi(x), hq = tf32_hi(xq);
-                    *reinterpret_cast<float*>(bp + tc::sw128_off(NB, j, c)) = hi;
-                    *reinterpret_cast<float*>(bp + tc::sw128_off(NB, 16 + 2 * E + j, c)) = x - hi;
-                    *reinterpret_cast<float*>(kq + tc::sw128_off(2 * NJ, j, c)) = hq;
-                    *reinterpret_cast<float*>(kq + tc::sw128_off(2 * NJ, NJ + j, c)) = xq - hq;
-                }
-                tab.gw[c] = gam;
-                float suf = 1.f;
-                for (int j = NJ - 1; j >= 0; --j) {
-                    float x = 0.f;
-                    if (j < n) {
-                        x = suf * bf2f(kraw[j * K + c]);
-                        suf *= graw[j * K + c];
-                    }
-                    const float hi = tf32_hi(x);
-                    const uint32_t o = tc::sw32b_off(NJ, j, c);
-                    *reinterpret_cast<float*>(sm + L.ku + o) = hi;
-                    *reinterpret_cast<float*>(sm + L.ku2 + o) = x - hi;
-                }
-            }
-            slow = wsync_or(tiny) && FAM == KDA;                        // tab.gw is written
-            // ---- phase 1b: the probes (KDA: scaled by G(n-1,-1)), hi and lo halves ----------------
-            for (int idx = t; idx < E * (K / 4); idx += NWK) {
-                const int e = idx / (K / 4), c = (idx % (K / 4)) * 4;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (e < r_h) {
-                    x = *reinterpret_cast<const float4*>(braw + e * K + c);
-                } else if (e == r_h && p.has_token) {
-                    const uint2 w = *reinterpret_cast<const uint2*>(tq + c);
-                    x = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
-                }
-                if (FAM == KDA) x = mul4(x, *reinterpret_cast<const float4*>(tab.gw + c));
-                const float4 hi = hi4(x);
-                *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, 16 + e, c)) = hi;
-                *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, 16 + E + e, c)) =
-                    make_float4(x.x - hi.x, x.y - hi.y, x.z - hi.z, x.w - hi.w);
-            }
-            tc::wait_st();
-            tc::fence_proxy_async();
         }
         tc::fence_before();
-        if (t == 0) *slow_flag = slow ? 1 : 0;
-        if (csync_or(fail)) { ok = false; break; }                      // (1) operands written, tile read
+        if (csync_or(fail)) { ok = false; break; }                      // (2) S_0 in TMEM, tile read
         tph ^= 1u;
-        wph ^= 1u;
-        slow = FAM == KDA && *slow_flag != 0;
+        if (u_prev >= 0) cph ^= 1u;
+        if (issuer && u_prev >= 0) pending &= ~(16u | 32u);
 
         if (ctl) {
             if (issuer) {
                 tc::fence_after();
-                pending &= ~2u;
-                if (more && !slow) {                                    // the window buffers are free
-                    tc_issue_window<FAM, K>(p, u + stride, sm, L, wbar, 0u);
-                    pending |= 2u;
-                }
-                // Gm = [keys | probes] K'^T: the pass buffer's rows against the keys
-                if (!slow && n > 0) {
-                    const uint32_t id_g = tc::idesc_tf32(128, NG, 0, 0);
-                    const uint32_t s_b = FAM == KDA ? s_kq : s_bp;
-                    const int brows = FAM == KDA ? 2 * NJ : NB;
-#pragma unroll 1
-                    for (int q = 0; q < K / 8; ++q) {
-                        const uint32_t ko = (q & 3) * 32;
-                        const uint64_t a = tc::sdesc(s_bp + (q >> 2) * (NB * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
-                        const uint64_t bk = tc::sdesc(s_b + (q >> 2) * (brows * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
-                        tc::mma_ss(tmem + T_W, a, bk, id_g, q > 0);
-                    }
-                }
-                tc::commit(gbar);
                 // D = S_0^T [keys | probes]: the hi half against every row, the lo half against the first 16 + E
                 const uint32_t id_hi = tc::idesc_tf32(TV, NB, 0, 0), id_lo = tc::idesc_tf32(TV, 16 + E, 0, 0);
 #pragma unroll 1
@@ -544,21 +682,16 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     tc::mma_ts(tmem + T_D, tmem + T_LO + 8 * q, bd, id_lo, 1);
                 }
                 tc::commit(pbar);
-                pending |= 4u | 8u;
+                pending |= 8u;
             }
             __syncwarp();
         } else {
-            // ---- phase 2 (beside Gm and the pass) ----------------------------------------------
+            // ---- phase 2 (beside the pass) -----------------------------------------------------------
             if (n > 0) {
                 // the previous head's S_W (in C) to the tile buffer, then C = Diag(g) S_0
                 if (u_prev >= 0) fail = stage_sw();
                 else mbar_arrive(sbar);                                 // the tile is read
                 if (!fail) {
-                    float g1 = 1.f;
-                    if (FAM == GDN) {
-#pragma unroll
-                        for (int i = 0; i < NJ; ++i) g1 *= i < n ? tab.al[i] : 1.f;
-                    }
 #pragma unroll 1
                     for (int k0 = 0; k0 < KH; k0 += 32) {
                         const int kb = hk * KH + k0;
@@ -643,8 +776,8 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                         if (jj < n && e < ne) {
                             for (int c = 0; c < K; ++c) {
                                 const uint32_t o = tc::sw32b_off(NJ, jj, c);
-                                const float kk = *reinterpret_cast<const float*>(sm + L.ku + o) +
-                                                 *reinterpret_cast<const float*>(sm + L.ku2 + o);
+                                const float kk = *reinterpret_cast<const float*>(kub + o) +
+                                                 *reinterpret_cast<const float*>(kub2 + o);
                                 const float x = e < r_h ? braw[e * K + c] : bf2f(tq[c]);
                                 s = fmaf(kk, x, s);
                             }
@@ -653,13 +786,11 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                         xb[idx] = 0.f;
                     }
                 }
+            } else {
+                mbar_arrive(sbar);                                      // the tile is read
             }
-            if (n == 0) mbar_arrive(sbar);                              // the tile is read
-            wsync();                                                    // (2) Gm's pieces
-            if (t == 0 && slow && more) {                               // KDA slow path: the window now
-                tc_issue_window<FAM, K>(p, u + stride, sm, L, wbar, 0u);
-                pending |= 2u;
-            }
+            wsync();                                                    // (3) Gm's pieces
+            if (t == 0 && slow) mbar_arrive(xbar);                      // KDA slow path: the window buffers are free now
             // k^_j . x_e as the correction's B operand (K-major [e][j]), hi and lo
             for (int idx = t; idx < E * NJ; idx += NWK) {
                 const int e = idx / NJ, j = idx % NJ;
@@ -703,7 +834,7 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
 #pragma unroll
                 for (int j = 0; j < NJ; ++j) tab.P[tt * NJ + j] = (j < tt && tt < n) ? pr[j] : 0.f;
             }
-            wsync();                                                    // (3) tables
+            wsync();                                                    // (4) tables
 
             // ---- the pass is done: Y -> w (recursion), W~ into TMEM ----------------------------
             if (!fail) fail = wsync_or(!mbar_wait(pbar, pph));
@@ -726,7 +857,8 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                 float w[NJ];
 #pragma unroll
                 for (int tt = 0; tt < NJ; ++tt) {
-                    float x = tab.cb[tt] * vv[tt] - tab.cy[tt] * y[tt];
+                    const float vt = (tt & 1) ? bf2f_hi(vv[tt >> 1]) : bf2f_lo(vv[tt >> 1]);
+                    float x = tab.cb[tt] * vt - tab.cy[tt] * y[tt];
 #pragma unroll
                     for (int j = 0; j < tt; ++j) x = fmaf(-tab.P[tt * NJ + j], w[j], x);
                     w[tt] = tt < n ? x : 0.f;
@@ -745,15 +877,16 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             }
         }
         tc::fence_before();
-        if (csync_or(fail)) { ok = false; break; }                      // (4) W~ and k^.x ready
+        if (csync_or(fail)) { ok = false; break; }                      // (5) W~ and k^.x ready
         gph ^= 1u;
         pph ^= 1u;
-        if (n > 0 && u_prev >= 0) uph ^= 1u;
+        if (u_prev >= 0 && n > 0) uph ^= 1u;                            // the previous update, waited above
         if (issuer) {
-            pending &= ~(4u | 8u | 32u);
+            pending &= ~(4u | 8u);
             tc::fence_after();
-            // Dc = W~^T (K^ X^T) into the first E columns of the (now free) S_0
-            // region, then C += W~^T K^; each group completes on its own mbarrier
+            // Dc = W~^T (K^ X^T) into the first E columns of the S_0 region (read by the
+            // next head's workers before its S_0 lands there), then C += W~^T K^; each
+            // group completes on its own mbarrier (committed even when empty)
             const int nq = (n + 7) / 8;
             if (n > 0 && ne > 0) {
                 const uint32_t id_x = tc::idesc_tf32(TV, E, 0, 0);
@@ -768,6 +901,7 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             tc::commit(cbar);
             if (n > 0) {
                 const uint32_t id_u = tc::idesc_tf32(TV, K, 0, 1);
+                const uint32_t s_ku = smem_u32(kub), s_ku2 = smem_u32(kub2);
                 for (int q = 0; q < nq; ++q) {
                     const uint64_t bh = tc::sdesc(s_ku + q * 1024, NJ * 128, 512, tc::LAYOUT_SW128_32B);
                     tc::mma_ts(tmem + T_C, tmem + T_W + 8 * q, bh, id_u, 1);
@@ -781,58 +915,22 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             }
             pending |= 16u;
         }
-        if (!ctl) {
-            fail = wsync_or(!mbar_wait(cbar, cph));
-            tc::fence_after();
-            // the staging buffer is free once the mover has stored the previous read-out
-            if (!fail && u != (long long)blockIdx.x) fail = wsync_or(!mbar_wait(xbar, xph));
-            // ---- read-out: S_W^T x_e = g (D_hi + D_lo)[e] + Dc[e]; this thread's half of the columns
-            const int e0 = 16 * hk;
-            if (!fail && e0 < ne) {
-                float g1 = 1.f;
-                if (FAM == GDN) {
-#pragma unroll
-                    for (int i = 0; i < NJ; ++i) g1 *= i < n ? tab.al[i] : 1.f;
-                }
-                uint32_t dh[16], dl[16], dc[16];
-                tc::ld16(tmem + lane_q + T_D + 16 + e0, dh);
-                tc::ld16(tmem + lane_q + T_D + 16 + E + e0, dl);
-                if (n > 0) tc::ld16(tmem + lane_q + T_HI + e0, dc);
-                tc::wait_ld();
-                unsigned char* ust = sm + L.ust;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int e = e0 + i;
-                    if (e < ne) {
-                        float x = g1 * (__uint_as_float(dh[i]) + __uint_as_float(dl[i]));
-                        if (n > 0) x += __uint_as_float(dc[i]);
-                        if (e < r_h) {
-                            if (p.sketch_bf16) reinterpret_cast<uint16_t*>(ust)[e * TV + v] = f2bf(x);
-                            else reinterpret_cast<float*>(ust)[e * TV + v] = x;
-                        } else {
-                            reinterpret_cast<float*>(ust + E * TV * 4)[v] = x;
-                        }
-                    }
-                }
-            }
-            tc::fence_proxy_async();
-            if (!fail) mbar_arrive(rbar);
-        }
-        cph ^= 1u;
-        tc::fence_before();
-        if (csync_or(fail)) { ok = false; break; }                      // (5) TMEM, tables and buffers read
-        if (u != (long long)blockIdx.x) xph ^= 1u;
-        if (issuer) pending &= ~16u;
-        if (n > 0) u_prev = u;
+        u_prev = u;
+        ne_prev = ne;
+        r_prev = r_h;
+        g_prev = FAM == GDN ? g1 : 1.f;
     }
-    // the last head's S_W: staged by the workers, stored by the mover
-    if (!mov && ok && n > 0 && u_prev >= 0) {
+    // the last head's read-out and S_W (staged by the workers, stored by the mover)
+    if (!mov && ok && u_prev >= 0) {
         bool f = false;
-        if (!ctl) f = stage_sw();
+        if (!ctl) {
+            f = readout(ne_prev, r_prev, g_prev);
+            if (!f && n > 0) f = stage_sw();
+        }
         if (csync_or(f)) ok = false;
-        else if (issuer) pending &= ~32u;
+        else if (issuer) pending &= ~(16u | 32u);
     }
-    if (!ok && (issuer || t == 0)) {
+    if (!ok && issuer) {
         // a bounded wait ran out: report it, then wait (bounded) for this
         // thread's copies and MMAs still in flight before the memory is released
         if (issuer) report_timeout(p.status);
@@ -840,7 +938,6 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
         if (pending & 8u) mbar_wait(pbar, pph);
         if (pending & 16u) mbar_wait(cbar, cph);
         if (pending & 32u) mbar_wait(ubar, uph);
-        if (pending & 2u) mbar_wait(wbar, wph);
     }
     tc::fence_before();
     __syncthreads();
