@@ -50,17 +50,22 @@
 // Work split.  Persistent CTAs, one per SM, of 8 worker warps, an issuing warp
 // and a moving warp; CTA c walks heads c, c + grid, ...  Worker (v, half) owns
 // state column v and half of the dk rows.  Lane 0 of the issuing warp issues
-// the window copies and every MMA.  Lane 0 of the moving warp moves data in
-// and out with bulk copies, paced by mbarriers only (it takes part in no
-// barrier of the others): a head's tile is split into TMEM early in the head;
-// its buffer then stages the previous head's S_W (read from C), which the
-// mover stores before it loads the next head's tile into the same buffer; the
-// read-out is staged in shared memory and stored the same way.  No worker or
-// issuer waits for the tensor core's queue or for stores to drain.  MMA
-// groups complete on mbarriers.  Every wait on an mbarrier is bounded: when one runs
-// out the kernel sets SS_DEVICE_TIMEOUT in the caller's status word, waits
-// (bounded) for its own copies and MMAs in flight, releases its tensor memory
-// and returns.
+// every MMA; lane 0 of the moving warp every bulk copy in and out.  The three
+// roles are paced by mbarriers only: the workers arrive (256 arrivals) when
+// the keys and probes are staged, when S_0 is in TMEM and when W~ is, and the
+// issuer waits for those before Gm, the pass and the correction and update;
+// MMA groups complete on mbarriers the workers wait for.  The mover issues a
+// head's window once phase 1 of the previous head has read the window buffers
+// (fetching the scalars each copy needs a head ahead), splits nothing itself:
+// a head's tile is moved into TMEM by the workers early in the head; its
+// buffer then stages the previous head's S_W (read from C), which the mover
+// stores before it loads the next head's tile into the same buffer; the
+// read-out is staged in shared memory and stored the same way.  No worker
+// waits for the issuer, and no one for the tensor core's queue or for stores
+// to drain.  Every wait on an mbarrier is bounded: when one runs out the
+// kernel sets SS_DEVICE_TIMEOUT in the caller's status word, waits (bounded)
+// for its own copies and MMAs in flight, releases its tensor memory and
+// returns.
 #include "ss_mma.cuh"
 #include "ss_tc.cuh"
 
@@ -98,17 +103,6 @@ __device__ __forceinline__ bool wsync_or(bool x) {
     return r != 0;
 }
 
-// Barrier of the workers and the issuing warp (named barrier 2), returning
-// whether any of them passed `x` true.
-__device__ __forceinline__ bool csync_or(bool x) {
-    unsigned r;
-    asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 2, 288, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-        : "=r"(r)
-        : "r"(unsigned(x))
-        : "memory");
-    return r != 0;
-}
 
 // Rows of the pass's B buffer (K-major, 16-byte-atom swizzle, dk columns):
 //   [0, 16)              Y's keys (KDA: hi half of G(t,-1) ⊙ k_t)
@@ -326,6 +320,9 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     uint64_t* rbar = bars + 7;                                       // read-out staged (256 arrivals)
     uint64_t* ebar = bars + 10;                                      // the mover's stores have read the staging buffers
     uint64_t* xbar = bars + 11;                                      // phase 1 has read the window buffers
+    uint64_t* obar1 = bars + 12;                                     // workers -> issuer: keys and probes staged,
+    uint64_t* obar2 = bars + 13;                                     //   S_0 in TMEM,
+    uint64_t* obar5 = bars + 14;                                     //   W~ and k^.x ready (256 arrivals each)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
     volatile int* slow_flag = reinterpret_cast<volatile int*>(bars + 9);
     const bool stall = p.stall && blockIdx.x == 0;
@@ -351,6 +348,9 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
         mbar_init(rbar, NWK);
         mbar_init(ebar, 1);
         mbar_init(xbar, 1);
+        mbar_init(obar1, NWK);
+        mbar_init(obar2, NWK);
+        mbar_init(obar5, NWK);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -365,10 +365,9 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     griddep_wait();                                                   // the previous kernel's writes are visible
     griddep_launch_next();
 
-    // MMA groups in flight, for the issuer's bounded waits before an early
-    // exit: bits 2..5 (the Gm, pass, correction and update groups).  The
-    // mover keeps its own copies.
-    unsigned pending = 0;
+    // MMA groups the issuer committed to gbar, pbar, cbar and ubar: before the
+    // memory is released it waits (bounded) for the last of each.
+    unsigned ng = 0, np = 0, nc = 0, nu = 0;
     unsigned tph = 0, wph = 0, gph = 0, pph = 0, cph = 0, uph = 0, sph = 0, rph = 0, eph = 0;
     long long u = blockIdx.x;
     const long long stride = gridDim.x;
@@ -416,21 +415,24 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             tc::ld16(tmem + lane_q + T_D + 16 + E + e0, dl);
             if (n > 0) tc::ld16(tmem + lane_q + T_HI + e0, dc);
             tc::wait_ld();
+            // every sketch slot of this half is written (rows at or past r_p are
+            // never copied out), so that no store sits behind a branch
             unsigned char* ust = sm + L.ust;
+            float x[16], tokx = 0.f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int e = e0 + i;
-                if (e < ne_p) {
-                    float x = g_p * (__uint_as_float(dh[i]) + __uint_as_float(dl[i]));
-                    if (n > 0) x += __uint_as_float(dc[i]);
-                    if (e < r_p) {
-                        if (p.sketch_bf16) reinterpret_cast<uint16_t*>(ust)[e * TV + v] = f2bf(x);
-                        else reinterpret_cast<float*>(ust)[e * TV + v] = x;
-                    } else {
-                        reinterpret_cast<float*>(ust + E * TV * 4)[v] = x;
-                    }
-                }
+                x[i] = g_p * (__uint_as_float(dh[i]) + __uint_as_float(dl[i]));
+                if (n > 0) x[i] += __uint_as_float(dc[i]);
+                tokx = e0 + i == r_p ? x[i] : tokx;
             }
+            if (p.sketch_bf16) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) reinterpret_cast<uint16_t*>(ust)[(e0 + i) * TV + v] = f2bf(x[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) reinterpret_cast<float*>(ust)[(e0 + i) * TV + v] = x[i];
+            }
+            if (p.has_token && r_p >= e0 && r_p < e0 + 16) reinterpret_cast<float*>(ust + E * TV * 4)[v] = tokx;
         }
         tc::fence_proxy_async();
         mbar_arrive(rbar);
@@ -534,23 +536,113 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
         u = units;                                                      // the loop below is not the mover's
     }
 
+    if (ctl) {
+        // ---- the issuing thread: MMA groups as the workers' operands become ready ------------------
+        if (issuer) {
+            unsigned o1 = 0, o2 = 0, o5 = 0;
+            for (int k = 0; u < units; u += stride, ++k) {
+                unsigned char* const kub = sm + L.ku[0] + (k & 1) * (NJ * K * 4);
+                unsigned char* const kub2 = sm + L.ku2[0] + (k & 1) * (FAM == KDA ? NJ * K * 4 : 0);
+                // (1) keys and probes in shared memory, the slow-path verdict set
+                if (!mbar_wait(obar1, o1)) { ok = false; break; }
+                o1 ^= 1u;
+                tc::fence_after();
+                const int ne = tab.hr[k & 1] + p.has_token;             // read-out columns
+                const bool slow = FAM == KDA && *slow_flag != 0;
+                if (!slow) mbar_arrive(xbar);                           // the window buffers are free
+                // the previous head's MMAs have finished reading W~ and the B buffers
+                if (k > 0 && n > 0) {
+                    if (!mbar_wait(ubar, uph)) { ok = false; break; }
+                    uph ^= 1u;
+                }
+                tc::fence_after();
+                // Gm = [keys | probes] K'^T: the pass buffer's rows against the keys
+                if (!slow && n > 0) {
+                    const uint32_t id_g = tc::idesc_tf32(128, NG, 0, 0);
+                    const uint32_t s_b = FAM == KDA ? s_kq : s_bp;
+                    const int brows = FAM == KDA ? 2 * NJ : NB;
+#pragma unroll 1
+                    for (int q = 0; q < K / 8; ++q) {
+                        const uint32_t ko = (q & 3) * 32;
+                        const uint64_t a = tc::sdesc(s_bp + (q >> 2) * (NB * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
+                        const uint64_t bk = tc::sdesc(s_b + (q >> 2) * (brows * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
+                        tc::mma_ss(tmem + T_W, a, bk, id_g, q > 0);
+                    }
+                }
+                tc::commit(gbar);
+                ++ng;
+                // (2) S_0 in TMEM (the previous head's read-out has read the correction)
+                if (!mbar_wait(obar2, o2)) { ok = false; break; }
+                o2 ^= 1u;
+                tc::fence_after();
+                // D = S_0^T [keys | probes]: the hi half against every row, the lo half against the first 16 + E
+                const uint32_t id_hi = tc::idesc_tf32(TV, NB, 0, 0), id_lo = tc::idesc_tf32(TV, 16 + E, 0, 0);
+#pragma unroll 1
+                for (int q = 0; q < K / 8; ++q) {
+                    const uint64_t bd = tc::sdesc(s_bp + (q >> 2) * (NB * 128) + (q & 3) * 32, 16, 1024, tc::LAYOUT_SW128);
+                    tc::mma_ts(tmem + T_D, tmem + T_HI + 8 * q, bd, id_hi, q > 0);
+                    tc::mma_ts(tmem + T_D, tmem + T_LO + 8 * q, bd, id_lo, 1);
+                }
+                tc::commit(pbar);
+                ++np;
+                // (5) W~ in TMEM and k^.x in shared memory (Gm and the pass were read)
+                if (!mbar_wait(obar5, o5)) { ok = false; break; }
+                o5 ^= 1u;
+                tc::fence_after();
+                // Dc = W~^T (K^ X^T) into the first E columns of the S_0 region (read by the
+                // next head's workers before its S_0 lands there), then C += W~^T K^; each
+                // group completes on its own mbarrier (committed even when empty)
+                const int nq = (n + 7) / 8;
+                if (n > 0 && ne > 0) {
+                    const uint32_t id_x = tc::idesc_tf32(TV, E, 0, 0);
+                    for (int q = 0; q < nq; ++q) {
+                        const uint64_t xh = tc::sdesc(s_kxh + q * 32, 16, 1024, tc::LAYOUT_SW128);
+                        const uint64_t xl = tc::sdesc(s_kxl + q * 32, 16, 1024, tc::LAYOUT_SW128);
+                        tc::mma_ts(tmem + T_HI, tmem + T_W + 8 * q, xh, id_x, q > 0);
+                        tc::mma_ts(tmem + T_HI, tmem + T_W + 8 * q, xl, id_x, 1);
+                        tc::mma_ts(tmem + T_HI, tmem + T_W + 16 + 8 * q, xh, id_x, 1);
+                    }
+                }
+                tc::commit(cbar);
+                ++nc;
+                if (n > 0) {
+                    const uint32_t id_u = tc::idesc_tf32(TV, K, 0, 1);
+                    const uint32_t s_ku = smem_u32(kub), s_ku2 = smem_u32(kub2);
+                    for (int q = 0; q < nq; ++q) {
+                        const uint64_t bh = tc::sdesc(s_ku + q * 1024, NJ * 128, 512, tc::LAYOUT_SW128_32B);
+                        tc::mma_ts(tmem + T_C, tmem + T_W + 8 * q, bh, id_u, 1);
+                        tc::mma_ts(tmem + T_C, tmem + T_W + 16 + 8 * q, bh, id_u, 1);
+                        if (FAM == KDA)
+                            tc::mma_ts(tmem + T_C, tmem + T_W + 8 * q,
+                                       tc::sdesc(s_ku2 + q * 1024, NJ * 128, 512, tc::LAYOUT_SW128_32B), id_u, 1);
+                    }
+                    tc::commit(ubar);
+                    ++nu;
+                }
+            }
+        }
+        u = units;                                                      // the loop below is the workers'
+    }
+
+    // ---- the workers ----------------------------------------------------------------------------------
     // the previous head, whose read-out and S_W are finished during this one
     long long u_prev = -1;
     int ne_prev = 0, r_prev = 0;
     float g_prev = 1.f;
     for (int k = 0; u < units; u += stride, ++k) {
-        int r_h = 0, ne = 0;                                            // basis rows; read-out columns [Omega_h | q]
         unsigned char* const kub = sm + L.ku[0] + (k & 1) * (NJ * K * 4);            // this head's update keys
         unsigned char* const kub2 = sm + L.ku2[0] + (k & 1) * (FAM == KDA ? NJ * K * 4 : 0);
         bool fail = false, slow = false;
         uint32_t vv[NJ / 2];                                            // this column's values, bf16 pairs
         float g1 = 1.f;                                                 // GDN: A(n-1,-1)
 
-        if (!ctl) {
-            fail = wsync_or(!mbar_wait(wbar, wph));                     // the same verdict for every worker
-            r_h = tab.hr[k & 1];                                        // written before the window was issued
-        }
-        if (!ctl && !fail) {
+        // the window (this barrier also ends every worker's use of the previous
+        // head's tables and buffers)
+        if (wsync_or(!mbar_wait(wbar, wph))) { ok = false; break; }
+        wph ^= 1u;
+        const int r_h = tab.hr[k & 1];                                  // written before the window was issued
+        const int ne = r_h + p.has_token;                               // read-out columns [Omega_h | q]
+        {
             // ---- phase 1x: values, scalars, keys, probes (the window buffers) ----------------------
 #pragma unroll
             for (int j = 0; j < NJ / 2; ++j) {
@@ -608,36 +700,9 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             tc::fence_proxy_async();
         }
         if (t == 0) *slow_flag = slow ? 1 : 0;
-        if (csync_or(fail)) { ok = false; break; }                      // (1) operands in shared memory
-        wph ^= 1u;
-        r_h = tab.hr[k & 1];
-        ne = r_h + p.has_token;
-        slow = FAM == KDA && *slow_flag != 0;
+        mbar_arrive(obar1);                                             // (1) operands in shared memory
 
-        if (ctl) {
-            if (issuer) {
-                if (!slow) mbar_arrive(xbar);                           // the window buffers are free
-                // the previous head's MMAs have finished reading W~ and the B buffers
-                if (u_prev >= 0 && n > 0 && !mbar_wait(ubar, uph)) fail = true;
-                tc::fence_after();
-                // Gm = [keys | probes] K'^T: the pass buffer's rows against the keys
-                if (!fail && !slow && n > 0) {
-                    const uint32_t id_g = tc::idesc_tf32(128, NG, 0, 0);
-                    const uint32_t s_b = FAM == KDA ? s_kq : s_bp;
-                    const int brows = FAM == KDA ? 2 * NJ : NB;
-#pragma unroll 1
-                    for (int q = 0; q < K / 8; ++q) {
-                        const uint32_t ko = (q & 3) * 32;
-                        const uint64_t a = tc::sdesc(s_bp + (q >> 2) * (NB * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
-                        const uint64_t bk = tc::sdesc(s_b + (q >> 2) * (brows * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
-                        tc::mma_ss(tmem + T_W, a, bk, id_g, q > 0);
-                    }
-                }
-                tc::commit(gbar);
-                pending |= 4u;
-            }
-            __syncwarp();
-        } else {
+        {
             // the previous head's read-out (its correction ran during phase 1x)
             if (u_prev >= 0) fail = readout(ne_prev, r_prev, g_prev);
             // the tile; the barrier also orders the TMEM Dc reads before S_0 lands there
@@ -664,28 +729,13 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                 tc::wait_st();
             }
         }
-        tc::fence_before();
-        if (csync_or(fail)) { ok = false; break; }                      // (2) S_0 in TMEM, tile read
+        if (fail) { ok = false; break; }
         tph ^= 1u;
         if (u_prev >= 0) cph ^= 1u;
-        if (issuer && u_prev >= 0) pending &= ~(16u | 32u);
+        tc::fence_before();
+        mbar_arrive(obar2);                                             // (2) S_0 in TMEM, tile read
 
-        if (ctl) {
-            if (issuer) {
-                tc::fence_after();
-                // D = S_0^T [keys | probes]: the hi half against every row, the lo half against the first 16 + E
-                const uint32_t id_hi = tc::idesc_tf32(TV, NB, 0, 0), id_lo = tc::idesc_tf32(TV, 16 + E, 0, 0);
-#pragma unroll 1
-                for (int q = 0; q < K / 8; ++q) {
-                    const uint64_t bd = tc::sdesc(s_bp + (q >> 2) * (NB * 128) + (q & 3) * 32, 16, 1024, tc::LAYOUT_SW128);
-                    tc::mma_ts(tmem + T_D, tmem + T_HI + 8 * q, bd, id_hi, q > 0);
-                    tc::mma_ts(tmem + T_D, tmem + T_LO + 8 * q, bd, id_lo, 1);
-                }
-                tc::commit(pbar);
-                pending |= 8u;
-            }
-            __syncwarp();
-        } else {
+        {
             // ---- phase 2 (beside the pass) -----------------------------------------------------------
             if (n > 0) {
                 // the previous head's S_W (in C) to the tile buffer, then C = Diag(g) S_0
@@ -876,68 +926,31 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                 tc::wait_st();
             }
         }
-        tc::fence_before();
-        if (csync_or(fail)) { ok = false; break; }                      // (5) W~ and k^.x ready
+        if (fail) { ok = false; break; }
         gph ^= 1u;
         pph ^= 1u;
-        if (u_prev >= 0 && n > 0) uph ^= 1u;                            // the previous update, waited above
-        if (issuer) {
-            pending &= ~(4u | 8u);
-            tc::fence_after();
-            // Dc = W~^T (K^ X^T) into the first E columns of the S_0 region (read by the
-            // next head's workers before its S_0 lands there), then C += W~^T K^; each
-            // group completes on its own mbarrier (committed even when empty)
-            const int nq = (n + 7) / 8;
-            if (n > 0 && ne > 0) {
-                const uint32_t id_x = tc::idesc_tf32(TV, E, 0, 0);
-                for (int q = 0; q < nq; ++q) {
-                    const uint64_t xh = tc::sdesc(s_kxh + q * 32, 16, 1024, tc::LAYOUT_SW128);
-                    const uint64_t xl = tc::sdesc(s_kxl + q * 32, 16, 1024, tc::LAYOUT_SW128);
-                    tc::mma_ts(tmem + T_HI, tmem + T_W + 8 * q, xh, id_x, q > 0);
-                    tc::mma_ts(tmem + T_HI, tmem + T_W + 8 * q, xl, id_x, 1);
-                    tc::mma_ts(tmem + T_HI, tmem + T_W + 16 + 8 * q, xh, id_x, 1);
-                }
-            }
-            tc::commit(cbar);
-            if (n > 0) {
-                const uint32_t id_u = tc::idesc_tf32(TV, K, 0, 1);
-                const uint32_t s_ku = smem_u32(kub), s_ku2 = smem_u32(kub2);
-                for (int q = 0; q < nq; ++q) {
-                    const uint64_t bh = tc::sdesc(s_ku + q * 1024, NJ * 128, 512, tc::LAYOUT_SW128_32B);
-                    tc::mma_ts(tmem + T_C, tmem + T_W + 8 * q, bh, id_u, 1);
-                    tc::mma_ts(tmem + T_C, tmem + T_W + 16 + 8 * q, bh, id_u, 1);
-                    if (FAM == KDA)
-                        tc::mma_ts(tmem + T_C, tmem + T_W + 8 * q,
-                                   tc::sdesc(s_ku2 + q * 1024, NJ * 128, 512, tc::LAYOUT_SW128_32B), id_u, 1);
-                }
-                tc::commit(ubar);
-                pending |= 32u;
-            }
-            pending |= 16u;
-        }
+        if (u_prev >= 0 && n > 0) uph ^= 1u;                            // the previous update, waited in phase 2
+        tc::fence_before();
+        mbar_arrive(obar5);                                             // (5) W~ and k^.x ready
         u_prev = u;
         ne_prev = ne;
         r_prev = r_h;
         g_prev = FAM == GDN ? g1 : 1.f;
     }
     // the last head's read-out and S_W (staged by the workers, stored by the mover)
-    if (!mov && ok && u_prev >= 0) {
-        bool f = false;
-        if (!ctl) {
-            f = readout(ne_prev, r_prev, g_prev);
-            if (!f && n > 0) f = stage_sw();
-        }
-        if (csync_or(f)) ok = false;
-        else if (issuer) pending &= ~(16u | 32u);
+    if (!ctl && !mov && ok && u_prev >= 0) {
+        bool f = readout(ne_prev, r_prev, g_prev);
+        if (!f && n > 0) f = stage_sw();
+        if (f) ok = false;
     }
-    if (!ok && issuer) {
-        // a bounded wait ran out: report it, then wait (bounded) for this
-        // thread's copies and MMAs still in flight before the memory is released
-        if (issuer) report_timeout(p.status);
-        if (pending & 4u) mbar_wait(gbar, gph);
-        if (pending & 8u) mbar_wait(pbar, pph);
-        if (pending & 16u) mbar_wait(cbar, cph);
-        if (pending & 32u) mbar_wait(ubar, uph);
+    // a bounded wait ran out: report it; the issuer waits (bounded) for its last
+    // MMA groups before the tensor memory is released
+    if (!ok && (issuer || mover || t == 0)) report_timeout(p.status);
+    if (issuer) {
+        if (ng > 0) mbar_wait(gbar, (ng - 1) & 1u);
+        if (np > 0) mbar_wait(pbar, (np - 1) & 1u);
+        if (nc > 0) mbar_wait(cbar, (nc - 1) & 1u);
+        if (nu > 0) mbar_wait(ubar, (nu - 1) & 1u);
     }
     tc::fence_before();
     __syncthreads();
