@@ -364,6 +364,7 @@ __device__ __forceinline__ void window_read(const StepParams& p, int h, int l, i
 // on more CTAs measured faster than on deeper per-warp pipelines.
 // ---------------------------------------------------------------------------
 constexpr int DEC_WARPS = 4;              // warps per decode CTA
+constexpr int DEC_UREG_ROWS = 16;         // sketch rows a unit can hold in registers
 
 // Lanes per unit.  Mamba-2's reads are independent dot products, which 16
 // lanes (2 units per warp) reduce cheaply; the delta rule's sweep is serial
@@ -504,11 +505,15 @@ __device__ __forceinline__ void axpy(float a, const float (&x)[E], float (&y)[E]
     for (int e = 0; e < E; ++e) y[e] = fmaf(a, x[e], y[e]);
 }
 
-template <int FAM, int K, int V, bool UB16, bool MIXED>
+// UREG: the unit's sketch rows (bf16, at most DEC_UREG_ROWS, four channels a
+// lane) are read straight into registers at the top of the unit instead of
+// being staged in shared memory, which leaves room for more resident units.
+template <int FAM, int K, int V, bool UB16, bool MIXED, bool UREG>
 __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_constant__ StepParams p,
                                                                int rmax, int ns, int stage_bytes) {
     constexpr int G = dec_gl(FAM), UPW = 32 / G;
     constexpr int EK = K / G, EV = V / G, ESZ = UB16 ? 2 : 4;
+    static_assert(!UREG || (UB16 && EV == 4 && Own<V, G>::M == 1), "register sketch rows: bf16, 4 channels a lane");
     extern __shared__ __align__(16) unsigned char smem[];
     const int wpc = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -526,7 +531,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
     // sketch dtype) after its sketch rows; otherwise the CTA stages the
     // head's shared fp32 C once.
     const bool smap = p.cmap != nullptr;
-    const UnitSmem L = unit_smem(FAM, K, V, P, dec_ubytes(K, V, rmax, ESZ, smap, p.dense_any));
+    const UnitSmem L = unit_smem(FAM, K, V, P, UREG ? 0 : dec_ubytes(K, V, rmax, ESZ, smap, p.dense_any));
     const int cbytes = smap ? 0 : align16(rmax * K * 4);
     const float* csm = reinterpret_cast<const float*>(smem);
     uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + cbytes);
@@ -545,7 +550,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
             if (b < p.B && Pb >= 0 && Pb < p.W - 1)
                 stage_unit_bulk<FAM, K, V>(p, (long long)b * p.H + h, Pb, wbase + s * stage_bytes + 16 + g * L.total, L,
                                            static_cast<const char*>(p.sketch) + (b * (long long)p.R + off) * (V * ESZ),
-                                           r * V * ESZ, bar(s), (stall && it == 0 && g == 0) ? 16u : 0u,
+                                           UREG ? 0 : r * V * ESZ, bar(s), (stall && it == 0 && g == 0) ? 16u : 0u,
                                            smap ? static_cast<const char*>(p.cmap) + (b * (long long)p.R + off) * (K * ESZ)
                                                 : nullptr,
                                            smap ? r * K * ESZ : 0);
@@ -585,6 +590,14 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
         if (active) {
             if (FAM != KDA) tgate = p.tok_gate[u];
             if (FAM != MAMBA2) tbeta = p.tok_beta[u];
+        }
+        uint2 ureg[UREG ? DEC_UREG_ROWS : 1];                  // this lane's channels of the sketch rows
+        if constexpr (UREG) {
+            const uint16_t* urow = static_cast<const uint16_t*>(p.sketch) + (b * (long long)p.R + off) * V +
+                                   Own<V, G>::base(0, l);
+#pragma unroll
+            for (int i = 0; i < DEC_UREG_ROWS; ++i)
+                ureg[i] = active && i < r ? __ldg(reinterpret_cast<const uint2*>(urow + i * V)) : make_uint2(0u, 0u);
         }
         ok = __all_sync(FULL, mbar_wait(bar(s), (phases >> s) & 1u));
         if (!ok) break;
@@ -846,7 +859,33 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const __grid_con
             if (smap) row_any<K, G, UB16>(cmu + i * K * ESZ, l, ci);
             else row_f32<K, G>(csm + i * K, l, ci);
         };
-        int i = 0;
+        if constexpr (UREG) {
+#pragma unroll
+            for (int i0 = 0; i0 < DEC_UREG_ROWS; i0 += 4) {
+                if (i0 < r) {
+                    float c[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        c[q] = 0.f;
+                        if (i0 + q < r) {
+                            float ci[EK];
+                            crow(i0 + q, ci);
+                            c[q] = dot<EK>(ci, x);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) c[q] = gsum<G>(c[q]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {             // rows past r are zero
+                        float ui[EV];
+                        unpack2(ureg[i0 + q].x, ui);
+                        unpack2(ureg[i0 + q].y, ui + 2);
+                        axpy<EV>(c[q], ui, ob);
+                    }
+                }
+            }
+        }
+        int i = UREG ? r : 0;
         for (; i + 4 <= r; i += 4) {
             float c[4];
 #pragma unroll
@@ -976,24 +1015,24 @@ __global__ void __launch_bounds__(128) replay_kernel(const __grid_constant__ Ste
 // ---------------------------------------------------------------------------
 // One warp's staging buffer; with the state-dependent map (`smap`) each unit
 // also stages its own map rows.
-int decode_stage(int fam, int K, int V, int P, int rmax, int esz, bool smap, bool dense_any) {
-    return dec_stage_bytes(fam, K, V, P, dec_ubytes(K, V, rmax, esz, smap, dense_any));
+int decode_stage(int fam, int K, int V, int P, int rmax, int esz, bool smap, bool dense_any, bool ureg = false) {
+    return dec_stage_bytes(fam, K, V, P, ureg ? 0 : dec_ubytes(K, V, rmax, esz, smap, dense_any));
 }
 
 // The CTA-wide part: the head's shared C (fixed map only) and its mbarrier.
 int decode_cpart(int K, int rmax, bool smap) { return (smap ? 0 : align16(rmax * K * 4)) + 16; }
 
-template <int FAM, int K, int V, bool UB16, bool MIXED>
+template <int FAM, int K, int V, bool UB16, bool MIXED, bool UREG>
 cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
     constexpr int esz = UB16 ? 2 : 4, upw = 32 / dec_gl(FAM);
     const bool smap = p.cmap != nullptr;
-    const int stage = decode_stage(FAM, K, V, p.p, rmax, esz, smap, p.dense_any != 0);
+    const int stage = decode_stage(FAM, K, V, p.p, rmax, esz, smap, p.dense_any != 0, UREG);
     const int cpart = decode_cpart(K, rmax, smap);
     if (cpart + stage > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
     int wpc = DEC_WARPS;
     while (wpc > 1 && cpart + wpc * stage > SMEM_LIMIT) --wpc;
     const int bytes = cpart + wpc * stage;
-    auto kern = decode_kernel<FAM, K, V, UB16, MIXED>;
+    auto kern = decode_kernel<FAM, K, V, UB16, MIXED, UREG>;
     static KernelCache kc;
     cudaError_t e = ensure_smem(kern, kc, bytes);
     if (e != cudaSuccess) return e;
@@ -1002,13 +1041,53 @@ cudaError_t decode_launch(const StepParams& p, int rmax, cudaStream_t stream) {
     return launch_pdl(kern, dim3(unsigned(nb), unsigned(p.H)), dim3(wpc * 32), bytes, stream, p, rmax, 1, stage);
 }
 
+// Resident CTAs per SM of a decode launch from its registers a thread and
+// shared memory (1 KB of each SM's reserved per CTA).
+int dec_blocks_per_sm(int regs, int bytes) {
+    const int rr = (regs + 7) & ~7;
+    const int by_regs = 65536 / (DEC_WARPS * 32 * rr);
+    const int by_smem = SMEM_SM / (bytes + 1024);
+    const int by_thr = 2048 / (DEC_WARPS * 32);
+    return std::min(std::min(by_regs, by_smem), by_thr);
+}
+
+// Whether the register-held sketch rows fit more units on an SM than staging
+// them: they free shared memory but cost registers.
+template <int FAM, int K, int V, bool MIXED, bool OK>
+bool dec_prefer_ureg(const StepParams& p, int rmax) {
+    if constexpr (!OK) {
+        return false;
+    } else {
+        constexpr int esz = 2;
+        static KernelCache kc0, kc1;
+        int r0 = 0, r1 = 0;
+        if (cached_regs(decode_kernel<FAM, K, V, true, MIXED, false>, kc0, &r0) != cudaSuccess ||
+            cached_regs(decode_kernel<FAM, K, V, true, MIXED, true>, kc1, &r1) != cudaSuccess)
+            return false;
+        const int cpart = decode_cpart(K, rmax, false);
+        const int b0 = cpart + DEC_WARPS * decode_stage(FAM, K, V, p.p, rmax, esz, false, false, false);
+        const int b1 = cpart + DEC_WARPS * decode_stage(FAM, K, V, p.p, rmax, esz, false, false, true);
+        return dec_blocks_per_sm(r1, b1) > dec_blocks_per_sm(r0, b0);
+    }
+}
+
 template <int FAM, int K, int V>
 cudaError_t decode_t(const StepParams& p, int rmax, cudaStream_t stream) {
-    if (p.fill_in)
-        return p.sketch_bf16 ? decode_launch<FAM, K, V, true, true>(p, rmax, stream)
-                             : decode_launch<FAM, K, V, false, true>(p, rmax, stream);
-    return p.sketch_bf16 ? decode_launch<FAM, K, V, true, false>(p, rmax, stream)
-                         : decode_launch<FAM, K, V, false, false>(p, rmax, stream);
+    // bf16 sketch rows of the fixed map, no dense-fallback head: held in
+    // registers when that leaves more units resident
+    constexpr int G = dec_gl(FAM);
+    constexpr bool UREG_OK = V / G == 4 && Own<V, G>::M == 1;
+    const bool ureg = UREG_OK && p.sketch_bf16 && p.cmap == nullptr && !p.dense_any && rmax <= DEC_UREG_ROWS &&
+                      (p.fill_in ? dec_prefer_ureg<FAM, K, V, true, UREG_OK>(p, rmax)
+                                  : dec_prefer_ureg<FAM, K, V, false, UREG_OK>(p, rmax));
+    if (p.fill_in) {
+        if (!p.sketch_bf16) return decode_launch<FAM, K, V, false, true, false>(p, rmax, stream);
+        return ureg ? decode_launch<FAM, K, V, true, true, UREG_OK>(p, rmax, stream)
+                    : decode_launch<FAM, K, V, true, true, false>(p, rmax, stream);
+    }
+    if (!p.sketch_bf16) return decode_launch<FAM, K, V, false, false, false>(p, rmax, stream);
+    return ureg ? decode_launch<FAM, K, V, true, false, UREG_OK>(p, rmax, stream)
+                : decode_launch<FAM, K, V, true, false, false>(p, rmax, stream);
 }
 
 template <int FAM, int K, int V>
