@@ -163,7 +163,7 @@ def kernel_traffic_record(name, workload, coef="fixed"):
         with open(path) as f:
             rec = json.load(f)
         sha = kernel_source_sha()
-        r = rec.get(name)
+        r = rec.get(f"{name}@{workload}") or rec.get(name)
         if r and r.get("source_sha") == sha and r.get("workload") == workload:
             return r
     except (OSError, ValueError):
@@ -299,10 +299,17 @@ def kernel_stats(plan, B, W, dec_ms, n_dec, fl_ms, n_fl, flush_name, peak, wl_na
     return kernels
 
 
-def flush_kernel_name(family, smap, synth):
-    """The kernel that runs a family's flush (see launch_flush in the library)."""
+def flush_kernel_name(family, smap, synth, wl=None, rmax=0):
+    """The kernel that runs a family's flush (see launch_flush in the library):
+    Mamba-2 with the fixed map on the warp-MMA kernel; GDN and KDA with the
+    fixed map, dv = 128, dk = 64 or 128, at most 16 updates and 32 read-out
+    columns (rank + the token) on the tensor-core kernel; the rest on the
+    CUDA-core kernel."""
     if family == synth.MAMBA2 and not smap:
         return "flush_mma_kernel"
+    if (not smap and wl is not None and wl.dv == 128 and wl.dk in (64, 128) and wl.window <= 16
+            and rmax + 1 <= 32):
+        return "flush_tc_kernel"
     return "flush_kernel"
 
 
@@ -350,7 +357,8 @@ def other_families(args, dev, stream, torch, B, synth, DecodeLayer, peak, names=
             fl_ms = sum(m[1].elapsed_time(m[2]) for m in marks)
             tot_ms = sum(m[0].elapsed_time(m[2]) for m in marks)
             kern = kernel_stats(layers[0].plan, B, W, dec_ms, nwin * NL * (W - 1), fl_ms, nwin * NL,
-                                flush_kernel_name(wl.family, False, synth), peak, wl.name)
+                                flush_kernel_name(wl.family, False, synth, wl, int(np.max(st.ranks))), peak,
+                                wl.name)
             out[name] = {"value": wl.units * W * NL * nwin / (tot_ms / 1e3), "unit": "seq*heads/s",
                          "windows": nwin, "layers": NL, "kernels": kern,
                          "status": int(sum(int(l.status[0].item()) for l in layers))}
@@ -449,7 +457,7 @@ def run_ours(args, rank, world):
     peaks, peak_kind = measured_peaks()
     peak = float(peaks["hbm_gbs"])
     plan = layers[0].plan
-    flush_name = flush_kernel_name(wl.family, smap, synth)
+    flush_name = flush_kernel_name(wl.family, smap, synth, wl, int(np.max(st.ranks)))
     kernels = kernel_stats(plan, B, W, dec_ms, n_dec, fl_ms, n_fl, flush_name, peak, wl.name, args.coef)
     if W > 1:
         kernels["decode_kernel"]["by_phase_us"] = [

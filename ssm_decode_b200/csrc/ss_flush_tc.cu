@@ -116,7 +116,7 @@ __host__ __device__ constexpr int pass_rows(int fam, int E) { return 16 + 2 * E 
 
 // Per-CTA shared-memory layout (byte offsets from a 1024-byte-aligned base).
 struct TcLayout {
-    int tile, bp, ku[2], ku2[2], kq, kxh, kxl, part, ust, kraw, vraw, graw, braw, sg, sb, tq, tab, bars, total;
+    int tile, bp, g16, k16, ku[2], ku2[2], kq, kxh, kxl, part, ust, kraw, vraw, graw, braw, sg, sb, tq, tab, bars, total;
 };
 
 __host__ __device__ inline TcLayout tc_layout(int fam, int K, int E) {
@@ -125,6 +125,8 @@ __host__ __device__ inline TcLayout tc_layout(int fam, int K, int E) {
     int o = 0;
     L.tile = o; o += K * TV * 4;                    // the state tile (32-byte-atom swizzle), then S_W
     L.bp = o;   o += pass_rows(fam, E) * K * 4;     // the pass's B buffer
+    L.g16 = o;  o += kda ? 0 : 128 * K * 2;         // GDN: Gm's A in bf16, [keys | probes in three parts]
+    L.k16 = o;  o += kda ? 0 : NJ * K * 2;          // GDN: Gm's B, the keys in bf16
     for (int i = 0; i < 2; ++i) {                   // update keys, MN-major (KDA: hi half), by head parity
         L.ku[i] = o; o += NJ * K * 4;
     }
@@ -134,7 +136,7 @@ __host__ __device__ inline TcLayout tc_layout(int fam, int K, int E) {
     L.kq = o;   o += kda ? 2 * NJ * K * 4 : 0;      // KDA: k_j / G(j,-1), K-major, hi rows then lo rows
     L.kxh = o;  o += E * 128;                       // k^_j . x_e, K-major [e][j] (j < 32), hi half
     L.kxl = o;  o += E * 128;                       // and lo half
-    L.part = o; o += (2 * NJ + 2 * E) * NJ * 4;     // pieces of the pair weights and of k^ . x
+    L.part = o; o += (2 * NJ + (kda ? 2 : 3) * E) * NJ * 4;   // pieces of the pair weights and of k^ . x
     L.ust = o;  o += E * TV * 4 + TV * 4;           // the read-out staged: sketch rows, then o
     L.kraw = o; o += NJ * K * 2;
     L.vraw = o; o += NJ * TV * 2;
@@ -240,6 +242,10 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+// Four fp32 values rounded to bf16, packed in memory order.
+__device__ __forceinline__ uint2 bf16x4(float4 x) {
+    return make_uint2(uint32_t(f2bf(x.x)) | (uint32_t(f2bf(x.y)) << 16), uint32_t(f2bf(x.z)) | (uint32_t(f2bf(x.w)) << 16));
+}
 __device__ __forceinline__ float4 hi4(float4 x) { return make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w)); }
 
 // KDA, phase 1x: thread (c, HALF) takes slots j of its half of the window.
@@ -340,6 +346,7 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     float* const pb = pa + NJ * NJ;                                   // [NJ][NJ] KDA: from the keys' lo rows
     float* const xa = pb + NJ * NJ;                                   // [E][NJ] from the probes' hi rows
     float* const xb = xa + E * NJ;                                    // [E][NJ] from the probes' lo rows
+    float* const xc = xb + E * NJ;                                    // [E][NJ] GDN: the third bf16 part
     const size_t esz = p.sketch_bf16 ? 2 : 4;
 
     if (t == 0) {
@@ -556,8 +563,19 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     uph ^= 1u;
                 }
                 tc::fence_after();
-                // Gm = [keys | probes] K'^T: the pass buffer's rows against the keys
-                if (!slow && n > 0) {
+                // Gm = [keys | probes] K'^T.  GDN: bf16 operands, the keys exact and
+                // the probes in three parts, K = 16 an instruction
+                if (FAM == GDN && n > 0) {
+                    const uint32_t id_g = tc::idesc_bf16(128, NJ);
+                    const uint32_t s_g16 = smem_u32(sm + L.g16), s_k16 = smem_u32(sm + L.k16);
+#pragma unroll 1
+                    for (int q = 0; q < K / 16; ++q) {
+                        const uint32_t ko = (q & 3) * 32;
+                        const uint64_t a = tc::sdesc(s_g16 + (q >> 2) * (128 * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
+                        const uint64_t bk = tc::sdesc(s_k16 + (q >> 2) * (NJ * 128) + ko, 16, 1024, tc::LAYOUT_SW128);
+                        tc::mma_ss_bf16(tmem + T_W, a, bk, id_g, q > 0);
+                    }
+                } else if (!slow && n > 0) {
                     const uint32_t id_g = tc::idesc_tf32(128, NG, 0, 0);
                     const uint32_t s_b = FAM == KDA ? s_kq : s_bp;
                     const int brows = FAM == KDA ? 2 * NJ : NB;
@@ -662,23 +680,27 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             }
             bool tiny = false;
             if constexpr (FAM == GDN) {
+#pragma unroll
                 for (int i = t; i < NJ * (K / 4); i += NWK) {
                     const int j = i / (K / 4), c = (i % (K / 4)) * 4;
-                    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (j < n) {
-                        const uint2 w = *reinterpret_cast<const uint2*>(kraw + j * K + c);
-                        v4 = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
-                    }
+                    uint2 w = make_uint2(0u, 0u);
+                    if (j < n) w = *reinterpret_cast<const uint2*>(kraw + j * K + c);
+                    const float4 v4 = make_float4(bf2f_lo(w.x), bf2f_hi(w.x), bf2f_lo(w.y), bf2f_hi(w.y));
                     *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, j, c)) = v4;
                     *reinterpret_cast<float4*>(kub + tc::sw32b_off(NJ, j, c)) = v4;
+                    // Gm in bf16: the keys as its B operand and as A's first rows
+                    *reinterpret_cast<uint2*>(sm + L.k16 + tc::sw128h_off(NJ, j, c)) = w;
+                    *reinterpret_cast<uint2*>(sm + L.g16 + tc::sw128h_off(128, j, c)) = w;
                 }
             } else if (t < 2 * K) {
                 if (t < K) tiny = kda_keys<K, 0>(t, n, E, NB, kraw, graw, bp, sm + L.kq, kub, kub2, tab.gw);
                 else tiny = kda_keys<K, 1>(t - K, n, E, NB, kraw, graw, bp, sm + L.kq, kub, kub2, tab.gw);
             }
             slow = wsync_or(tiny) && FAM == KDA;                        // tab.gw is written
-            // the probes (KDA: scaled by G(n-1,-1)), hi and lo halves
-            for (int idx = t; idx < E * (K / 4); idx += NWK) {
+            // the probes (KDA: scaled by G(n-1,-1)), hi and lo halves; rows past
+            // ne keep stale values, which only reach columns no one reads
+#pragma unroll 2
+            for (int idx = t; idx < ne * (K / 4); idx += NWK) {
                 const int e = idx / (K / 4), c = (idx % (K / 4)) * 4;
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (e < r_h) {
@@ -692,10 +714,23 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                 *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, 16 + e, c)) = hi;
                 *reinterpret_cast<float4*>(bp + tc::sw128_off(NB, 16 + E + e, c)) =
                     make_float4(x.x - hi.x, x.y - hi.y, x.z - hi.z, x.w - hi.w);
-            }
-            if (FAM == GDN) {
+                if constexpr (FAM == GDN) {
+                    // Gm's A rows in bf16: x = p1 + p2 + p3 exactly (each part the
+                    // rounded remainder of the previous ones)
+                    float4 r = x;
 #pragma unroll
-                for (int i = 0; i < NJ; ++i) g1 *= i < n ? tab.al[i] : 1.f;
+                    for (int pi = 0; pi < 3; ++pi) {
+                        const uint2 h = bf16x4(r);
+                        *reinterpret_cast<uint2*>(sm + L.g16 + tc::sw128h_off(128, 16 + pi * E + e, c)) = h;
+                        r = make_float4(r.x - bf2f_lo(h.x), r.y - bf2f_hi(h.x), r.z - bf2f_lo(h.y), r.w - bf2f_hi(h.y));
+                    }
+                }
+            }
+            if (FAM == GDN) {                                           // A(n-1,-1), as a product tree
+                float g4[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                for (int i = 0; i < NJ; ++i) g4[i & 3] *= i < n ? tab.al[i] : 1.f;
+                g1 = (g4[0] * g4[1]) * (g4[2] * g4[3]);
             }
             tc::fence_proxy_async();
         }
@@ -775,6 +810,7 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                     else if (r < 16 + E) dst = xa + (r - 16) * NJ;
                     else if (r < 16 + 2 * E) { dst = xb + (r - 16 - E) * NJ; both = false; }
                     else if (FAM == KDA && r < 32 + 2 * E) { dst = pb + (r - 16 - 2 * E) * NJ; both = false; }
+                    else if (FAM == GDN && r < 16 + 3 * E) dst = xc + (r - 16 - 2 * E) * NJ;
                     if (dst != nullptr) {
 #pragma unroll
                         for (int j = 0; j < NJ; ++j)
@@ -844,7 +880,7 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
             // k^_j . x_e as the correction's B operand (K-major [e][j]), hi and lo
             for (int idx = t; idx < E * NJ; idx += NWK) {
                 const int e = idx / NJ, j = idx % NJ;
-                const float x = (j < n && e < ne) ? xa[idx] + xb[idx] : 0.f;
+                const float x = (j < n && e < ne) ? xa[idx] + xb[idx] + (FAM == GDN ? xc[idx] : 0.f) : 0.f;
                 const float hi = tf32_hi(x);
                 *reinterpret_cast<float*>(sm + L.kxh + tc::sw128_off(E, e, j)) = hi;
                 *reinterpret_cast<float*>(sm + L.kxl + tc::sw128_off(E, e, j)) = x - hi;

@@ -41,6 +41,22 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, int a_mn, int b_
            (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
+// Instruction descriptor of a dense bf16 x bf16 -> fp32 MMA (kind::f16, K = 16
+// per instruction): A and B formats 1 (bf16) in bits 7-9 and 10-12, both
+// K-major, N / 8 in bits 17-22, M / 16 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A * B with both operands bf16 in shared memory.  One thread issues.
+__device__ __forceinline__ void mma_ss_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
 // D[tmem] (+)= A[smem desc] * B[smem desc]; acc = 0 overwrites D.  One thread issues.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
@@ -123,6 +139,10 @@ __device__ __forceinline__ void st16(uint32_t a, const uint32_t (&r)[16]) {
 //               writes for a box of 32 fp32 columns).
 __host__ __device__ constexpr uint32_t sw128_off(int rows, int row, int col) {
     return uint32_t((col >> 5) * (rows * 128) + row * 128 + ((((col & 31) >> 2) ^ (row & 7)) << 4) + ((col & 3) << 2));
+}
+// The same 16-byte-chunk swizzle for bf16 elements: column blocks of 64 values.
+__host__ __device__ constexpr uint32_t sw128h_off(int rows, int row, int col) {
+    return uint32_t((col >> 6) * (rows * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1));
 }
 __host__ __device__ constexpr uint32_t sw32b_off(int rows, int row, int col) {
     return uint32_t((col >> 5) * (rows * 128) + row * 128 + ((((col & 31) >> 3) ^ (row & 3)) << 5) + ((col & 7) << 2));
