@@ -446,6 +446,44 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
         return false;
     };
 
+    // The read-out of a head in two parts: its values from TMEM (this thread's
+    // half of the columns, once the correction has completed), then, once the
+    // mover has read the previous read-out out of the staging buffer, the
+    // staging stores and the arrival on rbar.
+    auto ro_load = [&](int ne_p, int r_p, float g_p, float (&x)[16], float& tokx) {
+        const int e0 = 16 * hk;
+        if (e0 >= ne_p) return;
+        uint32_t dh[16], dl[16], dc[16];
+        tc::ld16(tmem + lane_q + T_D + 16 + e0, dh);
+        tc::ld16(tmem + lane_q + T_D + 16 + E + e0, dl);
+        if (n > 0) tc::ld16(tmem + lane_q + T_HI + e0, dc);
+        tc::wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            x[i] = g_p * (__uint_as_float(dh[i]) + __uint_as_float(dl[i]));
+            if (n > 0) x[i] += __uint_as_float(dc[i]);
+            tokx = e0 + i == r_p ? x[i] : tokx;
+        }
+    };
+    auto ro_stage = [&](int ne_p, int r_p, const float (&x)[16], float tokx) {
+        const int e0 = 16 * hk;
+        if (e0 < ne_p) {
+            // every sketch slot of this half is written (rows at or past r_p are
+            // never copied out), so that no store sits behind a branch
+            unsigned char* ust = sm + L.ust;
+            if (p.sketch_bf16) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) reinterpret_cast<uint16_t*>(ust)[(e0 + i) * TV + v] = f2bf(x[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) reinterpret_cast<float*>(ust)[(e0 + i) * TV + v] = x[i];
+            }
+            if (p.has_token && r_p >= e0 && r_p < e0 + 16) reinterpret_cast<float*>(ust + E * TV * 4)[v] = tokx;
+        }
+        tc::fence_proxy_async();
+        mbar_arrive(rbar);
+    };
+
     bool ok = true;
     if (mov) {
         // ---- the moving warp: windows and tiles in; read-outs and S_W out ----------------------------
@@ -653,6 +691,7 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
         bool fail = false, slow = false;
         uint32_t vv[NJ / 2];                                            // this column's values, bf16 pairs
         float g1 = 1.f;                                                 // GDN: A(n-1,-1)
+        float rx[16], rtok = 0.f;                                       // the previous head's read-out
 
         // the window (this barrier also ends every worker's use of the previous
         // head's tables and buffers)
@@ -696,7 +735,20 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
                 if (t < K) tiny = kda_keys<K, 0>(t, n, E, NB, kraw, graw, bp, sm + L.kq, kub, kub2, tab.gw);
                 else tiny = kda_keys<K, 1>(t - K, n, E, NB, kraw, graw, bp, sm + L.kq, kub, kub2, tab.gw);
             }
-            slow = wsync_or(tiny) && FAM == KDA;                        // tab.gw is written
+            // KDA: the previous head's read-out, from TMEM: its correction was
+            // issued as this head began and has had phase 1 to complete.  The
+            // values wait in registers until the staging buffer is free (after
+            // the operands are in).  (GDN, whose phase 1 is shorter, reads it in
+            // one piece after the operands.)
+            bool cf = false;
+            if (FAM == KDA && u_prev >= 0) {
+                cf = !mbar_wait(cbar, cph);
+                tc::fence_after();
+                if (!cf) ro_load(ne_prev, r_prev, g_prev, rx, rtok);
+            }
+            const bool v1 = wsync_or(tiny || cf);                       // tab.gw is written
+            if (v1 && wsync_or(cf)) { ok = false; break; }
+            slow = v1 && FAM == KDA;
             // the probes (KDA: scaled by G(n-1,-1)), hi and lo halves; rows past
             // ne keep stale values, which only reach columns no one reads
 #pragma unroll 2
@@ -738,10 +790,17 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
         mbar_arrive(obar1);                                             // (1) operands in shared memory
 
         {
-            // the previous head's read-out (its correction ran during phase 1x)
-            if (u_prev >= 0) fail = readout(ne_prev, r_prev, g_prev);
-            // the tile; the barrier also orders the TMEM Dc reads before S_0 lands there
-            fail = wsync_or(fail || !mbar_wait(tbar, tph));
+            // the previous head's read-out into the staging buffer for the mover
+            bool ef = false;
+            if (FAM == KDA && u_prev >= 0) {
+                ef = !mbar_wait(ebar, eph);
+                eph ^= 1u;
+                if (!ef) ro_stage(ne_prev, r_prev, rx, rtok);
+            } else if (u_prev >= 0) {
+                ef = readout(ne_prev, r_prev, g_prev);
+            }
+            // the tile (earlier barriers ordered the TMEM Dc reads before S_0 lands there)
+            fail = wsync_or(ef || !mbar_wait(tbar, tph));
             // ---- phase 1y: S_0 into TMEM (beside Gm) ---------------------------------------------------
             if (!fail) {
                 // S_0's raw value (the hi half) and its lo half, this thread's column
