@@ -237,38 +237,46 @@ def other_modes(args, wl, st, layers, toks, W, units, dev, stream, torch, B, Dec
                         "status": int(sum(int(l.status[0].item()) for l in layers))}
     except Exception as e:                 # noqa: BLE001 - reported in the line
         out["mixed"] = {"error": repr(e)[:200]}
-    try:                                   # the state-dependent coefficient map (rho 0.01)
-        import numpy as np  # noqa: F401
-        skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
-        sl = []
-        for _ in range(2):
-            lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev,
-                              coef_mode=B.SS_COEF_STATE, coef_ridge=0.01)
-            lay.state.copy_(layers[0].state)
-            lay.basis.copy_(layers[0].basis)
-            lay.A.copy_(layers[0].A)
-            lay.prime()
-            sl.append(lay)
-        ts = []
-        for k in range(3):
-            a, b = ev(), ev()
-            a.record(stream)
-            for p in range(W):
-                for l, lay in enumerate(sl):
-                    lay.step(toks[(p + l) % W])
-            b.record(stream)
-            torch.cuda.synchronize()
-            if k:
-                ts.append(a.elapsed_time(b))
-        ms = min(ts) / len(sl)
-        approx = sketch_vs_exact(sl, toks, W, torch)
-        out["state_map"] = {"what": "the same window with the state-dependent map (rho 0.01) built by every flush",
-                            "ms_per_window": ms, "value": units * W / (ms / 1e3), "unit": "seq*heads/s",
-                            "approx_mean": approx["mean"], "approx_aggregate": approx["aggregate"]}
-        del sl
-        torch.cuda.empty_cache()
-    except Exception as e:                 # noqa: BLE001
-        out["state_map"] = {"error": repr(e)[:200]}
+    # the state-dependent coefficient maps (rho 0.01): the exact least-squares
+    # map (paper §A.2.1) and the low-rank-plus-diagonal one (§A.2.2)
+    for key, mode, what in (("state_map", B.SS_COEF_STATE, "the exact least-squares map"),
+                            ("lrd_map", B.SS_COEF_LRD, "the low-rank-plus-diagonal map (4 pivots)")):
+        try:
+            import numpy as np  # noqa: F401
+            skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
+            sl = []
+            for _ in range(2):
+                lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev,
+                                  coef_mode=mode, coef_ridge=0.01)
+                lay.state.copy_(layers[0].state)
+                lay.basis.copy_(layers[0].basis)
+                lay.A.copy_(layers[0].A)
+                lay.prime()
+                sl.append(lay)
+            ts, fs = [], []
+            for k in range(3):
+                a, f0, b = ev(), ev(), ev()
+                a.record(stream)
+                for p in range(W):
+                    if p == W - 1:
+                        f0.record(stream)
+                    for l, lay in enumerate(sl):
+                        lay.step(toks[(p + l) % W])
+                b.record(stream)
+                torch.cuda.synchronize()
+                if k:
+                    ts.append(a.elapsed_time(b))
+                    fs.append(f0.elapsed_time(b))
+            ms = min(ts) / len(sl)
+            approx = sketch_vs_exact(sl, toks, W, torch)
+            out[key] = {"what": f"the same window with {what} (rho 0.01) built by every flush",
+                        "ms_per_window": ms, "flush_us": min(fs) / len(sl) * 1e3,
+                        "value": units * W / (ms / 1e3), "unit": "seq*heads/s",
+                        "approx_mean": approx["mean"], "approx_aggregate": approx["aggregate"]}
+            del sl
+            torch.cuda.empty_cache()
+        except Exception as e:             # noqa: BLE001
+            out[key] = {"error": repr(e)[:200]}
     return out
 
 
@@ -382,13 +390,14 @@ def run_ours(args, rank, world):
     if args.batch:
         wl = dataclasses.replace(wl, name=f"{wl.name}@batch{args.batch}", batch=args.batch)
     skd = B.SS_BF16 if args.sketch_dtype == "bf16" else B.SS_F32
-    smap = args.coef == "state"
+    smap = args.coef in ("state", "lrd")
     W, NL = wl.window, args.layers
     st = synth.static_inputs(wl)
     layers = []
     for _ in range(NL):
         lay = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, W, st.ranks, skd, device=dev,
-                          coef_mode=B.SS_COEF_STATE if smap else B.SS_COEF_FIXED, coef_ridge=args.ridge)
+                          coef_mode={"state": B.SS_COEF_STATE, "lrd": B.SS_COEF_LRD}.get(args.coef, B.SS_COEF_FIXED),
+                          coef_ridge=args.ridge)
         lay.load(st.state, st.basis, st.coef, st.A)
         layers.append(lay)
     st.state = None
@@ -567,7 +576,8 @@ def run_ours(args, rank, world):
         "config": {"workload": wl.name, "family": synth.FAMILY_NAMES[wl.family], "batch": wl.batch,
                    "heads": wl.heads, "dk": wl.dk, "dv": wl.dv, "window": W, "mean_rank": wl.mean_rank,
                    "layers": NL, "sketch": args.sketch_dtype, "inputs": "bf16 q/k/v, fp32 state",
-                   "coef": (f"state-dependent map, rho = {args.ridge}" if smap else "fixed C = P^T"),
+                   "coef": ({"state": f"state-dependent map, rho = {args.ridge}",
+                             "lrd": f"low-rank-plus-diagonal map, rho = {args.ridge}"}.get(args.coef, "fixed C = P^T")),
                    "step": f"one window of {W} tokens through {NL} independent layers",
                    "l2": f"inputs larger than L2: {NL} layers rotated, back-to-back launches",
                    "parallelism": f"replicas x{world}"},
@@ -787,10 +797,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-families", action="store_true",
                     help="skip the GDN / KDA kernel timings that follow the default Mamba-2 line")
-    ap.add_argument("--coef", default="fixed", choices=["fixed", "state"],
-                    help="coefficient map: the fixed C = P^T of the workloads, or the state-dependent "
-                         "least-squares map rebuilt by every flush")
-    ap.add_argument("--ridge", type=float, default=0.01, help="rho of the state-dependent map")
+    ap.add_argument("--coef", default="fixed", choices=["fixed", "state", "lrd"],
+                    help="coefficient map: the fixed C = P^T of the workloads, the state-dependent "
+                         "least-squares map rebuilt by every flush, or its low-rank-plus-diagonal form")
+    ap.add_argument("--ridge", type=float, default=0.01, help="rho of the state-dependent maps")
     ap.add_argument("--sweep", action="store_true",
                     help="the batch x window x rank sweep on the Mamba-2 shape (1 GPU), instead of the bench line")
     ap.add_argument("--sweep-batches", default="1,32,128,320,1024")

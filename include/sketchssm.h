@@ -48,7 +48,7 @@
  *   sketch     float or bf16 [B][R][dv]       row off_h + i is u_i = S^T omega_i of head h
  *   basis      float    [R][dk]               row off_h + i is omega_i of head h (shared by the batch)
  *   coef       float    [R][dk]               rows off_h .. off_h + r_h - 1 are head h's map C
- *   coef_state float or bf16 [B][R][dk]       SS_COEF_STATE: sequence b's map rows of head h at
+ *   coef_state float or bf16 [B][R][dk]       SS_COEF_STATE, SS_COEF_LRD: sequence b's map rows of head h at
  *                                             off_h .. off_h + r_h - 1 (dtype of the sketch)
  *   A          float    [H]                   Mamba-2 decay rates (A_h < 0 for decay)
  *   q, k       uint16_t [B][H][dk] bf16;  v uint16_t [B][H][dv] bf16
@@ -95,8 +95,8 @@ typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_sketch_dtype;
 /* Set by ss_step_mixed when a fill count lies outside 0..W-1: that sequence
  * is neither decoded nor flushed and its fill_out entry is left as it was. */
 #define SS_DEVICE_BAD_FILL 2
-/* Set by a flush in SS_COEF_STATE mode when a head's Gram matrix
- * U^T U + lambda I is not numerically positive definite (a Cholesky pivot
+/* Set by a flush in SS_COEF_STATE or SS_COEF_LRD mode when a head's Gram matrix
+ * (U^T U + lambda I, or P^T H P + lambda I) is not numerically positive definite (a Cholesky pivot
  * <= 0 or not finite, e.g. an all-zero state with rho = 0): that head's map
  * rows are written as zeros. */
 #define SS_DEVICE_SINGULAR_MAP 4
@@ -105,11 +105,22 @@ typedef enum { SS_F32 = 0, SS_BF16 = 1 } ss_sketch_dtype;
  * "Per step · Non-flush: Coefficient vector & readout"). */
 typedef enum {
     SS_COEF_FIXED = 0,       /* C = bufs->coef: one fp32 [R][dk] map shared by the batch */
-    SS_COEF_STATE = 1        /* per (sequence, head) map C = (U^T U + lambda I)^-1 U^T S^T,
+    SS_COEF_STATE = 1,       /* per (sequence, head) map C = (U^T U + lambda I)^-1 U^T S^T,
                               * lambda = rho tr(U^T U) / r (project page, "Per window ·
                               * Flush: Sketch & coefficient map"; paper §A.2.1), rebuilt
                               * by every flush from the new state and sketch, fused into
                               * it (no second state read); stored in bufs->coef_state */
+    SS_COEF_LRD = 2          /* per (sequence, head) map of the low-rank-plus-diagonal
+                              * state metric (paper §A.2.2): H = L L^T + D, L = the 4
+                              * output columns of the new state S with the largest
+                              * energy ||S[:, v]||^2 (the lower column on a tie), D =
+                              * the diagonal of the other columns' contribution;
+                              * C = (P^T H P + lambda I)^-1 P^T H with the head's basis
+                              * P, lambda = rho tr(P^T H P) / r.  Built, stored and read
+                              * like SS_COEF_STATE (same buffers and layout); needs
+                              * room for the pivots and the r x r Gram matrix in the
+                              * flush's tile buffer (ss_create returns
+                              * SS_ERR_UNSUPPORTED for a rank beyond it) */
 } ss_coef_mode;
 
 typedef struct {
@@ -122,7 +133,7 @@ typedef struct {
     const int32_t* ranks;    /* host [heads]: sketch rank r_h of each head; copied */
     int32_t sketch_dtype;    /* ss_sketch_dtype of the stored sketch U */
     int32_t coef_mode;       /* ss_coef_mode; 0 (zero-initialised) = SS_COEF_FIXED */
-    float coef_ridge;        /* rho >= 0 of SS_COEF_STATE (ignored otherwise) */
+    float coef_ridge;        /* rho >= 0 of SS_COEF_STATE and SS_COEF_LRD (else ignored) */
     const uint8_t* dense_heads; /* host [heads] or NULL; copied.  Nonzero: a dense-fallback head
                               * (paper App. D: at non-flush steps it reads a BF16 copy of its
                               * state).  Its rank must be dk; its dk sketch rows hold the
@@ -137,7 +148,7 @@ typedef struct ss_plan ss_plan;
 typedef struct {
     size_t state, ring_k, ring_v, ring_gate, ring_beta, sketch, basis, coef, A;
     size_t q, k, v, gate, beta, out;
-    size_t coef_state;       /* SS_COEF_STATE: [B][R][dk] in the sketch dtype; else 0 */
+    size_t coef_state;       /* SS_COEF_STATE, SS_COEF_LRD: [B][R][dk] in the sketch dtype; else 0 */
     int32_t total_rank;      /* R = sum of ranks */
     int32_t gate_stride;     /* Wg (scalar-gate families) or W * dk (KDA), floats per (b, h) */
 } ss_sizes;
@@ -153,7 +164,7 @@ typedef struct {
     const float* coef;       /* needed by ss_decode_step */
     const float* A;          /* needed for Mamba-2 */
     int32_t* status;         /* optional device int32 (4-byte aligned), see SS_DEVICE_TIMEOUT; NULL: no report */
-    void* coef_state;        /* SS_COEF_STATE only: device [B][R][dk] in the sketch dtype, the
+    void* coef_state;        /* SS_COEF_STATE and SS_COEF_LRD only: device [B][R][dk] in the sketch dtype, the
                               * per-(sequence, head) maps (head h's rows at the rank offset,
                               * like the sketch); written by ss_prime / ss_flush with a sketch,
                               * read by ss_decode_step; bufs->coef is then unused */
@@ -206,7 +217,9 @@ typedef struct {
  * with rank 128, dk = dv = 128 and W = 32 does not).  Every rank up to 64 at W <= 16,
  * and up to 32 at W <= 32, is supported.  SS_COEF_STATE needs every rank
  * <= dv (U^T U must be invertible) and a finite coef_ridge >= 0; its flushes
- * run on the CUDA-core flush kernel for every family.  The plan starts at
+ * run on the CUDA-core flush kernel for every family.  SS_COEF_LRD likewise,
+ * with every rank small enough for its scratch: up to 56 at dk = dv = 64,
+ * 64 at dk = 64, dv = 128, 81 at dk = 128, dv = 64 and 118 at dk = dv = 128.  The plan starts at
  * phase 0 with no valid sketch. */
 ss_status ss_create(const ss_config* cfg, ss_plan** out);
 ss_status ss_destroy(ss_plan* plan);

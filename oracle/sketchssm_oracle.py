@@ -51,7 +51,8 @@ Readings of points the pages leave open:
   The pages' cheaper variant (§A.2.2: the state metric approximated as low
   rank plus diagonal with P = 4 pivots) is read as keeping the n_piv output
   columns of S with the most energy exactly and the rest as a diagonal
-  (coefficient_map_lrd); no kernel builds it yet.
+  (coefficient_map_lrd); a session can refresh that map instead
+  (``map_kind="lrd"``).
 * P7 a bf16 sketch is the fp64 sketch rounded once to bf16 (nearest, ties
   to even).
 
@@ -198,8 +199,7 @@ def coefficient_map_lrd(S, P, n_piv=4, rho=0.0):
     with the largest energy ||S[:, v]||^2 (their correlations kept exactly)
     and D = diag of the remaining columns' contribution (their coordinate-wise
     energy).  C = (P^T H^ P + lambda I)^-1 P^T H^, lambda = rho tr(P^T H^ P) / r.
-    S [..., K, V], basis P [K, r] -> C [..., r, K].  Oracle only so far (no
-    kernel builds it yet)."""
+    S [..., K, V], basis P [K, r] -> C [..., r, K]."""
     S = np.asarray(S, dtype=np.float64)
     P = np.asarray(P, dtype=np.float64)
     K, V = S.shape[-2], S.shape[-1]
@@ -276,7 +276,7 @@ class Session:
     """
 
     def __init__(self, family, state, window, A=None, basis=None, coef=None,
-                 offsets=None, sketch_bf16=False, state_map=False, rho=0.0, dense=None):
+                 offsets=None, sketch_bf16=False, state_map=False, rho=0.0, dense=None, map_kind="exact"):
         self.family = family
         self.S = np.asarray(state, dtype=np.float64).copy()     # [B, H, K, V]
         self.B, self.H, self.K, self.V = self.S.shape
@@ -298,6 +298,7 @@ class Session:
             self.C[h] = np.eye(self.K)
         self.sketch_bf16 = sketch_bf16
         self.state_map, self.rho = state_map, rho
+        self.map_kind = map_kind   # "exact" (§A.2.1) or "lrd" (§A.2.2, coefficient_map_lrd)
         self.ring = []
         self.U = None
         self.Cs = None             # state-dependent maps, list over heads of [B, r_h, K]
@@ -323,8 +324,12 @@ class Session:
             U = [round_bf16(u) for u in U]
         self.U = U
         if self.state_map:
-            Cs = [None if self.dense[h] else coefficient_map(U[h], self.S[:, h], self.rho)
-                  for h in range(self.H)]
+            if self.map_kind == "lrd":
+                Cs = [None if self.dense[h] else coefficient_map_lrd(self.S[:, h], self.P[h], 4, self.rho)
+                      for h in range(self.H)]
+            else:
+                Cs = [None if self.dense[h] else coefficient_map(U[h], self.S[:, h], self.rho)
+                      for h in range(self.H)]
             self.Cs = [c if c is None or not self.sketch_bf16 else round_bf16(c) for c in Cs]
 
     def coef(self, h):

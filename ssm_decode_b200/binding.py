@@ -19,7 +19,7 @@ SS_OK, SS_ERR_INVALID_ARG, SS_ERR_ALIGNMENT, SS_ERR_UNSUPPORTED, SS_ERR_SCHEDULE
 SS_DEVICE_TIMEOUT = 1
 SS_DEVICE_BAD_FILL = 2
 SS_DEVICE_SINGULAR_MAP = 4
-SS_COEF_FIXED, SS_COEF_STATE = 0, 1
+SS_COEF_FIXED, SS_COEF_STATE, SS_COEF_LRD = 0, 1, 2
 SS_MAMBA2, SS_GDN, SS_KDA = 0, 1, 2
 SS_F32, SS_BF16 = 0, 1
 (SS_OP_DECODE, SS_OP_FLUSH, SS_OP_FLUSH_NO_TOKEN, SS_OP_PRIME, SS_OP_EXACT, SS_OP_REPLAY,

@@ -14,6 +14,7 @@ namespace ss {
 int flush_smem_bytes(int family, int dk, int dv, int n, int rpad, bool smap);
 int decode_smem_bytes(int family, int dk, int dv, int P, int rmax, int esz, bool smap, bool dense_any);
 bool flush_map_fits(int dk, int dv, int r);
+bool flush_lrd_fits(int dk, int dv, int r);
 }  // namespace ss
 
 struct ss_plan {
@@ -75,7 +76,7 @@ ss_status check_status(const ss_buffers* b) {
     return SS_OK;
 }
 
-bool state_map(const ss_plan* pl) { return pl->cfg.coef_mode == SS_COEF_STATE; }
+bool state_map(const ss_plan* pl) { return pl->cfg.coef_mode == SS_COEF_STATE || pl->cfg.coef_mode == SS_COEF_LRD; }
 
 // The map buffer a flush that refreshes the sketch must also refresh.
 ss_status check_map(const ss_plan* pl, const ss_buffers* b) {
@@ -132,6 +133,7 @@ ss::FlushParams flush_params(const ss_plan* pl, const ss_buffers* b, const ss_st
     if (state_map(pl) && b->sketch != nullptr) {
         p.cmap = b->coef_state;
         p.ridge = pl->cfg.coef_ridge;
+        p.lrd = pl->cfg.coef_mode == SS_COEF_LRD;
     }
     std::memcpy(p.dense, pl->dense, sizeof p.dense);
     std::memcpy(p.off, pl->off, sizeof(int32_t) * (pl->cfg.heads + 1));
@@ -198,9 +200,9 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
     if (c.sketch_dtype != SS_F32 && c.sketch_dtype != SS_BF16)
         return fail(SS_ERR_INVALID_ARG, "unknown sketch dtype %d", c.sketch_dtype);
     if (c.ranks == nullptr) return fail(SS_ERR_INVALID_ARG, "ranks is NULL");
-    if (c.coef_mode != SS_COEF_FIXED && c.coef_mode != SS_COEF_STATE)
+    if (c.coef_mode != SS_COEF_FIXED && c.coef_mode != SS_COEF_STATE && c.coef_mode != SS_COEF_LRD)
         return fail(SS_ERR_INVALID_ARG, "unknown coef_mode %d", c.coef_mode);
-    if (c.coef_mode == SS_COEF_STATE && !(c.coef_ridge >= 0.f && c.coef_ridge < 3.0e38f))
+    if (c.coef_mode != SS_COEF_FIXED && !(c.coef_ridge >= 0.f && c.coef_ridge < 3.0e38f))
         return fail(SS_ERR_INVALID_ARG, "coef_ridge must be finite and >= 0");
     if ((long long)c.batch * c.heads > (1ll << 31) / 2)
         return fail(SS_ERR_UNSUPPORTED, "batch * heads too large");
@@ -235,6 +237,11 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
             return fail(SS_ERR_UNSUPPORTED, "ranks[%d] = %d: the state-dependent map needs rank <= dv and "
                         "room for U and its Gram matrix in the flush's tile buffer", h, r);
         }
+        if (c.coef_mode == SS_COEF_LRD && !ss::flush_lrd_fits(c.dk, c.dv, r)) {
+            delete pl;
+            return fail(SS_ERR_UNSUPPORTED, "ranks[%d] = %d: the low-rank-plus-diagonal map needs room for "
+                        "its pivots, diagonal and Gram matrix in the flush's tile buffer", h, r);
+        }
         pl->ranks[h] = r;
         pl->off[h + 1] = pl->off[h] + r;
         if (r > pl->rmax) pl->rmax = r;
@@ -243,7 +250,7 @@ ss_status ss_create(const ss_config* cfg, ss_plan** out) {
     pl->Wg = (c.window + 3) & ~3;
     // Every launch must fit one head (flush) or one warp (decode) in shared memory.
     const int rpad = (pl->rmax + 1 + 3) & ~3;
-    const bool smap = c.coef_mode == SS_COEF_STATE;
+    const bool smap = c.coef_mode != SS_COEF_FIXED;
     const int fl = ss::flush_smem_bytes(c.family, c.dk, c.dv, c.window, rpad, smap);
     const int dec = ss::decode_smem_bytes(c.family, c.dk, c.dv, c.window - 1, pl->rmax, esize(pl), smap,
                                           pl->n_dense > 0);
@@ -524,14 +531,14 @@ ss_status ss_traffic_bytes(const ss_plan* pl, int32_t op, int32_t tau, ss_traffi
     double rd = 0, wr = 0, prd = 0, pwr = 0;
     const double bh = B * H;
     const double sketch_bytes = B * R * V * sk;          // U of every sequence
-    const bool smap = c.coef_mode == SS_COEF_STATE;
+    const bool smap = c.coef_mode != SS_COEF_FIXED;
     // Dense-fallback heads: their dk sketch rows are the state copy; no
     // basis, coef or map rows of theirs are read, and each flush that
     // sketches reads their new state once more to write the copy.
     const double nd = pl->n_dense, Rs = R - nd * K;      // ranks of the sketched heads
     const double basis_s = Rs * K * 4;                   // basis / fixed map rows actually read
     const double copy_rd = B * nd * D;
-    const double map_bytes = smap ? B * Rs * K * sk : 0; // per-sequence maps (SS_COEF_STATE)
+    const double map_bytes = smap ? B * Rs * K * sk : 0; // per-sequence maps (state-dependent modes)
     const double paper_tg = B * Rs * (K + V) * 2 + (m2 ? 0 : B * Rs * W * 2) + B * nd * K * V * 2;
     switch (op) {
         case SS_OP_DECODE:

@@ -312,6 +312,167 @@ __host__ __device__ inline bool map_fits(int K, int V, int r) {
     return r <= V && free_floats >= (V / 16) * K && free_floats >= r * r;
 }
 
+// The low-rank-plus-diagonal map's scratch in the tile buffer (floats):
+// column energies (V), the pivots (4 ints, padded to 16), the pivot columns
+// L (4 x dk), the diagonal d (dk), per-warp partials of d ((dv/16) x dk),
+// P^T L (r x 4), then the Gram matrix (r x r).
+constexpr int LRD_PIV = 4;
+__host__ __device__ inline int lrd_g_offset(int K, int V, int r) {
+    return V + 16 + LRD_PIV * K + K + (V / 16) * K + LRD_PIV * r;
+}
+__host__ __device__ inline bool lrd_map_fits(int K, int V, int r) {
+    return r <= K && lrd_g_offset(K, V, r) + r * r <= K * V;
+}
+
+// The low-rank-plus-diagonal map's Z and Gram matrix (paper §A.2.2, read as
+// in the oracle's coefficient_map_lrd): the state metric H = S S^T is replaced
+// by H^ = L L^T + diag(d), L = the LRD_PIV output columns of S with the most
+// energy ||S[:, v]||^2 (ties to the lower column), d[k] = the energy of row k
+// in the other columns.  With P the head's basis (rows in the extended-basis
+// buffer, as P^T):
+//     Z = P^T H^ = (P^T L) L^T + P^T diag(d)       (r x dk, in place over P^T)
+//     G = P^T H^ P = (P^T L)(P^T L)^T + P^T diag(d) P
+// from the updated state (this thread's R x 4 tile in `st`), with no pass over
+// HBM.  Returns G's address in the tile buffer.
+template <int K, int V>
+__device__ __forceinline__ float* lrd_metric(const FlushParams& p, const float2 (&st)[K / 8][2], int r,
+                                             unsigned char* smem, const FlushLayout& L, int t) {
+    using S = FS<K, V>;
+    constexpr int T = S::T, R = S::R, NW = T / 32;
+    const int lane = t & 31, warp = t >> 5;
+    const int cgw = lane & 3, rb = lane >> 2;
+    const int c0 = warp * 16 + cgw * 4, row0 = rb * R;
+    float* energy = reinterpret_cast<float*>(smem + L.tile);   // [V]
+    int* piv = reinterpret_cast<int*>(energy + V);             // [LRD_PIV]
+    float* lcol = energy + V + 16;                             // [LRD_PIV][K]
+    float* dg = lcol + LRD_PIV * K;                            // [K]
+    float* dpart = dg + K;                                     // [NW][K]
+    float* pl = dpart + NW * K;                                // [r][LRD_PIV]
+    float* g = energy + lrd_g_offset(K, V, r);                 // [r][r]
+    float* pt = reinterpret_cast<float*>(smem + L.pt);         // [r][K]: P^T, then Z
+    const auto elem = [&](int i, int c) { return (c & 1) ? st[i][c >> 1].y : st[i][c >> 1].x; };
+
+    // column energies: this thread's rows, then the sum over the row blocks
+    float en[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < R; i += 2) {
+            s0 = fmaf(elem(i, c), elem(i, c), s0);
+            s1 = fmaf(elem(i + 1, c), elem(i + 1, c), s1);
+        }
+        float x = s0 + s1;
+        x += __shfl_xor_sync(FULL, x, 4);
+        x += __shfl_xor_sync(FULL, x, 8);
+        x += __shfl_xor_sync(FULL, x, 16);
+        en[c] = x;
+    }
+    if (rb == 0) *reinterpret_cast<float4*>(energy + c0) = make_float4(en[0], en[1], en[2], en[3]);
+    __syncthreads();
+    // the pivots: LRD_PIV rounds of a warp arg-max (the lower column on ties)
+    if (warp == 0) {
+        float ev[V / 32];
+#pragma unroll
+        for (int j = 0; j < V / 32; ++j) ev[j] = energy[lane + 32 * j];
+        for (int q = 0; q < LRD_PIV; ++q) {
+            float bv = -INFINITY;
+            int bi = V;
+#pragma unroll
+            for (int j = 0; j < V / 32; ++j)
+                if (ev[j] > bv) { bv = ev[j]; bi = lane + 32 * j; }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) {
+                const float ov = __shfl_xor_sync(FULL, bv, m);
+                const int oi = __shfl_xor_sync(FULL, bi, m);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if (lane == 0) piv[q] = bi;
+#pragma unroll
+            for (int j = 0; j < V / 32; ++j)
+                if (lane + 32 * j == bi) ev[j] = -INFINITY;
+        }
+    }
+    __syncthreads();
+    int pv[LRD_PIV];
+#pragma unroll
+    for (int q = 0; q < LRD_PIV; ++q) pv[q] = piv[q];
+    // L (the pivot columns) and this warp's part of d (the other columns' energy per row)
+    float dr[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) dr[i] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        int q = -1;
+#pragma unroll
+        for (int qq = 0; qq < LRD_PIV; ++qq)
+            if (pv[qq] == c0 + c) q = qq;
+        if (q >= 0) {
+#pragma unroll
+            for (int i = 0; i < R; ++i) lcol[q * K + row0 + i] = elem(i, c);
+        } else {
+#pragma unroll
+            for (int i = 0; i < R; ++i) dr[i] = fmaf(elem(i, c), elem(i, c), dr[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        dr[i] += __shfl_xor_sync(FULL, dr[i], 1);
+        dr[i] += __shfl_xor_sync(FULL, dr[i], 2);
+    }
+    if (cgw == 0) {
+#pragma unroll
+        for (int i = 0; i < R; ++i) dpart[warp * K + row0 + i] = dr[i];
+    }
+    __syncthreads();
+    for (int k = t; k < K; k += T) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) s += dpart[w * K + k];
+        dg[k] = s;
+    }
+    // P^T L
+    for (int idx = t; idx < r * LRD_PIV; idx += T) {
+        const int e = idx / LRD_PIV, q = idx - e * LRD_PIV;
+        const float* pe = pt + e * K;
+        const float* lq = lcol + q * K;
+        float s0 = 0.f, s1 = 0.f;
+        for (int k = 0; k < K; k += 2) {
+            s0 = fmaf(pe[k], lq[k], s0);
+            s1 = fmaf(pe[k + 1], lq[k + 1], s1);
+        }
+        pl[idx] = s0 + s1;
+    }
+    __syncthreads();
+    // G = (P^T L)(P^T L)^T + P^T diag(d) P
+    for (int idx = t; idx < r * r; idx += T) {
+        const int e = idx / r, f = idx - e * r;
+        if (f > e) continue;
+        const float* pe = pt + e * K;
+        const float* pf = pt + f * K;
+        float s0 = 0.f, s1 = 0.f;
+        for (int k = 0; k < K; k += 2) {
+            s0 = fmaf(pe[k] * dg[k], pf[k], s0);
+            s1 = fmaf(pe[k + 1] * dg[k + 1], pf[k + 1], s1);
+        }
+        float s = s0 + s1;
+#pragma unroll
+        for (int q = 0; q < LRD_PIV; ++q) s = fmaf(pl[e * LRD_PIV + q], pl[f * LRD_PIV + q], s);
+        g[e * r + f] = s;
+        g[f * r + e] = s;
+    }
+    __syncthreads();
+    // Z = (P^T L) L^T + P^T diag(d), in place over P^T
+    for (int idx = t; idx < r * K; idx += T) {
+        const int e = idx / K, k = idx - e * K;
+        float z = pt[idx] * dg[k];
+#pragma unroll
+        for (int q = 0; q < LRD_PIV; ++q) z = fmaf(pl[e * LRD_PIV + q], lcol[q * K + k], z);
+        pt[idx] = z;
+    }
+    return g;
+}
+
 // State-dependent coefficient map of one head (project page, "Per window ·
 // Flush: Sketch & coefficient map"; paper §A.2.1):
 //     C = (U^T U + lambda I)^-1 U^T S^T,  lambda = ridge * tr(U^T U) / r,
@@ -341,10 +502,14 @@ __device__ __forceinline__ void build_map(const FlushParams& p, const float2 (&s
     constexpr int US = umap_stride(V);
     float* umap = reinterpret_cast<float*>(smem + L.tile);     // [r][US]
     float* zp = umap + r * US;                                 // [EC][NW][K], then G [r][r]
-    float* zs = reinterpret_cast<float*>(smem + L.pt);         // [r][K]: Z, then C
+    float* zs = reinterpret_cast<float*>(smem + L.pt);         // [r][K]: P, then Z, then C
     __shared__ int map_ok;
-    const int EC = min(r, (K * V - r * US) / (NW * K));
     __syncthreads();                                           // (D) U written, basis rows read
+    float* g = zp;
+    if (p.lrd) {
+        g = lrd_metric<K, V>(p, st, r, smem, L, t);
+    } else {
+    const int EC = min(r, (K * V - r * US) / (NW * K));
 
     // 1. Z = U^T S^T
     for (int e0 = 0; e0 < r; e0 += EC) {
@@ -397,8 +562,7 @@ __device__ __forceinline__ void build_map(const FlushParams& p, const float2 (&s
         __syncthreads();
     }
 
-    // 2. M = U^T U + lambda I, inverted in place by warp 0
-    float* g = zp;
+    // 2. M = U^T U
     for (int idx = t; idx < r * r; idx += T) {
         const int e = idx / r, f = idx - e * r;
         if (f > e) continue;
@@ -418,6 +582,8 @@ __device__ __forceinline__ void build_map(const FlushParams& p, const float2 (&s
         g[e * r + f] = sum;
         g[f * r + e] = sum;
     }
+    }
+    // M + lambda I, inverted in place by warp 0
     __syncthreads();
     if (warp == 0) {
         float tr = 0.f;
@@ -814,7 +980,7 @@ cudaError_t flush_launch(const FlushParams& p, int rmax, cudaStream_t stream) {
     const int rpad = ((p.do_sketch ? rmax : 0) + p.has_token + 3) & ~3;
     const int bytes = flush_layout(FAM, K, V, n, rpad).total;
     if (bytes > SMEM_LIMIT) return cudaErrorInvalidConfiguration;
-    if (MAP && !map_fits(K, V, rmax)) return cudaErrorInvalidConfiguration;
+    if (MAP && !(p.lrd ? lrd_map_fits(K, V, rmax) : map_fits(K, V, rmax))) return cudaErrorInvalidConfiguration;
     auto kern = flush_kernel<FAM, K, V, MIXED, MAP>;
     static KernelCache kc;
     cudaError_t e = ensure_smem(kern, kc, bytes);
@@ -852,6 +1018,7 @@ cudaError_t launch_flush(int family, int dk, int dv, const FlushParams& p, int r
 }
 
 bool flush_map_fits(int dk, int dv, int r) { return map_fits(dk, dv, r); }
+bool flush_lrd_fits(int dk, int dv, int r) { return lrd_map_fits(dk, dv, r); }
 
 namespace {
 

@@ -41,6 +41,9 @@ struct FlushParams {
     // for every head it sketches, as [B][R][dk] in the sketch dtype.
     void* cmap;
     float ridge;
+    // SS_COEF_LRD: the map of the low-rank-plus-diagonal state metric instead,
+    // C = (P^T H P + lambda I)^-1 P^T H with H = L L^T + D (see build_map).
+    int lrd;
     // Dense-fallback heads (bit h): the sketch rows of head h hold a copy of
     // its state, row k = S[k][:], in the sketch dtype, written by the flush
     // instead of S^T Omega; no basis rows are read for them.

@@ -56,9 +56,9 @@ class DecodeLayer:
         self.sketch = torch.zeros((batch, max(self.R, 1), dv), dtype=sk_dtype, device=device)
         self.basis = z(max(self.R, 1), dk)
         self.coef = z(max(self.R, 1), dk)
-        # per-(sequence, head) coefficient maps of SS_COEF_STATE, sketch dtype
+        # per-(sequence, head) coefficient maps of SS_COEF_STATE / SS_COEF_LRD, sketch dtype
         self.coef_state = (torch.zeros((batch, max(self.R, 1), dk), dtype=sk_dtype, device=device)
-                           if coef_mode == B.SS_COEF_STATE else None)
+                           if coef_mode in (B.SS_COEF_STATE, B.SS_COEF_LRD) else None)
         self.A = z(heads)
         self.out = z(batch, heads, dv)
         self.status = torch.zeros(4, dtype=torch.int32, device=device)   # device status word (+ padding)

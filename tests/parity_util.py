@@ -59,21 +59,23 @@ class Pair:
     compare sampled sequences); the GPU always runs the whole batch.
     """
 
-    def __init__(self, wl, st=None, sketch_dtype=B.SS_F32, sel=None, state_map=False, rho=0.0, dense=None):
+    def __init__(self, wl, st=None, sketch_dtype=B.SS_F32, sel=None, state_map=False, rho=0.0, dense=None,
+                 map_kind="exact"):
         import torch
         self.wl = wl
         self.st = st if st is not None else synth.static_inputs(wl)
         self.sel = np.arange(wl.batch) if sel is None else np.asarray(sel)
-        self.state_map = state_map
+        self.state_map, self.map_kind = state_map, map_kind
+        mode = (B.SS_COEF_LRD if map_kind == "lrd" else B.SS_COEF_STATE) if state_map else B.SS_COEF_FIXED
         self.layer = DecodeLayer(wl.family, wl.batch, wl.heads, wl.dk, wl.dv, wl.window,
                                  self.st.ranks, sketch_dtype,
-                                 coef_mode=B.SS_COEF_STATE if state_map else B.SS_COEF_FIXED,
+                                 coef_mode=mode,
                                  coef_ridge=rho, dense_heads=dense)
         self.layer.load(self.st.state, self.st.basis, self.st.coef, self.st.A)
         self.sess = orc.Session(wl.family, self.st.state[self.sel], wl.window, self.st.A,
                                 self.st.basis, self.st.coef, self.st.offsets,
                                 sketch_bf16=sketch_dtype == B.SS_BF16, state_map=state_map, rho=rho,
-                                dense=dense)
+                                dense=dense, map_kind=map_kind)
         self.bf16 = sketch_dtype == B.SS_BF16
         self.ring_k = np.zeros((wl.batch, wl.heads, wl.window, wl.dk), np.uint16)
         self.ring_v = np.zeros((wl.batch, wl.heads, wl.window, wl.dv), np.uint16)
@@ -124,7 +126,9 @@ class Pair:
         if not self.state_map:
             return
         g = to_np(self.layer.coef_state)[self.sel]
-        if self.bf16:
+        if self.bf16 and self.map_kind == "lrd":
+            ref = self.sess.packed_map()     # a function of the state alone: the oracle's, rounded
+        elif self.bf16:
             Ug = self.gpu_sketch_heads()
             ref = np.concatenate([np.zeros((len(self.sel), self.wl.dk, self.wl.dk)) if self.sess.dense[h] else
                                   orc.round_bf16(orc.coefficient_map(Ug[h], self.sess.S[:, h], self.sess.rho))

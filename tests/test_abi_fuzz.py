@@ -45,14 +45,20 @@ def _map_fits(K, V, r):
     return r <= V and free >= (V // 16) * K and free >= r * r
 
 
+def _lrd_fits(K, V, r):
+    """The low-rank-plus-diagonal map's scratch: energies, pivots, 4 pivot
+    columns, the diagonal, per-warp partials, P^T L and the Gram matrix."""
+    return r <= K and V + 16 + 4 * K + K + (V // 16) * K + 4 * r + r * r <= K * V
+
+
 def _breaks_a_rule(family, batch, heads, dk, dv, window, ranks, dtype, coef_mode, ridge, dense):
     if family not in (0, 1, 2) or batch < 1 or not 1 <= heads <= 512:
         return True
     if dk not in (64, 128) or dv not in (64, 128) or not 1 <= window <= 32:
         return True
-    if dtype not in (0, 1) or coef_mode not in (0, 1):
+    if dtype not in (0, 1) or coef_mode not in (0, 1, 2):
         return True
-    if coef_mode == 1 and not (ridge >= 0 and ridge < 3.0e38):
+    if coef_mode in (1, 2) and not (ridge >= 0 and ridge < 3.0e38):
         return True
     if batch * heads > 2 ** 30:
         return True
@@ -62,6 +68,8 @@ def _breaks_a_rule(family, batch, heads, dk, dv, window, ranks, dtype, coef_mode
         if not 0 <= r <= dk or (d and r != dk):
             return True
         if coef_mode == 1 and not d and not _map_fits(dk, dv, r):
+            return True
+        if coef_mode == 2 and not d and not _lrd_fits(dk, dv, r):
             return True
     return False
 
@@ -79,7 +87,7 @@ configs = st.fixed_dictionaries({
     "dv": st.sampled_from([64, 128]),
     "window": st.integers(1, 32),
     "dtype": st.sampled_from([0, 1]),
-    "coef_mode": st.sampled_from([0, 0, 1]),
+    "coef_mode": st.sampled_from([0, 0, 1, 2]),
     "ridge": st.sampled_from([0.0, 0.01, 1.0]),
     "seed": st.integers(0, 2 ** 32 - 1),
     "with_dense": st.booleans(),
@@ -89,7 +97,7 @@ configs = st.fixed_dictionaries({
 })
 
 _BAD = {"family": [3, -1], "batch": [0, -3], "heads": [0, 513], "dk": [32, 256], "dv": [96, 32],
-        "window": [0, 33], "dtype": [2, -1], "coef_mode": [2, -1]}
+        "window": [0, 33], "dtype": [2, -1], "coef_mode": [3, -1]}
 
 
 @settings(max_examples=400, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
@@ -104,7 +112,7 @@ def test_random_configs(L, c):
     if brk == "batch_heads":
         c["heads"], c["batch"] = 512, (1 << 21) + 1               # batch * heads just above 2^30
     if brk == "ridge":
-        c["coef_mode"], c["ridge"] = 1, rnd.choice([-1.0, float("inf"), float("nan")])
+        c["coef_mode"], c["ridge"] = rnd.choice([1, 2]), rnd.choice([-1.0, float("inf"), float("nan")])
     heads, dk = c["heads"], c["dk"]
     n = max(heads, 1)
     hi = dk if dk in (64, 128) else 128
@@ -157,7 +165,7 @@ def test_random_configs(L, c):
         assert s.gate == (Bt * H * K if fam == B.SS_KDA else Bt * H) * 4
         assert s.beta == (0 if fam == B.SS_MAMBA2 else Bt * H * 4)
         assert s.out == Bt * H * V * 4
-        assert s.coef_state == (Bt * R * K * esz if c["coef_mode"] == B.SS_COEF_STATE else 0)
+        assert s.coef_state == (Bt * R * K * esz if c["coef_mode"] in (B.SS_COEF_STATE, B.SS_COEF_LRD) else 0)
         assert s.gate_stride == (W * K if fam == B.SS_KDA else Wg)
         # traffic: defined for every phase the schedule allows, linear in the phase
         t = B.ss_traffic()

@@ -174,6 +174,28 @@ def test_state_map_config_sizes_and_traffic(L):
         B.Plan(B.SS_MAMBA2, 1, 1, K, V, 16, [min(K, V) // 2], B.SS_BF16, B.SS_COEF_STATE)
 
 
+def test_lrd_map_config_sizes_and_limits(L):
+    """SS_COEF_LRD: the same map buffer and bytes as SS_COEF_STATE; its rank
+    limit comes from its own scratch (pivots, diagonal, Gram matrix)."""
+    lrd = B.Plan(B.SS_GDN, 3, 2, 128, 64, 6, [5, 7], B.SS_BF16, B.SS_COEF_LRD, 0.25)
+    st = B.Plan(B.SS_GDN, 3, 2, 128, 64, 6, [5, 7], B.SS_BF16, B.SS_COEF_STATE, 0.25)
+    assert B.ss_buffer_sizes(lrd)["coef_state"] == B.ss_buffer_sizes(st)["coef_state"] == 3 * 12 * 128 * 2
+    for op in (B.SS_OP_DECODE, B.SS_OP_FLUSH):
+        assert B.ss_traffic_bytes(lrd, op, 2 if op == B.SS_OP_DECODE else 0) == \
+            B.ss_traffic_bytes(st, op, 2 if op == B.SS_OP_DECODE else 0)
+    for ridge in (-1.0, float("nan"), float("inf")):
+        with pytest.raises(B.SSError) as e:
+            B.Plan(B.SS_GDN, 1, 1, 64, 64, 4, [4], B.SS_F32, B.SS_COEF_LRD, ridge)
+        assert e.value.status == B.SS_ERR_INVALID_ARG
+    # largest ranks per shape: 56 (64 x 64), 64 (64 x 128), 81 (128 x 64), 118 (128 x 128)
+    for (K, V), rmax in {(64, 64): 56, (64, 128): 64, (128, 64): 81, (128, 128): 118}.items():
+        B.Plan(B.SS_KDA, 1, 1, K, V, 8, [rmax], B.SS_F32, B.SS_COEF_LRD)
+        if rmax < K:
+            with pytest.raises(B.SSError) as e:
+                B.Plan(B.SS_KDA, 1, 1, K, V, 8, [rmax + 1], B.SS_F32, B.SS_COEF_LRD)
+            assert e.value.status == B.SS_ERR_UNSUPPORTED
+
+
 def test_dense_heads_config_and_traffic(L):
     """Dense-fallback heads: rank dk, their state copy in the sketch rows."""
     with pytest.raises(B.SSError) as e:

@@ -163,3 +163,61 @@ def test_state_map_mixed_positions(cuda_ok, family):
         fill = (fill + 1) % W
         fin, fout = fout, fin
     assert int(layer.status[0].item()) == 0
+
+
+# ---------------------------------------------------------------------------
+# SS_COEF_LRD: the map of the low-rank-plus-diagonal state metric (paper
+# §A.2.2, read as in oracle.coefficient_map_lrd: the 4 output columns of S with
+# the most energy kept exactly, the rest as a diagonal).  The pivots are a
+# ranking of column energies computed in fp32 on the GPU and fp64 in the
+# oracle; on these random states the 4th and 5th energies are never close
+# enough for the two to rank them differently.
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (128, 64), (64, 128), (64, 64)])
+def test_lrd_map_families_and_shapes(cuda_ok, family, dk, dv):
+    wl = small(FAM[family], dk, dv, seed=3000 + dk + dv)
+    w = run(Pair(wl, state_map=True, rho=RHO, map_kind="lrd"), 20)
+    assert w["map"] <= TOL and w["sketched"] <= TOL
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+def test_lrd_map_unregularized_and_bf16(cuda_ok, family):
+    """rho = 0 (the diagonal keeps P^T H P positive definite) with a bf16
+    sketch and map, over a flush."""
+    wl = small(FAM[family], 128, 128, seed=3100)
+    run(Pair(wl, sketch_dtype=B.SS_BF16, state_map=True, rho=0.0, map_kind="lrd"), wl.window + 3)
+
+
+@pytest.mark.parametrize("family", ["mamba2", "gdn", "kda"])
+def test_lrd_map_ragged_ranks_with_zero_and_one(cuda_ok, family):
+    wl = small(FAM[family], 128, 64, heads=4, seed=3200)
+    st = synth.static_inputs(wl)
+    ranks = np.array([0, 1, 16, 7], np.int32)
+    offs = np.concatenate([[0], np.cumsum(ranks)]).astype(np.int32)
+    rng = np.random.default_rng(32)
+    basis = np.concatenate([np.linalg.qr(rng.standard_normal((wl.dk, wl.dk)))[0][:, :r].T
+                            for r in ranks]).astype(np.float32)
+    st.ranks, st.offsets, st.basis, st.coef = ranks, offs, basis, basis.copy()
+    run(Pair(wl, st=st, state_map=True, rho=RHO, map_kind="lrd"), 18)
+
+
+def test_lrd_map_of_zero_state_is_singular(cuda_ok):
+    """An all-zero state: every energy ties at zero (the pivots are the first
+    columns), L = 0 and d = 0, so P^T H P = 0: flagged, and a zero map."""
+    wl = small(synth.KDA, 128, 128, batch=2, heads=3, window=4, seed=3300)
+    st = synth.static_inputs(wl)
+    st.state = np.zeros_like(st.state)
+    p = Pair(wl, st=st, state_map=True, map_kind="lrd")
+    p.prime()
+    assert int(p.layer.status[0].item()) & B.SS_DEVICE_SINGULAR_MAP
+    assert not to_np(p.layer.coef_state).any()
+    p.layer.status.zero_()
+
+
+def test_lrd_map_full_size_sampled(cuda_ok):
+    """GDN batch 256 x 32 heads in LRD mode, one window plus a flush, three
+    sampled sequences."""
+    wl = synth.WORKLOADS["gdn_b256"]
+    p = Pair(wl, sketch_dtype=B.SS_BF16, sel=[0, wl.batch // 2, wl.batch - 1], state_map=True, rho=RHO,
+             map_kind="lrd")
+    run(p, wl.window + 1)
