@@ -42,15 +42,29 @@ def test_clock_summary_without_samples_is_none(tmp_path):
 
 
 def test_traffic_record_only_for_current_sources_and_workload(monkeypatch):
+    """Records are keyed kernel@workload: each workload gets its own kernel's
+    record, and only while the device-code hash matches."""
     with open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")) as f:
         rec = json.load(f)
-    name = next(k for k, v in rec.items() if isinstance(v, dict) and "source_sha" in v)
-    r = rec[name]
+    recs = {k: v for k, v in rec.items() if isinstance(v, dict) and "source_sha" in v}
+    assert recs and all(k == f"{v['kernel']}@{v['workload']}" for k, v in recs.items())
+    r = next(iter(recs.values()))
     monkeypatch.setattr(bench, "kernel_source_sha", lambda: r["source_sha"])
-    assert bench.kernel_traffic_record(name, r["workload"]) == r
+    for v in recs.values():
+        assert bench.kernel_traffic_record(v["kernel"], v["workload"]) == v
+    name = r["kernel"]
     assert bench.kernel_traffic_record(name, r["workload"] + "_other") is None
     assert bench.kernel_traffic_record(name, r["workload"], coef="state") is None
     assert bench.kernel_traffic_record("no_such_kernel", r["workload"]) is None
+    # the same kernel on two workloads: two different records
+    by_kernel = {}
+    for v in recs.values():
+        by_kernel.setdefault(v["kernel"], []).append(v)
+    for vs in by_kernel.values():
+        if len(vs) > 1:
+            a, b = vs[0], vs[1]
+            assert bench.kernel_traffic_record(a["kernel"], a["workload"])["dram_bytes_per_launch"] != \
+                bench.kernel_traffic_record(b["kernel"], b["workload"])["dram_bytes_per_launch"]
     monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)
     assert bench.kernel_traffic_record(name, r["workload"]) is None
 
