@@ -28,16 +28,19 @@
 //     S_W^T x = S_0^T (g ⊙ x) + sum_j w~_j (k^_j . x),
 // and for KDA k^_j . x = (k_j / G(j,-1)) . (g ⊙ x).
 //
-// Tensor-core products per head (tf32 operands, fp32 accumulators in TMEM):
-//     Gm = [keys | probes] K'^T     M = 128 rows of the pass's B buffer, N = 16
-//          (GDN K' = the keys; KDA K' = k_j / G(j,-1), hi and lo: N = 32) --
-//          the pair weights and k^_j . x, for the recursion and the read-out
+// Tensor-core products per head (fp32 accumulators in TMEM):
+//     Gm = [keys | probes] K'^T     M = 128, N = 16 (GDN) or 32 (KDA) --
+//          the pair weights and k^_j . x, for the recursion and the read-out.
+//          GDN in bf16: K' = the keys (exact in bf16), each probe in three
+//          bf16 parts that sum to it exactly, K = 16 an instruction.  KDA in
+//          tf32: K' = k_j / G(j,-1), hi and lo, against the pass's B rows
 //     D  = S_0^T [keys | probes | their lo halves]   M = dv, N <= 96, K = dk
 //     Dc = W~^T (K^ X^T)                              M = dv, N = 16 or 32, K = 16
 //     C += W~^T K^   (C = Diag(g) S_0 before)         M = dv, N = dk, K = 16
 // D, Dc and C have lane v = state column v; C ends as S_W^T.  An instruction
-// costs about as much at N = 16 as at N = 128 (it is bound by reading its
-// 128 x 8 slice of A), so products that share an A operand are packed along N.
+// costs about as much at N = 16 as at N = 128 (about 82 cycles with A in
+// TMEM, 93 with A in shared memory, measured at M = 128), so products that
+// share an A operand are packed along N.
 // fp32 accuracy from tf32 operands: each fp32 operand is split x = hi + lo,
 // hi = x with the low 13 mantissa bits cleared (the tensor core takes a tf32
 // operand from fp32 by this truncation, so a raw fp32 value serves as its own
@@ -56,11 +59,11 @@
 // issuer waits for those before Gm, the pass and the correction and update;
 // MMA groups complete on mbarriers the workers wait for.  The mover issues a
 // head's window once phase 1 of the previous head has read the window buffers
-// (fetching the scalars each copy needs a head ahead), splits nothing itself:
-// a head's tile is moved into TMEM by the workers early in the head; its
-// buffer then stages the previous head's S_W (read from C), which the mover
-// stores before it loads the next head's tile into the same buffer; the
-// read-out is staged in shared memory and stored the same way.  No worker
+// (fetching the scalars each copy needs a head ahead).  The workers move a
+// head's tile into TMEM early in the head; its buffer then stages the
+// previous head's S_W (read from C), which the mover stores before it loads
+// the next head's tile into the same buffer; the read-out is staged in shared
+// memory and stored the same way.  No worker
 // waits for the issuer, and no one for the tensor core's queue or for stores
 // to drain.  Every wait on an mbarrier is bounded: when one runs out the
 // kernel sets SS_DEVICE_TIMEOUT in the caller's status word, waits (bounded)
@@ -305,7 +308,7 @@ __global__ void __launch_bounds__(TT, 1) flush_tc_kernel(const __grid_constant__
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const bool ctl = warp == NWK / 32;                                // the issuing warp
     const bool mov = warp == NWK / 32 + 1;                            // the moving warp
-    const bool issuer = ctl && lane == 0;                             // window copies and MMAs
+    const bool issuer = ctl && lane == 0;                             // every MMA
     const bool mover = mov && lane == 0;                              // bulk copies in and out
     const int v = t & (TV - 1);                                       // a worker's state column
     const int hk = (t >> 7) & 1;                                      // which half of the dk rows
