@@ -437,6 +437,40 @@ def test_lrd_map_matches_a_direct_construction():
         assert relerr(C[i] @ q[i], c_ls) < 1e-8
 
 
+def test_lrd_map_of_a_state_on_few_columns_is_the_exact_map():
+    """A state whose energy sits in at most n_piv output columns: those columns
+    are the pivots, the rest is zero (D = 0), so H^ = H and the map is exact."""
+    S, P, U, q = _map_case(10, n=3, K=9, V=12, r=3)
+    S = S.copy()
+    S[0][:, [0, 1, 2, 4, 6, 7, 8, 9, 11]] = 0.0          # columns 3, 5, 10 remain
+    S[1][:, :-4] = 0.0                                     # the last four remain
+    S[2][:, 4:] = 0.0                                      # the first four remain,
+    S[2][:, 0] *= 50.0                                     # one of them dominant
+    U = orc.sketch(S, P)
+    for rho in (0.0, 0.1):
+        C = orc.coefficient_map_lrd(S, P, n_piv=4, rho=rho)
+        assert relerr(C, orc.coefficient_map(U, S, rho)) < 1e-10
+
+
+def test_lrd_map_ties_keep_the_lower_column():
+    """Equal energies rank the lower column first (the pages leave ties open;
+    this is the stable ranking the kernel shares): with one pivot and columns 1
+    and 3 tied for the largest energy, H^ = s1 s1^T + diag(s3^2 + rest)."""
+    rng = np.random.default_rng(11)
+    K, r = 6, 2
+    S = np.zeros((K, 5))
+    S[:, 1] = rng.standard_normal(K)
+    S[:, 3] = S[:, 1] * np.array([1, -1, 1, 1, -1, 1])    # same squares: an exact tie
+    S[:, 0] = 0.1 * rng.standard_normal(K)
+    P = np.linalg.qr(rng.standard_normal((K, K)))[0][:, :r]
+    H = np.outer(S[:, 1], S[:, 1]) + np.diag(S[:, 0] ** 2 + S[:, 3] ** 2)
+    want = np.linalg.solve(P.T @ H @ P, P.T @ H)
+    assert relerr(orc.coefficient_map_lrd(S, P, n_piv=1), want) < 1e-10
+    # the other choice is a different map: the pin can tell them apart
+    H3 = np.outer(S[:, 3], S[:, 3]) + np.diag(S[:, 0] ** 2 + S[:, 1] ** 2)
+    assert relerr(np.linalg.solve(P.T @ H3 @ P, P.T @ H3), want) > 1e-3
+
+
 @pytest.mark.parametrize("family", FAMS)
 def test_session_state_map_identity_basis_reads_exactly(family):
     """Session with the state map and P = I (r = K <= V): every sketched read
@@ -508,17 +542,54 @@ def _mut_lrd_no_diagonal(S, P, n_piv=4, rho=0.0):
     return ORIG_LRD(S * mask[..., None, :], P, n_piv, rho)
 
 
-def test_planted_lrd_mistake_is_caught(monkeypatch):
-    def run():
-        try:
-            test_lrd_map_of_isotropic_energy_is_the_fixed_map()
-            test_lrd_map_matches_a_direct_construction()
-        except AssertionError:
-            return False
-        return True
-    assert run()
-    monkeypatch.setattr(orc, "coefficient_map_lrd", _mut_lrd_no_diagonal)
-    assert not run(), "dropping the diagonal went unnoticed"
+def _lrd_variant(S, P, n_piv, rho, smallest=False, diag_all=False, ridge_of_h=False,
+                 ties_high=False):
+    """The low-rank-plus-diagonal map with one plausible mistake switched on."""
+    S = np.asarray(S, np.float64)
+    K, r = S.shape[-2], P.shape[-1]
+    e = np.einsum("...kv,...kv->...v", S, S)
+    key = e if smallest else -e
+    if ties_high:
+        order = S.shape[-1] - 1 - np.argsort(key[..., ::-1], axis=-1, kind="stable")
+    else:
+        order = np.argsort(key, axis=-1, kind="stable")
+    piv = order[..., :n_piv]
+    mask = np.zeros(e.shape, bool)
+    np.put_along_axis(mask, piv, True, axis=-1)
+    L = S * mask[..., None, :]
+    d = np.einsum("...kv,...kv->...k", S if diag_all else S * ~mask[..., None, :], S)
+    H = np.einsum("...kp,...jp->...kj", L, L) + d[..., :, None] * np.eye(K)
+    G = np.einsum("kr,...kj,js->...rs", P, H, P)
+    tr = np.trace(H if ridge_of_h else G, axis1=-2, axis2=-1)
+    A = G + (rho * tr / r)[..., None, None] * np.eye(r)
+    return np.linalg.solve(A, np.einsum("kr,...kj->...rj", P, H))
+
+
+def _run_lrd_pins():
+    try:
+        test_lrd_map_with_every_column_kept_is_the_exact_map()
+        test_lrd_map_of_isotropic_energy_is_the_fixed_map()
+        test_lrd_map_matches_a_direct_construction()
+        test_lrd_map_of_a_state_on_few_columns_is_the_exact_map()
+        test_lrd_map_ties_keep_the_lower_column()
+    except AssertionError:
+        return False
+    return True
+
+
+@pytest.mark.parametrize("mutant", [
+    _mut_lrd_no_diagonal,
+    lambda S, P, n_piv=4, rho=0.0: _lrd_variant(S, P, n_piv, rho, smallest=True),
+    lambda S, P, n_piv=4, rho=0.0: _lrd_variant(S, P, n_piv, rho, diag_all=True),
+    lambda S, P, n_piv=4, rho=0.0: _lrd_variant(S, P, n_piv, rho, ridge_of_h=True),
+    lambda S, P, n_piv=4, rho=0.0: _lrd_variant(S, P, n_piv, rho, ties_high=True),
+], ids=["no_diagonal", "smallest_pivots", "diagonal_of_all", "ridge_of_H", "ties_high"])
+def test_planted_lrd_mistakes_are_caught(monkeypatch, mutant):
+    assert _run_lrd_pins()
+    monkeypatch.setattr(orc, "coefficient_map_lrd", lambda S, P, n_piv=4, rho=0.0: _lrd_variant(S, P, n_piv, rho))
+    assert _run_lrd_pins(), "the mutant harness itself must pass unmutated"
+    monkeypatch.setattr(orc, "coefficient_map_lrd", mutant)
+    assert not _run_lrd_pins(), "a mistake planted in coefficient_map_lrd went unnoticed"
 
 
 def _mut_map_no_ridge(U, S, rho=0.0):
